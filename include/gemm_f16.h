@@ -1,0 +1,121 @@
+/*
+ * gemm_f16.h -- C ABI of libttc05: fp16 GEMM with a fused ReLU epilogue on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one of "Writing high-performance kernels in TileLang"
+ * (atlascloud.ai blog), section "Escribamos un GEMM": A (M x K) and B (K x N)
+ * are row-major fp16 matrices, the products are accumulated in fp32, the
+ * accumulator is clamped with max(x, 0), and the result is written to the
+ * row-major fp16 matrix C (M x N), rounding to nearest-even.  The page checks
+ * the kernel against relu(a @ b) with rtol = atol = 1e-2, and so do the tests
+ * of this library.
+ *
+ * Conventions shared by every entry point
+ *   - A, B, C are DEVICE pointers (cudaMalloc / torch CUDA memory) to IEEE
+ *     binary16 storage on the current CUDA device.  Host pointers are rejected
+ *     with GEMM_ERR_INVALID_ARG.
+ *   - lda, ldb, ldc are row strides in ELEMENTS (lda >= K, ldb >= N, ldc >= N).
+ *     Columns are contiguous.
+ *   - Pointers must be 16-byte aligned and every ld a multiple of 8 elements
+ *     (16 bytes): the tiles are moved by the Tensor Memory Accelerator, whose
+ *     global strides must be multiples of 16 bytes.  Otherwise
+ *     GEMM_ERR_ALIGNMENT.
+ *   - M, N, K are in [0, 2^31 - 1].  M == 0 or N == 0 is a no-op that returns
+ *     GEMM_OK.  K == 0 writes C = +0 (the empty sum; ReLU of it is +0 too).
+ *   - The caller owns A, B and C; the library keeps no reference to them after
+ *     the call.  C must not overlap A or B (undefined result).
+ *   - Calls are asynchronous and stream-ordered on `stream` (0 = legacy default
+ *     stream): the return value only reports argument and launch errors.
+ *     Errors found on the device (a bounded wait that ran out) are recorded in
+ *     a per-device status word, read with gemm_get_device_status().
+ *   - Results are deterministic: the same inputs give the same bits on every
+ *     run, whatever the scheduling.
+ *   - Small-M problems (M <= 64) use a stream-K path whose fp32 partial tiles
+ *     and arrival counters live in a workspace the library allocates once per
+ *     (device, stream) on first use (cudaMalloc; about 10 MB on a 148-SM GPU)
+ *     and keeps until process exit.  Make that first call outside CUDA-graph
+ *     capture.  Two calls on different streams never share a workspace.
+ *   - No entry point throws; errors are negative return codes.
+ */
+#ifndef TTC05_GEMM_F16_H
+#define TTC05_GEMM_F16_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GEMM_API __attribute__((visibility("default")))
+#else
+#define GEMM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without including the CUDA headers */
+typedef struct CUstream_st* gemm_stream_t;
+
+enum gemm_status {
+  GEMM_OK = 0,
+  GEMM_ERR_INVALID_ARG = -1,        /* negative size, ld < cols, null or host pointer, size too large */
+  GEMM_ERR_ALIGNMENT = -2,          /* pointer not 16-byte aligned or ld % 8 != 0 */
+  GEMM_ERR_UNSUPPORTED_DEVICE = -3, /* current device is not compute capability 10.0 */
+  GEMM_ERR_LAUNCH = -4,             /* a CUDA runtime call or kernel launch failed */
+  GEMM_ERR_WORKSPACE = -5,          /* workspace allocation failed */
+  GEMM_ERR_DEVICE_TIMEOUT = -6      /* reported by gemm_get_device_status */
+};
+
+enum gemm_path {
+  GEMM_PATH_AUTO = 0,   /* choose by shape: M <= 64 -> STREAMK, else TILE */
+  GEMM_PATH_TILE = 1,   /* persistent 128 x BN tile kernel (any shape) */
+  GEMM_PATH_STREAMK = 2 /* swap-AB stream-K kernel (M <= 64 only) */
+};
+
+/* C = ReLU(A @ B).  "Escribamos un GEMM": the tiled fp16 matmul with the
+ * max(x, 0) epilogue fused before the fp16 store.  Returns GEMM_OK or a
+ * negative gemm_status. */
+GEMM_API int gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N,
+                           int64_t K, int64_t lda, int64_t ldb, int64_t ldc, gemm_stream_t stream);
+
+/* C = A @ B, the same kernels without the activation (no bias). */
+GEMM_API int gemm_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+             int64_t lda, int64_t ldb, int64_t ldc, gemm_stream_t stream);
+
+/* Either of the above with an explicit kernel choice.  relu: 0 or 1.  path:
+ * a gemm_path value; GEMM_PATH_STREAMK with M > 64 returns
+ * GEMM_ERR_INVALID_ARG. */
+GEMM_API int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                int64_t lda, int64_t ldb, int64_t ldc, int relu, int path,
+                gemm_stream_t stream);
+
+/* The path GEMM_PATH_AUTO takes for this shape (GEMM_PATH_TILE or
+ * GEMM_PATH_STREAMK).  Pure host function. */
+GEMM_API int gemm_select_path(int64_t M, int64_t N, int64_t K);
+
+/* Human-readable text for a gemm_status value (static storage). */
+GEMM_API const char* gemm_status_string(int status);
+
+/* Synchronises `stream`, then reports and clears the status word of the
+ * current device: *device_status = 0 if every kernel finished normally, else
+ * the code of the first bounded wait that gave up (non-zero; the kernel that
+ * gave up returned without completing its output).  After a non-zero status
+ * the stream-K workspaces of the device are re-zeroed.  Returns GEMM_OK, or
+ * GEMM_ERR_LAUNCH if a CUDA call failed. */
+GEMM_API int gemm_get_device_status(gemm_stream_t stream, int* device_status);
+
+/* Failure-detection self test: launches one CTA that waits, with the same
+ * bounded wait as the GEMM kernels and a limit of `timeout_ns`, on an mbarrier
+ * nothing will ever arrive on.  The wait runs out, the kernel records a
+ * timeout in the status word and returns normally; the context stays usable.
+ * Synchronises `stream` and stores the status word (then clears it) in
+ * *device_status.  Returns GEMM_OK or a negative gemm_status. */
+GEMM_API int gemm_selftest_wait_timeout(int64_t timeout_ns, gemm_stream_t stream, int* device_status);
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+GEMM_API int gemm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTC05_GEMM_F16_H */

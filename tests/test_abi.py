@@ -1,0 +1,76 @@
+"""The C-ABI library loads and exports every entry point the header declares;
+host-only entry points behave as documented (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gemm_f16.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_tensor_core_05_b200 import build, ops
+    build.build()
+    return ops.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"GEMM_API\s+[\w\s\*]+?\b(gemm_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"gemm_relu_f16", "gemm_f16", "gemm_f16_ex", "gemm_status_string",
+            "gemm_get_device_status", "gemm_selftest_wait_timeout"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_only_the_api_is_exported():
+    import subprocess
+    from tiled_tensor_core_05_b200 import ops
+    out = subprocess.run(["nm", "-D", "--defined-only", ops.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = sorted(line.split()[-1] for line in out.splitlines()
+                      if line.split() and line.split()[-2] in ("T", "W"))
+    assert set(exported) == set(declared_functions()), exported
+
+
+def test_status_strings(lib):
+    from tiled_tensor_core_05_b200 import ops
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        s = ops.status_string(code)
+        assert s and s != "unknown status", code
+    assert ops.status_string(12345) == "unknown status"
+
+
+def test_path_selection(lib):
+    from tiled_tensor_core_05_b200 import ops
+    assert ops.select_path(32, 28672, 8192) == ops.PATH_STREAMK
+    assert ops.select_path(64, 100, 100) == ops.PATH_STREAMK
+    assert ops.select_path(65, 100, 100) == ops.PATH_TILE
+    assert ops.select_path(8192, 8192, 8192) == ops.PATH_TILE
+
+
+def test_abi_version(lib):
+    assert lib.gemm_abi_version() >= 10000
+
+
+def test_argument_errors_are_reported_before_any_device_work(lib):
+    # Negative sizes and bad flags are rejected on the host, without touching a GPU.
+    null = ctypes.c_void_p(0)
+    assert lib.gemm_f16_ex(null, null, null, -1, 4, 4, 8, 8, 8, 1, 0, None) == -1
+    assert lib.gemm_f16_ex(null, null, null, 4, 4, 4, 8, 8, 8, 2, 0, None) == -1
+    assert lib.gemm_f16_ex(null, null, null, 4, 4, 4, 8, 8, 8, 1, 7, None) == -1
+    assert lib.gemm_f16_ex(null, null, null, 1 << 31, 4, 4, 8, 8, 8, 1, 0, None) == -1
+    # empty output: a no-op, whatever the pointers
+    assert lib.gemm_relu_f16(null, null, null, 0, 5, 5, 8, 8, 8, None) == 0
+    assert lib.gemm_f16(null, null, null, 5, 0, 5, 8, 8, 8, None) == 0

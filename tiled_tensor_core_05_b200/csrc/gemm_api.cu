@@ -1,0 +1,323 @@
+// Host side of libttc05: the C ABI declared in include/gemm_f16.h.
+//
+// Argument validation, per-device context (SM count, status word), TMA
+// tensor-map encoding, the choice between the tile kernel and the stream-K
+// kernel, the stream-K workspace cache and the status/self-test entry points.
+// The computation itself is the fused GEMM + ReLU of "Writing high-performance
+// kernels in TileLang" (atlascloud.ai blog), section "Escribamos un GEMM".
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+#include <vector>
+
+#include "../../include/gemm_f16.h"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace ttc {
+
+// One status word per device (first device-side error wins; 0 = none).
+__device__ int g_device_status;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s per wait
+constexpr int kMaxDevices = 64;
+
+struct DeviceEntry {
+  bool ready = false;
+  bool supported = false;
+  int sm_count = 0;
+  int* status = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceEntry g_devices[kMaxDevices];
+
+struct Workspace {
+  int device;
+  cudaStream_t stream;
+  void* ptr;
+  size_t bytes;
+};
+std::vector<Workspace> g_workspaces;
+
+// ------------------------------------------------------ driver entry points ---
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+EncodeTiledFn g_encode = nullptr;
+AddressRangeFn g_addr_range = nullptr;
+std::once_flag g_entry_once;
+
+void load_entry_points() {
+  std::call_once(g_entry_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_addr_range = reinterpret_cast<AddressRangeFn>(fn);
+  });
+}
+
+// ------------------------------------------------------------ device state ---
+int get_device(DeviceCtx* ctx) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GEMM_ERR_LAUNCH;
+  if (dev < 0 || dev >= kMaxDevices) return GEMM_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceEntry& e = g_devices[dev];
+  if (!e.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return GEMM_ERR_LAUNCH;
+    e.supported = (major == 10 && minor == 0);
+    e.sm_count = sms;
+    if (e.supported) {
+      // The symbol's device address for this device (host code cannot use the
+      // symbol itself as a pointer).
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return GEMM_ERR_LAUNCH;
+      e.status = static_cast<int*>(p);
+    }
+    e.ready = true;
+  }
+  if (!e.supported) return GEMM_ERR_UNSUPPORTED_DEVICE;
+  ctx->device = dev;
+  ctx->sm_count = e.sm_count;
+  ctx->status = e.status;
+  ctx->timeout_ns = kDefaultTimeoutNs;
+  return GEMM_OK;
+}
+
+// Device memory of the current device (or managed memory) only.
+bool is_device_pointer(const void* p, int device) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error state of this query
+    return false;
+  }
+  if (attr.type == cudaMemoryTypeManaged) return true;
+  return attr.type == cudaMemoryTypeDevice && attr.device == device;
+}
+
+// The bytes [p, p + (rows-1)*ld*2 + cols*2) lie in one allocation.
+bool extent_in_allocation(const void* p, int64_t rows, int64_t cols, int64_t ld) {
+  if (g_addr_range == nullptr) return true;  // cannot check; TMA bounds still apply
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (g_addr_range(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS) return false;
+  const uint64_t start = reinterpret_cast<uint64_t>(p);
+  const uint64_t span = (static_cast<uint64_t>(rows - 1) * static_cast<uint64_t>(ld) +
+                         static_cast<uint64_t>(cols)) * 2u;
+  return start >= base && start - base + span <= size;
+}
+
+int check_matrix(const void* p, int64_t rows, int64_t cols, int64_t ld, int device) {
+  if (p == nullptr) return GEMM_ERR_INVALID_ARG;
+  if (ld < cols || ld < 1) return GEMM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0 || (ld & 7) != 0) return GEMM_ERR_ALIGNMENT;
+  if (static_cast<uint64_t>(ld) * 2u >= (1ull << 40)) return GEMM_ERR_INVALID_ARG;
+  if (!is_device_pointer(p, device)) return GEMM_ERR_INVALID_ARG;
+  if (!extent_in_allocation(p, rows, cols, ld)) return GEMM_ERR_INVALID_ARG;
+  return GEMM_OK;
+}
+
+int get_workspace(const DeviceCtx& d, cudaStream_t stream, void** ptr, size_t* bytes) {
+  const size_t need = streamk_workspace_bytes(d.sm_count, 64);
+  std::lock_guard<std::mutex> lock(g_mutex);
+  for (const Workspace& w : g_workspaces) {
+    if (w.device == d.device && w.stream == stream) {
+      *ptr = w.ptr;
+      *bytes = w.bytes;
+      return GEMM_OK;
+    }
+  }
+  void* p = nullptr;
+  if (cudaMalloc(&p, need) != cudaSuccess) {
+    cudaGetLastError();
+    return GEMM_ERR_WORKSPACE;
+  }
+  // the counters start at zero and every call leaves them at zero
+  if (cudaMemsetAsync(p, 0, need, stream) != cudaSuccess) {
+    cudaFree(p);
+    return GEMM_ERR_WORKSPACE;
+  }
+  g_workspaces.push_back({d.device, stream, p, need});
+  *ptr = p;
+  *bytes = need;
+  return GEMM_OK;
+}
+
+__global__ void zero_fill_kernel(__half* C, int64_t M, int64_t N, int64_t ldc) {
+  const int64_t total = M * N;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / N, c = i - r * N;
+    C[r * ldc + c] = __ushort_as_half(0);
+  }
+}
+
+__global__ void wait_probe_kernel(int* status, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives on `bar`: the wait must give up on its own
+    if (!mbar_wait(&bar, 0, &abort_flag, timeout_ns))
+      raise_abort(status, &abort_flag, kStatusTimeoutBase | (kRoleProbe << 4) | 1);
+  }
+}
+
+int read_and_clear_status(const DeviceCtx& d, cudaStream_t stream, int* out) {
+  int host = 0;
+  if (cudaMemcpyAsync(&host, d.status, sizeof(int), cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return GEMM_ERR_LAUNCH;
+  if (host != 0) {
+    if (cudaMemsetAsync(d.status, 0, sizeof(int), stream) != cudaSuccess)
+      return GEMM_ERR_LAUNCH;
+    // a kernel that gave up may have left stream-K arrival counters non-zero
+    std::lock_guard<std::mutex> lock(g_mutex);
+    for (const Workspace& w : g_workspaces)
+      if (w.device == d.device && cudaMemsetAsync(w.ptr, 0, w.bytes, stream) != cudaSuccess)
+        return GEMM_ERR_LAUNCH;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GEMM_ERR_LAUNCH;
+  }
+  *out = host;
+  return GEMM_OK;
+}
+
+}  // namespace
+
+int encode_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t ld, uint32_t box_inner, uint32_t box_outer) {
+  load_entry_points();
+  if (g_encode == nullptr) return GEMM_ERR_LAUNCH;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {ld * 2u};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estrides[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base),
+                              dims, strides, box, estrides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_INVALID_ARG;
+}
+
+int launch_zero_fill(const GemmProblem& p) {
+  const int64_t total = p.M * p.N;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  zero_fill_kernel<<<static_cast<int>(blocks), 256, 0, p.stream>>>(static_cast<__half*>(p.C),
+                                                                     p.M, p.N, p.ldc);
+  return cudaGetLastError() == cudaSuccess ? GEMM_OK : GEMM_ERR_LAUNCH;
+}
+
+}  // namespace ttc
+
+using namespace ttc;
+
+extern "C" {
+
+int gemm_abi_version(void) { return 10000; }
+
+int gemm_select_path(int64_t M, int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  return (M >= 1 && M <= 64) ? GEMM_PATH_STREAMK : GEMM_PATH_TILE;
+}
+
+const char* gemm_status_string(int status) {
+  switch (status) {
+    case GEMM_OK: return "ok";
+    case GEMM_ERR_INVALID_ARG: return "invalid argument (size, leading dimension or pointer)";
+    case GEMM_ERR_ALIGNMENT: return "pointer not 16-byte aligned or leading dimension not a multiple of 8";
+    case GEMM_ERR_UNSUPPORTED_DEVICE: return "current device is not an sm_100 (B200) GPU";
+    case GEMM_ERR_LAUNCH: return "CUDA runtime call or kernel launch failed";
+    case GEMM_ERR_WORKSPACE: return "stream-K workspace allocation failed";
+    case GEMM_ERR_DEVICE_TIMEOUT: return "a device-side wait ran out of time";
+    default: return "unknown status";
+  }
+}
+
+int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                int64_t lda, int64_t ldb, int64_t ldc, int relu, int path,
+                gemm_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return GEMM_ERR_INVALID_ARG;
+  if (relu != 0 && relu != 1) return GEMM_ERR_INVALID_ARG;
+  if (path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE && path != GEMM_PATH_STREAMK)
+    return GEMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return GEMM_OK;
+  DeviceCtx d;
+  int rc = get_device(&d);
+  if (rc != GEMM_OK) return rc;
+  rc = check_matrix(C, M, N, ldc, d.device);
+  if (rc != GEMM_OK) return rc;
+  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, relu != 0, stream};
+  if (K == 0) return launch_zero_fill(p);
+  rc = check_matrix(A, M, K, lda, d.device);
+  if (rc == GEMM_OK) rc = check_matrix(B, K, N, ldb, d.device);
+  if (rc != GEMM_OK) return rc;
+  if (path == GEMM_PATH_AUTO) path = gemm_select_path(M, N, K);
+  if (path == GEMM_PATH_STREAMK) {
+    if (streamk_m_pad(M) == 0) return GEMM_ERR_INVALID_ARG;
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+    rc = get_workspace(d, stream, &ws, &ws_bytes);
+    if (rc != GEMM_OK) return rc;
+    return launch_streamk_gemm(p, d, ws, ws_bytes);
+  }
+  return launch_tile_gemm(p, d);
+}
+
+int gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                  int64_t lda, int64_t ldb, int64_t ldc, gemm_stream_t stream) {
+  return gemm_f16_ex(A, B, C, M, N, K, lda, ldb, ldc, 1, GEMM_PATH_AUTO, stream);
+}
+
+int gemm_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+             int64_t lda, int64_t ldb, int64_t ldc, gemm_stream_t stream) {
+  return gemm_f16_ex(A, B, C, M, N, K, lda, ldb, ldc, 0, GEMM_PATH_AUTO, stream);
+}
+
+int gemm_get_device_status(gemm_stream_t stream, int* device_status) {
+  if (device_status == nullptr) return GEMM_ERR_INVALID_ARG;
+  DeviceCtx d;
+  const int rc = get_device(&d);
+  if (rc != GEMM_OK) return rc;
+  return read_and_clear_status(d, stream, device_status);
+}
+
+int gemm_selftest_wait_timeout(int64_t timeout_ns, gemm_stream_t stream, int* device_status) {
+  if (device_status == nullptr || timeout_ns <= 0 || timeout_ns > 10ll * 1000 * 1000 * 1000)
+    return GEMM_ERR_INVALID_ARG;
+  DeviceCtx d;
+  int rc = get_device(&d);
+  if (rc != GEMM_OK) return rc;
+  wait_probe_kernel<<<1, 32, 0, stream>>>(d.status, static_cast<uint64_t>(timeout_ns));
+  if (cudaGetLastError() != cudaSuccess) return GEMM_ERR_LAUNCH;
+  return read_and_clear_status(d, stream, device_status);
+}
+
+}  // extern "C"

@@ -1,0 +1,349 @@
+// Large-shape path of C = ReLU(A @ B) (or A @ B) for sm_100a.
+//
+// The operation and its blocking follow "Writing high-performance kernels in
+// TileLang" (atlascloud.ai blog), section "Escribamos un GEMM": one output
+// tile of block_M x block_N per work item, A and B tiles of block_K staged in
+// shared memory through a software pipeline, a tensor-core tile MMA into an
+// fp32 accumulator, max(x, 0) on the accumulator, a cast to fp16 on the way
+// out, and an L2-friendly ordering of the tiles (T.use_swizzle).
+//
+// Blackwell re-design:
+//   * persistent grid (one CTA per SM) walking the output tiles in
+//     grouped-panel order (group_m tile-rows per panel);
+//   * warp 0: TMA producer filling a STAGES-deep ring of 128-byte-swizzled
+//     A (128 x 64) and B (64 x BN) tiles, with mbarrier full/empty handshakes;
+//   * warp 1: allocates TMEM and issues tcgen05.mma (128 x BN x 16) from one
+//     thread into a double-buffered fp32 accumulator in TMEM;
+//   * warps 2-5: epilogue.  tcgen05.ld -> ReLU in fp32 -> RNE to fp16 ->
+//     swizzled shared-memory staging -> TMA store, which clips rows/columns
+//     beyond M/N (ragged edges).  The epilogue of tile i overlaps the
+//     main loop of tile i+1 thanks to the second accumulator.
+// Out-of-range A/B elements (M, N or K not a multiple of the tile) are
+// zero-filled by TMA and so contribute nothing to the sum.
+#include <atomic>
+#include <cstdlib>
+
+#include "../../include/gemm_f16.h"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace ttc {
+namespace {
+
+constexpr int kBM = 128;        // tile rows (MMA M)
+constexpr int kBK = 64;         // k-block: 64 fp16 = one 128-byte swizzle row
+constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
+constexpr int kThreads = 192;   // 6 warps
+constexpr int kEpiWarps = 4;
+constexpr int kEpiRows = 32;    // rows per epilogue warp
+constexpr int kEpiCols = 64;    // columns per epilogue chunk (128 bytes of fp16)
+constexpr int kEpiBuf = kEpiRows * kEpiCols * 2;
+
+template <int BN, int STAGES>
+struct TileCfg {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBChunk = kBK * 64 * 2;  // one 64-column slab of the B tile
+  static constexpr int kBBytes = kBK * BN * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiBuf;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
+  static constexpr uint32_t kTmemCols = 2 * BN;
+  static constexpr uint32_t kIdesc = idesc_f16_f32(kBM, BN, /*A MN-major*/ false,
+                                                   /*B MN-major*/ true);
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+// Grouped-panel rasterisation: consecutive tile indices sweep group_m
+// tile-rows of one panel column by column, so the CTAs that run at the same
+// time share A rows and B columns in L2.
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m,
+                                            int& mb, int& nb) {
+  const int per_group = group_m * num_n;
+  const int g = tile / per_group;
+  const int first_m = g * group_m;
+  const int rows = min(num_m - first_m, group_m);
+  const int r = tile - g * per_group;
+  mb = first_m + r % rows;
+  nb = r / rows;
+}
+
+template <int BN, int STAGES, bool RELU>
+__global__ void __launch_bounds__(kThreads, 1)
+    tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, int group_m,
+                     int* status, uint64_t timeout_ns) {
+  using Cfg = TileCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + STAGES * Cfg::kABytes;
+  uint8_t* smEpi = smem + STAGES * Cfg::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smEpi + Cfg::kEpiBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_m = (M + kBM - 1) / kBM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer ---
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, group_m, mb, nb);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+          tma_load_2d(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, mb * kBM);
+          uint8_t* bdst = smB + stage * Cfg::kBBytes;
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(&tmB, &full[stage], bdst + j * Cfg::kBChunk, nb * BN + j * 64, kb * kBK);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleProducer << 4) | 1);
+        // let every load already issued land before shared memory is released
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) (void)mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer ---
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      int site = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
+          ok = false;
+          site = 1;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
+            ok = false;
+            site = 2;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_u32(smA + stage * Cfg::kABytes);
+          const uint32_t b_addr = smem_u32(smB + stage * Cfg::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k) {
+            // A: K-major, advance 16 fp16 = 32 bytes along the swizzled row.
+            const uint64_t adesc = smem_desc_sw128(a_addr + k * (kUmmaK * 2), 16, 1024);
+            // B: N-major, advance 16 k-rows of 128 bytes.
+            const uint64_t bdesc =
+                smem_desc_sw128(b_addr + k * (kUmmaK * 128), Cfg::kBChunk, 1024);
+            umma_f16(d_tmem, adesc, bdesc, Cfg::kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleMma << 4) | site);
+        umma_commit(drain);  // wait for MMAs in flight before TMEM is released
+        (void)mbar_wait(drain, 0, nullptr, timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue ---
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint8_t* bufs = smEpi + (warp - 2) * 2 * kEpiBuf;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    uint32_t chunk_no = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, group_m, mb, nb);
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, timeout_ns) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0)
+          raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleEpilogue << 4) | 1);
+        break;
+      }
+      tc_fence_after_sync();
+      const int row0 = mb * kBM + q * kEpiRows;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / kEpiCols; ++c) {
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(t_row + c * kEpiCols, v0);
+        tmem_ld_32x32b_x32(t_row + c * kEpiCols + 32, v1);
+        tmem_wait_ld();
+        if (c == BN / kEpiCols - 1) {
+          // the accumulator has been read: hand it back to the MMA warp
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+        uint32_t h[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float x0 = __uint_as_float(v0[2 * i]), x1 = __uint_as_float(v0[2 * i + 1]);
+          float y0 = __uint_as_float(v1[2 * i]), y1 = __uint_as_float(v1[2 * i + 1]);
+          if (RELU) {
+            x0 = relu_f32(x0);
+            x1 = relu_f32(x1);
+            y0 = relu_f32(y0);
+            y1 = relu_f32(y1);
+          }
+          h[i] = pack_half2(x0, x1);
+          h[16 + i] = pack_half2(y0, y1);
+        }
+        uint8_t* buf = bufs + (chunk_no & 1u) * kEpiBuf;
+        if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+        __syncwarp();
+        // row `lane`, 128 bytes = 8 chunks of 16 bytes, chunk j stored at j ^ (row & 7)
+        const uint32_t row_addr = smem_u32(buf) + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), h[4 * j], h[4 * j + 1], h[4 * j + 2],
+                       h[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int col0 = nb * BN + c * kEpiCols;
+          if (row0 < M && col0 < N) tma_store_2d(&tmC, buf, col0, row0);
+          bulk_commit_group();
+        }
+        ++chunk_no;
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// Sets the dynamic shared-memory limit of a kernel once per device.
+bool ensure_smem_attr(const void* func, int bytes, int device, std::atomic<uint64_t>& done) {
+  const uint64_t bit = 1ull << (device & 63);
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
+int group_m_setting() {
+  static const int g = [] {
+    const char* s = std::getenv("TTC_GROUP_M");
+    const int v = s ? std::atoi(s) : 0;
+    return v > 0 ? v : 8;
+  }();
+  return g;
+}
+
+template <int BN, int STAGES, bool RELU>
+int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
+  using Cfg = TileCfg<BN, STAGES>;
+  static std::atomic<uint64_t> attr_done{0};
+  CUtensorMap tA, tB, tC;
+  int rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, kBM);
+  if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
+  if (rc == 0) rc = encode_tmap_f16_2d(&tC, p.C, p.N, p.M, p.ldc, kEpiCols, kEpiRows);
+  if (rc != 0) return rc;
+  auto kern = tile_gemm_kernel<BN, STAGES, RELU>;
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
+                        attr_done))
+    return GEMM_ERR_LAUNCH;
+  const int64_t num_tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
+  const int grid = static_cast<int>(num_tiles < d.sm_count ? num_tiles : d.sm_count);
+  kern<<<grid, kThreads, Cfg::kSmemBytes, p.stream>>>(
+      tA, tB, tC, static_cast<int>(p.M), static_cast<int>(p.N), static_cast<int>(p.K),
+      group_m_setting(), d.status, d.timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? 0 : GEMM_ERR_LAUNCH;
+}
+
+}  // namespace
+
+int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d) {
+  // 128 x 256 tiles when there are enough of them to fill the GPU, otherwise
+  // 128 x 128 tiles (twice as many CTAs for small problems).
+  const int64_t tiles256 = ((p.M + kBM - 1) / kBM) * ((p.N + 255) / 256);
+  const bool wide = tiles256 >= d.sm_count;
+  if (wide) return p.relu ? launch_impl<256, 4, true>(p, d) : launch_impl<256, 4, false>(p, d);
+  return p.relu ? launch_impl<128, 6, true>(p, d) : launch_impl<128, 6, false>(p, d);
+}
+
+}  // namespace ttc

@@ -1,0 +1,48 @@
+// Host-side declarations shared by the translation units of libttc05.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ttc {
+
+struct GemmProblem {
+  const void* A;
+  const void* B;
+  void* C;
+  int64_t M, N, K;
+  int64_t lda, ldb, ldc;
+  bool relu;
+  cudaStream_t stream;
+};
+
+struct DeviceCtx {
+  int device;
+  int sm_count;
+  int* status;          // device address of the status word of this device
+  uint64_t timeout_ns;  // limit for every device-side wait
+};
+
+// Encode a 2-D row-major fp16 tensor map with 128-byte swizzle.
+//   inner/outer: extents in elements (inner is contiguous)
+//   ld: row stride in elements; box_inner/box_outer: box extents in elements
+// Returns 0 or a GEMM_ERR_* code.
+int encode_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t ld, uint32_t box_inner, uint32_t box_outer);
+
+// Large-shape path: persistent warp-specialised tcgen05 kernel.
+int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d);
+
+// Small-M path: swap-AB stream-K kernel.  `workspace` holds partial tiles and
+// per-tile arrival counters (counters must be zero on entry; the kernel
+// leaves them zero).
+size_t streamk_workspace_bytes(int sm_count, int m_pad);
+int launch_streamk_gemm(const GemmProblem& p, const DeviceCtx& d, void* workspace,
+                        size_t workspace_bytes);
+int streamk_m_pad(int64_t M);  // MMA N used for M rows (0 if M is too large)
+
+// Writes C = 0 (used when K == 0: the empty sum, and ReLU of it, is +0).
+int launch_zero_fill(const GemmProblem& p);
+
+}  // namespace ttc

@@ -1,0 +1,146 @@
+"""Python binding of libttc05 (argument marshalling only).
+
+Every function here forwards device pointers, sizes, leading dimensions and
+the current CUDA stream of PyTorch to the C ABI of ``include/gemm_f16.h``; all
+arithmetic happens in the library's CUDA kernels.  There is no fallback: if
+the library is missing or the call fails, a ``RuntimeError`` is raised.
+
+The operation is C = ReLU(A @ B) (``gemm_relu_f16``) or C = A @ B
+(``gemm_f16``) on row-major fp16 matrices with fp32 accumulation, as in
+"Writing high-performance kernels in TileLang" (atlascloud.ai blog), section
+"Escribamos un GEMM".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libttc05.so")
+
+PATH_AUTO, PATH_TILE, PATH_STREAMK = 0, 1, 2
+
+_lib = None
+
+_SIGNATURES = {
+    "gemm_relu_f16": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
+                      ctypes.c_int),
+    "gemm_f16": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
+                 ctypes.c_int),
+    "gemm_f16_ex": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 +
+                    [ctypes.c_int, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
+    "gemm_select_path": ([ctypes.c_int64] * 3, ctypes.c_int),
+    "gemm_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "gemm_get_device_status": ([ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
+    "gemm_selftest_wait_timeout": ([ctypes.c_int64, ctypes.c_void_p,
+                                    ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
+    "gemm_abi_version": ([], ctypes.c_int),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m tiled_tensor_core_05_b200.build` (there is no CPU fallback)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().gemm_status_string(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"{what} failed: {status_string(rc)} ({rc})")
+
+
+def _stream_handle(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ld_padded(t: torch.Tensor) -> int:
+    """Row stride in elements.  A single-row matrix has no meaningful stride,
+    so its columns rounded up to the 8-element rule are passed instead."""
+    if t.dim() != 2:
+        raise ValueError("expected a 2-D tensor")
+    if t.size(1) > 1 and t.stride(1) != 1:
+        raise ValueError("columns must be contiguous (stride(1) == 1)")
+    if t.size(0) > 1:
+        return int(t.stride(0))
+    return (int(t.size(1)) + 7) // 8 * 8
+
+
+def gemm_f16_ex(a: torch.Tensor, b: torch.Tensor, out: torch.Tensor | None = None, *,
+                relu: bool = True, path: int = PATH_AUTO, stream=None) -> torch.Tensor:
+    """C = ReLU(A @ B) (relu=True) or A @ B on CUDA fp16 tensors.
+
+    ``a`` is (M, K), ``b`` is (K, N), ``out`` (allocated if None) is (M, N);
+    all fp16 on the same CUDA device with contiguous columns.  The call is
+    asynchronous on ``stream`` (default: the current stream)."""
+    if a.dtype != torch.float16 or b.dtype != torch.float16:
+        raise TypeError("a and b must be torch.float16")
+    if not (a.is_cuda and b.is_cuda):
+        raise ValueError("a and b must be CUDA tensors")
+    M, K = a.shape
+    K2, N = b.shape
+    if K != K2:
+        raise ValueError(f"shape mismatch {tuple(a.shape)} @ {tuple(b.shape)}")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
+    if out.dtype != torch.float16 or tuple(out.shape) != (M, N) or out.device != a.device:
+        raise ValueError("out must be an fp16 (M, N) tensor on the device of a")
+    dev = a.device
+    with torch.cuda.device(dev):
+        rc = lib().gemm_f16_ex(a.data_ptr(), b.data_ptr(), out.data_ptr(), M, N, K,
+                               _ld_padded(a), _ld_padded(b), _ld_padded(out), int(bool(relu)),
+                               int(path), _stream_handle(stream, dev))
+    _check(rc, "gemm_f16_ex")
+    return out
+
+
+def gemm_relu_f16(a, b, out=None, *, stream=None):
+    """C = ReLU(A @ B); see :func:`gemm_f16_ex`."""
+    return gemm_f16_ex(a, b, out, relu=True, stream=stream)
+
+
+def gemm_f16(a, b, out=None, *, stream=None):
+    """C = A @ B; see :func:`gemm_f16_ex`."""
+    return gemm_f16_ex(a, b, out, relu=False, stream=stream)
+
+
+def select_path(M: int, N: int, K: int) -> int:
+    return int(lib().gemm_select_path(M, N, K))
+
+
+def device_status(stream=None, device=None) -> int:
+    """Synchronise and return (then clear) the device status word (0 = ok)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    st = ctypes.c_int(0)
+    with torch.cuda.device(dev):
+        _check(lib().gemm_get_device_status(_stream_handle(stream, dev), ctypes.byref(st)),
+               "gemm_get_device_status")
+    return int(st.value)
+
+
+def selftest_wait_timeout(timeout_ns: int, stream=None, device=None) -> int:
+    """Run the bounded-wait self test; returns the status word it produced."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    st = ctypes.c_int(0)
+    with torch.cuda.device(dev):
+        _check(lib().gemm_selftest_wait_timeout(int(timeout_ns), _stream_handle(stream, dev),
+                                                ctypes.byref(st)),
+               "gemm_selftest_wait_timeout")
+    return int(st.value)
