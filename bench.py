@@ -1,0 +1,462 @@
+"""Benchmark of the fused fp16 GEMM + ReLU (C = ReLU(A @ B)) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload cube8192|mlp_up|decode|...] [--no-secondary]
+
+One step is one call of ``gemm_relu_f16`` (through the C ABI) over one set of
+synthetic, seeded inputs already resident in HBM.  The default workload is the
+compute-bound 8192^3 cube (A, B ~ N(0,1)/sqrt(K), seed 2); the MLP
+up-projection and the decode-shaped skinny product are reported alongside as
+``other_workloads``.  Timing: W untimed warm-up steps, then K steps between a
+barrier + synchronize on both sides, timed with CUDA events on the launching
+stream; the job time is the max over ranks.  With N > 1 (torchrun, one rank
+per GPU) every rank runs its own independent replica of the problem (weak
+scaling, no collective on the data path).
+
+``--impl reference`` times the CPU oracle (the plain fp64 definition of the
+operation) on a bounded sample of the same workload on the host cores; under
+torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fused GEMM+ReLU TFLOP/s and % of B200 dense fp16 peak (GB/s % HBM for skinny)"
+NOMINAL_FP16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["tiled_tensor_core_05_b200/csrc/gemm_tile.cu",
+                  "tiled_tensor_core_05_b200/csrc/gemm_streamk.cu",
+                  "tiled_tensor_core_05_b200/csrc/sm100.cuh"]
+
+
+# ------------------------------------------------------------------ utils ---
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = table.get(workload)
+    if not e or e.get("kernel_src_sha") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is busy."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, interval_ms: int = 20):
+        self.samples = []
+        self.proc = None
+        self.marks = {}
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(interval_ms), "-i", gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append((time.monotonic(), parts))
+
+    def wait_first(self, timeout=15.0):
+        t0 = time.monotonic()
+        while self.proc is not None and not self.samples and time.monotonic() - t0 < timeout:
+            time.sleep(0.02)
+
+    def mark(self, name):
+        self.marks[name] = time.monotonic()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, start="t0", end="t1"):
+        if self.proc is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        t0, t1 = self.marks.get(start, 0), self.marks.get(end, 1e30)
+        inside = [p for (t, p) in self.samples if t0 <= t <= t1 + 0.05]
+        note = "samples taken during the timed region"
+        if not inside:
+            # a timed region shorter than the sampling interval: use the
+            # samples of the surrounding busy period (warm-up included)
+            w0 = self.marks.get("warm0", t0)
+            inside = [p for (t, p) in self.samples if w0 <= t <= t1 + 0.1]
+            note = "timed region shorter than the sampling interval; warm-up + timed samples"
+        if not inside:
+            inside = [self.samples[-1][1]]
+            note = "no sample inside the busy period; last sample"
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[0]) for p in inside if num(p[0]) is not None]
+        smax = [num(p[1]) for p in inside if num(p[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in inside for i in range(4)
+                          if p[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(inside),
+                "power_w_max": max((num(p[2]) or 0.0) for p in inside), "note": note}
+
+
+def gpu_id_for(dev_index: int) -> str:
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(dev_index).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[dev_index]
+        return str(dev_index)
+
+
+# ----------------------------------------------------------- measurements ---
+
+def time_launches(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
+    """Warm up, then time `steps` calls with CUDA events on `stream`.
+    Returns (total_ms max over ranks, mean per-launch ms on this rank)."""
+    import torch
+    if sampler:
+        sampler.mark("warm0")
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    if sampler:
+        sampler.mark("t0")
+    ev0.record(stream)
+    for i in range(steps):
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark("t1")
+    if dist is not None:
+        dist.barrier()
+    total = ev0.elapsed_time(ev1)
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if dist is not None:
+        t = torch.tensor([total], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    return total, sum(per) / len(per)
+
+
+def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True):
+    import torch
+
+    from tiled_tensor_core_05_b200 import ops, workloads
+    w = workloads.WORKLOADS[name]
+    a_cpu, b_cpu = workloads.workload_inputs(name)
+    a, b = a_cpu.cuda(), b_cpu.cuda()
+    c = torch.empty((w.M, w.N), dtype=torch.float16, device="cuda")
+    stream = torch.cuda.current_stream()
+    lib = ops.lib()
+    h = int(stream.cuda_stream)
+    args = (a.data_ptr(), b.data_ptr(), c.data_ptr(), w.M, w.N, w.K, w.K, w.N, w.N, h)
+
+    def step():
+        rc = lib.gemm_relu_f16(*args)
+        if rc != 0:
+            raise RuntimeError(f"gemm_relu_f16 failed: {ops.status_string(rc)}")
+
+    total_ms, launch_ms = time_launches(step, steps, warmup, stream, dist, sampler)
+    st = ops.device_status()
+    if st != 0:
+        raise RuntimeError(f"device reported status {st:#x}")
+    res = {"total_ms": total_ms, "launch_ms": launch_ms, "w": w}
+    if e2e:
+        # end to end through the C ABI: pinned host inputs -> device, the
+        # kernel, result -> pinned host, every step
+        a_h = a_cpu.pin_memory()
+        b_h = b_cpu.pin_memory()
+        c_h = torch.empty((w.M, w.N), dtype=torch.float16).pin_memory()
+
+        def e2e_step():
+            a.copy_(a_h, non_blocking=True)
+            b.copy_(b_h, non_blocking=True)
+            step()
+            c_h.copy_(c, non_blocking=True)
+
+        e_steps = max(3, min(steps, 10))
+        e_total, _ = time_launches(e2e_step, e_steps, 1, stream, dist, None)
+        res["e2e_ms"] = e_total / e_steps
+        res["h2d"] = a.numel() * 2 + b.numel() * 2
+        res["d2h"] = c.numel() * 2
+        if not torch.equal(c_h.view(torch.int16), c.cpu().view(torch.int16)):
+            raise RuntimeError("end-to-end result differs from the device result")
+    del a, b, c
+    torch.cuda.empty_cache()
+    return res
+
+
+def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool):
+    from tiled_tensor_core_05_b200 import workloads
+    w = workloads.WORKLOADS[name]
+    if name == "decode":
+        # HBM bound: algorithmic bytes = A, B read once, C written once
+        achieved = w.bytes_min / (launch_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic_for(name),
+                "algorithmic_bytes_per_launch": w.bytes_min,
+                "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"}
+    achieved = w.flops / (launch_ms * 1e-3) / 1e12
+    key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
+    peak = peaks.get(key, peaks["bf16_tflops"])
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic_for(name),
+            "algorithmic_flops_per_launch": w.flops,
+            "peak_source": f"{peak_src} {key} (cuBLAS bf16; fp16 has the same nominal rate)"}
+
+
+def cpu_baseline(name, budget_s=10.0):
+    """The oracle timed on a bounded sample (leading rows) of the workload."""
+    import oracle
+    from tiled_tensor_core_05_b200 import workloads
+    w = workloads.WORKLOADS[name]
+    a, b = workloads.workload_inputs(name)
+    t0 = time.perf_counter()
+    oracle.gemm_relu(a[:1], b)
+    t_row = max(time.perf_counter() - t0, 1e-4)
+    rows = int(max(1, min(w.M, budget_s / t_row)))
+    t0 = time.perf_counter()
+    oracle.gemm_relu(a[:rows], b)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * w.N * w.K
+    if name == "decode":
+        value = (2.0 * (rows * w.K + w.K * w.N + rows * w.N)) / dt / 1e9
+        unit = "GB/s"
+    else:
+        value = flops / dt / 1e12
+        unit = "TFLOP/s"
+    return {"value": value, "unit": unit, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"first {rows} of {w.M} rows of C ({rows}x{w.N}x{w.K}), {dt:.1f} s",
+            "seconds": round(dt, 2)}
+
+
+# ------------------------------------------------------------------ arms ---
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from tiled_tensor_core_05_b200 import workloads
+    w = workloads.WORKLOADS[args.workload]
+    a, b = workloads.workload_inputs(args.workload)
+    # size one step to about a second of host work
+    t0 = time.perf_counter()
+    oracle.gemm_relu(a[:1], b)
+    t_row = max(time.perf_counter() - t0, 1e-4)
+    rows = int(max(1, min(w.M, 1.0 / t_row)))
+    for _ in range(args.warmup):
+        oracle.gemm_relu(a[:rows], b)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gemm_relu(a[:rows], b)
+    dt = (time.perf_counter() - t0) / args.steps
+    if args.workload == "decode":
+        value, unit = 2.0 * (rows * w.K + w.K * w.N + rows * w.N) / dt / 1e9, "GB/s"
+    else:
+        value, unit = 2.0 * rows * w.N * w.K / dt / 1e12, "TFLOP/s"
+    sample = f"first {rows} of {w.M} rows of C per step ({rows}x{w.N}x{w.K})"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": oracle.max_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    mib = (w.M * w.K + w.K * w.N) * 2 / 2 ** 20
+    if mib * 2 ** 20 > 126e6:
+        l2 = "A+B = %.0f MiB > 126 MB L2: inputs larger than L2, no flush" % mib
+    else:
+        l2 = "A+B = %.2f MiB fits in L2: L2-warm timing (latency-bound case)" % mib
+    return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "seed": w.seed,
+            "a_scale": w.a_scale, "b_scale": w.b_scale, "layout": "row-major, ld = cols",
+            "l2": l2, "parallelism": "replicas (one independent problem per GPU)"}
+
+
+def run_ours(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    from tiled_tensor_core_05_b200 import ops, workloads
+    ops.lib()
+    peaks, peak_src = load_peaks()
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.wait_first()
+    main = measure_workload(args.workload, args.steps, args.warmup, dist, sampler,
+                            e2e=not args.no_e2e)
+    sampler.stop()
+    clocks = sampler.summary()
+    w = main["w"]
+    long_run = main["total_ms"] > 2000.0
+    ms = main["total_ms"] / args.steps
+    if args.workload == "decode":
+        value, unit = world * w.bytes_min / (ms * 1e-3) / 1e9, "GB/s"
+    else:
+        value, unit = world * w.flops / (ms * 1e-3) / 1e12, "TFLOP/s"
+    line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic (seeded torch.randn on the CPU, cast to fp16)",
+            "config": workload_config(w), "gpu_launches": args.steps}
+    if args.workload == "decode":
+        line["pct_of_nominal_hbm"] = round(100 * value / world / NOMINAL_HBM_GBS, 2)
+    else:
+        line["pct_of_dense_fp16_peak"] = round(100 * value / world / NOMINAL_FP16_TFLOPS, 2)
+    line["roofline"] = roofline_entry(args.workload, main["launch_ms"], peaks, peak_src,
+                                      long_run)
+    line["roofline"]["kernel"] = ("streamk_gemm_kernel" if args.workload == "decode"
+                                  else "tile_gemm_kernel")
+    if "e2e_ms" in main:
+        e_ms = main["e2e_ms"]
+        ev = (w.flops / (e_ms * 1e-3) / 1e12) if unit == "TFLOP/s" else \
+            (w.bytes_min / (e_ms * 1e-3) / 1e9)
+        line["e2e"] = {"value": round(world * ev, 2), "unit": unit,
+                       "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"],
+                       "ms_per_step": round(e_ms, 4)}
+    line["clocks"] = clocks
+    if rank == 0 and not args.no_secondary:
+        others = []
+        for name in ("mlp_up", "decode", "cube1024", "cube256"):
+            if name == args.workload:
+                continue
+            r = measure_workload(name, max(args.steps, 20), max(args.warmup, 3), None, None,
+                                 e2e=False)
+            ow = r["w"]
+            entry = {"workload": name, "M": ow.M, "N": ow.N, "K": ow.K,
+                     "ms_per_launch": round(r["launch_ms"], 5),
+                     "tflops": round(ow.flops / (r["launch_ms"] * 1e-3) / 1e12, 2),
+                     "roofline": roofline_entry(name, r["launch_ms"], peaks, peak_src, False)}
+            if name == "decode":
+                entry["gbs"] = round(ow.bytes_min / (r["launch_ms"] * 1e-3) / 1e9, 1)
+                entry["pct_of_nominal_hbm"] = round(100 * entry["gbs"] / NOMINAL_HBM_GBS, 2)
+            else:
+                entry["pct_of_dense_fp16_peak"] = round(100 * entry["tflops"] /
+                                                        NOMINAL_FP16_TFLOPS, 2)
+            others.append(entry)
+        line["other_workloads"] = others
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="cube8192")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

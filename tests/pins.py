@@ -109,7 +109,8 @@ def exact_gemm_bits(a16: np.ndarray, b16: np.ndarray, relu: bool) -> np.ndarray:
 def within_tol(c16, ref16) -> np.ndarray:
     c = np.asarray(c16, dtype=np.float16).astype(np.float64)
     r = np.asarray(ref16, dtype=np.float16).astype(np.float64)
-    return np.abs(c - r) <= ATOL + RTOL * np.abs(r)
+    with np.errstate(invalid="ignore"):
+        return (c == r) | (np.abs(c - r) <= ATOL + RTOL * np.abs(r))
 
 
 def _cmp(name, got, want_bits, exact_ok: bool, fails: list, strict_zero: bool = True):

@@ -188,7 +188,7 @@ def test_empty_output_is_noop():
 
 def test_deterministic_bits_both_paths():
     a, b = workloads.make_inputs(64, 3000, 2500, seed=9)
-    ad, bd = a.cuda(), b.cuda()
+    ad, bd = to_dev(a, round8(2500)), to_dev(b)
     for path in (TILE, STREAMK):
         outs = []
         for _ in range(3):

@@ -74,8 +74,9 @@ template <int BN, int STAGES, bool RELU>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, int group_m,
-                     int* status, uint64_t timeout_ns) {
+                     const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
+                     int64_t ldc, int M, int N, int K, int group_m, int* status,
+                     uint64_t timeout_ns) {
   using Cfg = TileCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -97,6 +98,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + kBK - 1) / kBK;
+  // The TMA store writes whole 16-byte groups of columns, so it is given only
+  // the first N rounded down to 8 columns; the (< 8) remaining columns of a
+  // ragged edge are written with plain stores.
+  const int n8 = N & ~7;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -271,10 +276,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                        h[4 * j + 3]);
         fence_proxy_async_smem();
         __syncwarp();
+        const int col0 = nb * BN + c * kEpiCols;
         if (lane == 0) {
-          const int col0 = nb * BN + c * kEpiCols;
-          if (row0 < M && col0 < N) tma_store_2d(&tmC, buf, col0, row0);
+          if (row0 < M && col0 < n8) tma_store_2d(&tmC, buf, col0, row0);
           bulk_commit_group();
+        }
+        if (n8 < N && col0 + kEpiCols > n8 && col0 < N && row0 + lane < M) {
+          // ragged tail columns [max(n8, col0), min(N, col0 + 64)) of this row,
+          // read back from this thread's own (swizzled) staging row
+          const int j_end = min(N, col0 + kEpiCols);
+          __half* crow = C + static_cast<int64_t>(row0 + lane) * ldc;
+          for (int j = max(n8, col0); j < j_end; ++j) {
+            const int cc = j - col0;
+            const uint32_t addr = row_addr + ((((cc >> 3) ^ (lane & 7)) << 4) | ((cc & 7) << 1));
+            unsigned short bits;
+            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(bits) : "r"(addr) : "memory");
+            crow[j] = __ushort_as_half(bits);
+          }
         }
         ++chunk_no;
       }
@@ -321,7 +339,10 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   CUtensorMap tA, tB, tC;
   int rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, kBM);
   if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
-  if (rc == 0) rc = encode_tmap_f16_2d(&tC, p.C, p.N, p.M, p.ldc, kEpiCols, kEpiRows);
+  // inner extent N rounded down to 8 columns (see the kernel's ragged tail);
+  // the map is never used when that is 0
+  const uint64_t n8 = static_cast<uint64_t>(p.N) & ~7ull;
+  if (rc == 0) rc = encode_tmap_f16_2d(&tC, p.C, n8 > 0 ? n8 : 8, p.M, p.ldc, kEpiCols, kEpiRows);
   if (rc != 0) return rc;
   auto kern = tile_gemm_kernel<BN, STAGES, RELU>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
@@ -330,7 +351,8 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   const int64_t num_tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
   const int grid = static_cast<int>(num_tiles < d.sm_count ? num_tiles : d.sm_count);
   kern<<<grid, kThreads, Cfg::kSmemBytes, p.stream>>>(
-      tA, tB, tC, static_cast<int>(p.M), static_cast<int>(p.N), static_cast<int>(p.K),
+      tA, tB, tC, static_cast<__half*>(p.C), p.ldc, static_cast<int>(p.M),
+      static_cast<int>(p.N), static_cast<int>(p.K),
       group_m_setting(), d.status, d.timeout_ns);
   return cudaGetLastError() == cudaSuccess ? 0 : GEMM_ERR_LAUNCH;
 }
