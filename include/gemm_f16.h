@@ -62,7 +62,8 @@ enum gemm_status {
   GEMM_ERR_UNSUPPORTED_DEVICE = -3, /* current device is not compute capability 10.0 */
   GEMM_ERR_LAUNCH = -4,             /* a CUDA runtime call or kernel launch failed */
   GEMM_ERR_WORKSPACE = -5,          /* workspace allocation failed */
-  GEMM_ERR_DEVICE_TIMEOUT = -6      /* reported by gemm_get_device_status */
+  GEMM_ERR_DEVICE_TIMEOUT = -6,     /* reported by gemm_get_device_status */
+  GEMM_ERR_SCRATCH_LIMIT = -7       /* problem too large for gemm_relu_f16_noalloc's fixed scratch */
 };
 
 enum gemm_path {
@@ -110,6 +111,39 @@ GEMM_API int gemm_get_device_status(gemm_stream_t stream, int* device_status);
  * Synchronises `stream` and stores the status word (then clears it) in
  * *device_status.  Returns GEMM_OK or a negative gemm_status. */
 GEMM_API int gemm_selftest_wait_timeout(int64_t timeout_ns, gemm_stream_t stream, int* device_status);
+
+/* C = ReLU(A @ B) for callers that must not allocate device memory.
+ *
+ * No counterpart in the pages: this is an interface addition, not part of the
+ * method.  gemm_relu_f16 lazily cudaMalloc's a workspace for its small-M
+ * (stream-K) kernel on the first call per (device, stream).  Some callers
+ * cannot allow that: plugins whose enqueue step is forbidden to allocate,
+ * processes whose device memory is owned and accounted for by a pool
+ * allocator, and latency-critical loops where cudaMalloc's implicit device
+ * synchronisation would stall other work.  This entry point runs the same
+ * stream-K kernel, but keeps its scratch (fp32 partial tiles and per-tile
+ * arrival counters) in a fixed array that is part of the library image: every
+ * GPU that loads the library holds those 5,243,648 bytes (5 MiB) until the
+ * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   - Arguments, layout and ownership are those of gemm_relu_f16: device
+ *     pointers, row-major fp16, ld in elements (multiples of 8), 16-byte
+ *     aligned pointers; the caller still provides A, B and C.
+ *   - Limit: M <= 32 (any N and K up to 2^31 - 1).  Larger M returns
+ *     GEMM_ERR_SCRATCH_LIMIT and launches nothing.  M == 0 or N == 0 is a
+ *     no-op; K == 0 writes C = +0.
+ *   - The first call on each device looks up the device address of the array
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents; each call clears the arrival counters on `stream`
+ *     before its kernel.  Calls whose kernels overlap on the GPU (other
+ *     streams, other host threads) race on the array and give wrong results:
+ *     serialise them.
+ * Returns GEMM_OK or a negative gemm_status. */
+GEMM_API int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_t M, int64_t N,
+                                   int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                                   gemm_stream_t stream);
 
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
 GEMM_API int gemm_abi_version(void);

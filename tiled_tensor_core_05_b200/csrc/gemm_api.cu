@@ -256,6 +256,8 @@ const char* gemm_status_string(int status) {
     case GEMM_ERR_LAUNCH: return "CUDA runtime call or kernel launch failed";
     case GEMM_ERR_WORKSPACE: return "stream-K workspace allocation failed";
     case GEMM_ERR_DEVICE_TIMEOUT: return "a device-side wait ran out of time";
+    case GEMM_ERR_SCRATCH_LIMIT:
+      return "problem too large for the fixed scratch of gemm_relu_f16_noalloc (needs M <= 32)";
     default: return "unknown status";
   }
 }
@@ -299,6 +301,28 @@ int gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, i
 int gemm_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
              int64_t lda, int64_t ldb, int64_t ldc, gemm_stream_t stream) {
   return gemm_f16_ex(A, B, C, M, N, K, lda, ldb, ldc, 0, GEMM_PATH_AUTO, stream);
+}
+
+// The allocation-free entry point: the same validation as gemm_f16_ex, then
+// the stream-K kernel with the library's fixed scratch array (see the header).
+int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_t M, int64_t N,
+                          int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                          gemm_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return GEMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return GEMM_OK;
+  if (M > 32) return GEMM_ERR_SCRATCH_LIMIT;
+  DeviceCtx d;
+  int rc = get_device(&d);
+  if (rc != GEMM_OK) return rc;
+  rc = check_matrix(C, M, N, ldc, d.device);
+  if (rc != GEMM_OK) return rc;
+  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, true, stream};
+  if (K == 0) return launch_zero_fill(p);
+  rc = check_matrix(A, M, K, lda, d.device);
+  if (rc == GEMM_OK) rc = check_matrix(B, K, N, ldb, d.device);
+  if (rc != GEMM_OK) return rc;
+  return launch_streamk_gemm_noalloc(p, d);
 }
 
 int gemm_get_device_status(gemm_stream_t stream, int* device_status) {

@@ -21,6 +21,7 @@
 //     ReLU only after the full K reduction and stores fp16.  No CTA ever waits
 //     for another one, and the result does not depend on arrival order.
 #include <atomic>
+#include <mutex>
 
 #include "../../include/gemm_f16.h"
 #include "internal.h"
@@ -407,6 +408,78 @@ int launch_streamk_gemm(const GemmProblem& p, const DeviceCtx& d, void* ws, size
     return p.relu ? launch_impl<64, 8, true>(p, d, ws, ws_bytes)
                   : launch_impl<64, 8, false>(p, d, ws, ws_bytes);
   return GEMM_ERR_INVALID_ARG;
+}
+
+// ------------------------------------------------ allocation-free variant ---
+// Scratch of gemm_relu_f16_noalloc: the same layout as the lazily allocated
+// workspace (arrival counters, then two fp32 partial tiles per CTA), sized
+// for M <= 32 (MMA N = 32) and at most kNoAllocMaxCtas CTAs.  It is part of
+// the library image, so every GPU that loads the library holds it.
+namespace {
+
+constexpr int kNoAllocMP = 32;
+constexpr int kNoAllocMaxCtas = 160;
+constexpr size_t kNoAllocCounterBytes = kCounterBytes(kNoAllocMaxCtas);
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocCounterBytes +
+    static_cast<size_t>(kNoAllocMaxCtas) * 2 * kTN * kNoAllocMP * sizeof(float);
+static_assert(kNoAllocScratchBytes == 5243648, "documented scratch size");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[64] = {};  // device address of g_noalloc_scratch, per device
+
+// Host code cannot use the array's name as a device address (it names a host
+// stand-in); look the real address up once per device, with it current.
+int noalloc_scratch_address(int device, void** out) {
+  if (device < 0 || device >= 64) return GEMM_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[device] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return GEMM_ERR_LAUNCH;
+    }
+    g_noalloc_addr[device] = p;
+  }
+  *out = g_noalloc_addr[device];
+  return GEMM_OK;
+}
+
+}  // namespace
+
+int launch_streamk_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d) {
+  if (p.M > kNoAllocMP) return GEMM_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  int rc = noalloc_scratch_address(d.device, &scratch);
+  if (rc != GEMM_OK) return rc;
+  using Cfg = SkCfg<kNoAllocMP, 10>;
+  static std::atomic<uint64_t> attr_done{0};
+  const int64_t KB = (p.K + kBK - 1) / kBK;
+  const int64_t T = (p.N + kTN - 1) / kTN;
+  const int64_t total = KB * T;
+  int64_t grid = total < d.sm_count ? total : d.sm_count;
+  if (grid > kNoAllocMaxCtas) grid = kNoAllocMaxCtas;
+  CUtensorMap tA, tB;
+  rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, kNoAllocMP);
+  if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
+  if (rc != 0) return rc;
+  auto kern = streamk_gemm_kernel<kNoAllocMP, 10, true>;
+  if (!ensure_smem_attr_sk(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
+                           attr_done))
+    return GEMM_ERR_LAUNCH;
+  // the array keeps the previous call's contents: the arrival counters must
+  // start at zero (the partial tiles are always written before being read)
+  if (cudaMemsetAsync(scratch, 0, kNoAllocCounterBytes, p.stream) != cudaSuccess)
+    return GEMM_ERR_LAUNCH;
+  int* counters = static_cast<int*>(scratch);
+  float* partials =
+      reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kNoAllocCounterBytes);
+  kern<<<static_cast<int>(grid), kThreads, Cfg::kSmemBytes, p.stream>>>(
+      tA, tB, static_cast<__half*>(p.C), static_cast<int>(p.M), static_cast<int>(p.N),
+      static_cast<int>(p.K), p.ldc, partials, counters, d.status, d.timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? GEMM_OK : GEMM_ERR_LAUNCH;
 }
 
 }  // namespace ttc

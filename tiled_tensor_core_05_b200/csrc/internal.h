@@ -42,6 +42,10 @@ int launch_streamk_gemm(const GemmProblem& p, const DeviceCtx& d, void* workspac
                         size_t workspace_bytes);
 int streamk_m_pad(int64_t M);  // MMA N used for M rows (0 if M is too large)
 
+// The stream-K kernel with its scratch in a fixed device array of the
+// library (no allocation); M <= 32.  Returns GEMM_ERR_SCRATCH_LIMIT beyond.
+int launch_streamk_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d);
+
 // Writes C = 0 (used when K == 0: the empty sum, and ReLU of it, is +0).
 int launch_zero_fill(const GemmProblem& p);
 

@@ -36,6 +36,8 @@ _SIGNATURES = {
     "gemm_selftest_wait_timeout": ([ctypes.c_int64, ctypes.c_void_p,
                                     ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
     "gemm_abi_version": ([], ctypes.c_int),
+    "gemm_relu_f16_noalloc": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
+                              ctypes.c_int),
 }
 
 
