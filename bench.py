@@ -25,7 +25,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -83,93 +82,86 @@ def traffic_for(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the GPU is busy."""
+    """SM clock, power and clock-event reasons polled through NVML (read-only
+    queries) every ~1 ms from a background thread while the GPU works."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, gpu_id: str, interval_ms: int = 20):
+    def __init__(self, gpu_uuid: str, interval_s: float = 0.001):
         self.samples = []
-        self.proc = None
         self.marks = {}
+        self.ok = False
+        self._stop = threading.Event()
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", str(interval_ms), "-i", gpu_id],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.bits = [(name, getattr(pynvml, attr)) for name, attr in self.REASONS]
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = repr(e)
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.interval = interval_s
+        self.thread = threading.Thread(target=self._run, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 8:
-                self.samples.append((time.monotonic(), parts))
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((time.monotonic(), sm, rs, pw))
+            except Exception:
+                pass
+            time.sleep(self.interval)
 
-    def wait_first(self, timeout=15.0):
+    def wait_first(self, timeout=5.0):
         t0 = time.monotonic()
-        while self.proc is not None and not self.samples and time.monotonic() - t0 < timeout:
-            time.sleep(0.02)
+        while self.ok and not self.samples and time.monotonic() - t0 < timeout:
+            time.sleep(0.005)
 
     def mark(self, name):
         self.marks[name] = time.monotonic()
 
     def stop(self):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self.ok:
+            self.thread.join(timeout=2)
 
     def summary(self, start="t0", end="t1"):
-        if self.proc is None or not self.samples:
+        if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
-                    "note": "nvidia-smi unavailable"}
-        t0, t1 = self.marks.get(start, 0), self.marks.get(end, 1e30)
-        inside = [p for (t, p) in self.samples if t0 <= t <= t1 + 0.05]
-        note = "samples taken during the timed region"
-        if not inside:
-            # a timed region shorter than the sampling interval: use the
-            # samples of the surrounding busy period (warm-up included)
+                    "note": "NVML unavailable: " + getattr(self, "err", "")}
+        t0, t1 = self.marks.get(start, 0.0), self.marks.get(end, 1e30)
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "NVML samples taken during the timed region"
+        if len(inside) < 3:
             w0 = self.marks.get("warm0", t0)
-            inside = [p for (t, p) in self.samples if w0 <= t <= t1 + 0.1]
-            note = "timed region shorter than the sampling interval; warm-up + timed samples"
+            inside = [s for s in self.samples if w0 <= s[0] <= t1]
+            note = "timed region too short for 3 samples; warm-up + timed samples"
         if not inside:
-            inside = [self.samples[-1][1]]
-            note = "no sample inside the busy period; last sample"
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(p[0]) for p in inside if num(p[0]) is not None]
-        smax = [num(p[1]) for p in inside if num(p[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for p in inside for i in range(4)
-                          if p[4 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(inside),
-                "power_w_max": max((num(p[2]) or 0.0) for p in inside), "note": note}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": "no sample during the busy period"}
+        reasons = sorted({name for s in inside for name, bit in self.bits if s[2] & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in inside),
+                "sm_mhz_min": min(s[1] for s in inside),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
+                "power_w_max": round(max(s[3] for s in inside), 1), "note": note}
 
 
 def gpu_id_for(dev_index: int) -> str:
+    """NVML UUID string ("GPU-...") of a torch device index."""
     import torch
-    try:
-        u = torch.cuda.get_device_properties(dev_index).uuid
-        s = str(u)
-        return s if s.startswith("GPU-") else "GPU-" + s
-    except Exception:
-        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-        if vis:
-            return vis.split(",")[dev_index]
-        return str(dev_index)
+    s = str(torch.cuda.get_device_properties(dev_index).uuid)
+    return s if s.startswith("GPU-") else "GPU-" + s
 
 
 # ----------------------------------------------------------- measurements ---
@@ -395,8 +387,10 @@ def run_ours(args):
         line["pct_of_dense_fp16_peak"] = round(100 * value / world / NOMINAL_FP16_TFLOPS, 2)
     line["roofline"] = roofline_entry(args.workload, main["launch_ms"], peaks, peak_src,
                                       long_run)
-    line["roofline"]["kernel"] = ("streamk_gemm_kernel" if args.workload == "decode"
-                                  else "tile_gemm_kernel")
+    path = ops.select_path(w.M, w.N, w.K)
+    line["roofline"]["kernel"] = {ops.PATH_STREAMK: "streamk_gemm_kernel",
+                                  ops.PATH_TILE: "tile_gemm_kernel",
+                                  ops.PATH_TILE_PAIR: "tile_pair_gemm_kernel"}[path]
     if "e2e_ms" in main:
         e_ms = main["e2e_ms"]
         ev = (w.flops / (e_ms * 1e-3) / 1e12) if unit == "TFLOP/s" else \

@@ -67,9 +67,12 @@ enum gemm_status {
 };
 
 enum gemm_path {
-  GEMM_PATH_AUTO = 0,   /* choose by shape: M <= 64 -> STREAMK, else TILE */
-  GEMM_PATH_TILE = 1,   /* persistent 128 x BN tile kernel (any shape) */
-  GEMM_PATH_STREAMK = 2 /* swap-AB stream-K kernel (M <= 64 only) */
+  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> STREAMK; at least 64 tiles of
+                              256 x 256 -> TILE_PAIR; otherwise TILE */
+  GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile (any shape) */
+  GEMM_PATH_STREAMK = 2,   /* swap-AB stream-K kernel (M <= 64 only) */
+  GEMM_PATH_TILE_PAIR = 3  /* persistent kernel, two SMs (a CTA pair) per 256 x 256 tile
+                              (any shape) */
 };
 
 /* C = ReLU(A @ B).  "Escribamos un GEMM": the tiled fp16 matmul with the

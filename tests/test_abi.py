@@ -57,7 +57,9 @@ def test_path_selection(lib):
     assert ops.select_path(32, 28672, 8192) == ops.PATH_STREAMK
     assert ops.select_path(64, 100, 100) == ops.PATH_STREAMK
     assert ops.select_path(65, 100, 100) == ops.PATH_TILE
-    assert ops.select_path(8192, 8192, 8192) == ops.PATH_TILE
+    assert ops.select_path(1024, 1024, 1024) == ops.PATH_TILE
+    assert ops.select_path(8192, 8192, 8192) == ops.PATH_TILE_PAIR
+    assert ops.select_path(8192, 14336, 4096) == ops.PATH_TILE_PAIR
 
 
 def test_abi_version(lib):

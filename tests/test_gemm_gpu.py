@@ -19,7 +19,7 @@ from tiled_tensor_core_05_b200 import ops, workloads
 
 pytestmark = pytest.mark.gpu
 
-TILE, STREAMK = ops.PATH_TILE, ops.PATH_STREAMK
+TILE, STREAMK, PAIR = ops.PATH_TILE, ops.PATH_STREAMK, ops.PATH_TILE_PAIR
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -54,10 +54,11 @@ def run(a_cpu, b_cpu, relu=True, path=ops.PATH_AUTO, lda=None, ldb=None, ldc=Non
 
 @pytest.mark.parametrize("name", ["cube256", "cube1024", "ragged1000"])
 @pytest.mark.parametrize("relu", [True, False])
-def test_workload_full(oracle_mod, name, relu):
+@pytest.mark.parametrize("path", [ops.PATH_AUTO, TILE, PAIR], ids=["auto", "tile", "pair"])
+def test_workload_full(oracle_mod, name, relu, path):
     a, b = workloads.workload_inputs(name)
     ref = oracle_mod.gemm_relu(a, b) if relu else oracle_mod.gemm(a, b)
-    c = run(a, b, relu=relu)
+    c = run(a, b, relu=relu, path=path)
     check_parity(c, ref, relu, name)
 
 
@@ -79,10 +80,21 @@ GRID = [(m, n, k) for m in EDGE for n in EDGE for k in EDGE
 
 
 @pytest.mark.parametrize("m,n,k", GRID)
-def test_ragged_grid_tile(oracle_mod, m, n, k):
+@pytest.mark.parametrize("path", [TILE, PAIR], ids=["tile", "pair"])
+def test_ragged_grid_tile(oracle_mod, m, n, k, path):
     a, b = workloads.make_inputs(m, n, k, seed=1000 + m + 7 * n + 13 * k)
     ref = oracle_mod.gemm_relu(a, b)
-    check_parity(run(a, b, path=TILE), ref, True, f"tile {m}x{n}x{k}")
+    check_parity(run(a, b, path=path), ref, True, f"path {path} {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("m,n,k", [(600, 1100, 700), (513, 257, 1030), (2048, 2048, 512),
+                                   (4000, 300, 96)])
+def test_pair_kernel_multi_tile(oracle_mod, m, n, k):
+    """Several 256 x 256 pair tiles per CTA pair, ragged in every dimension."""
+    a, b = workloads.make_inputs(m, n, k, seed=3000 + m + n + k)
+    for relu in (True, False):
+        ref = oracle_mod.gemm_relu(a, b) if relu else oracle_mod.gemm(a, b)
+        check_parity(run(a, b, relu=relu, path=PAIR), ref, relu, f"pair {m}x{n}x{k}")
 
 
 @pytest.mark.parametrize("m,n,k", [(m, n, k) for (m, n, k) in GRID if m <= 64] +
@@ -94,7 +106,7 @@ def test_ragged_grid_streamk(oracle_mod, m, n, k):
         check_parity(run(a, b, relu=relu, path=STREAMK), ref, relu, f"stream-K {m}x{n}x{k}")
 
 
-@pytest.mark.parametrize("path", [TILE, STREAMK])
+@pytest.mark.parametrize("path", [TILE, STREAMK, PAIR])
 def test_padded_leading_dimensions(oracle_mod, path):
     m, n, k = 45, 300, 190
     a, b = workloads.make_inputs(m, n, k, seed=5)
@@ -118,7 +130,7 @@ def gpu_fn_for(path):
 
 
 @pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
-@pytest.mark.parametrize("path", [TILE, STREAMK], ids=["tile", "streamk"])
+@pytest.mark.parametrize("path", [TILE, STREAMK, PAIR], ids=["tile", "streamk", "pair"])
 def test_pins_on_gpu(pin, path):
     fails = pin(gpu_fn_for(path), exact=False)
     assert not fails, "\n".join(fails[:5])
@@ -168,7 +180,7 @@ def test_workload_fullsize_sampled(oracle_mod, name):
 
 # ------------------------------------------------------------ special cases ---
 
-@pytest.mark.parametrize("path", [ops.PATH_AUTO, TILE])
+@pytest.mark.parametrize("path", [ops.PATH_AUTO, TILE, PAIR])
 def test_k_zero_writes_zeros(path):
     a = torch.empty((5, 0), dtype=torch.float16, device="cuda")
     b = torch.empty((0, 9), dtype=torch.float16, device="cuda")
@@ -189,7 +201,7 @@ def test_empty_output_is_noop():
 def test_deterministic_bits_both_paths():
     a, b = workloads.make_inputs(64, 3000, 2500, seed=9)
     ad, bd = to_dev(a, round8(2500)), to_dev(b)
-    for path in (TILE, STREAMK):
+    for path in (TILE, STREAMK, PAIR):
         outs = []
         for _ in range(3):
             outs.append(ops.gemm_f16_ex(ad, bd, relu=True, path=path).view(torch.int16).cpu())

@@ -242,9 +242,10 @@ extern "C" {
 int gemm_abi_version(void) { return 10000; }
 
 int gemm_select_path(int64_t M, int64_t N, int64_t K) {
-  (void)N;
   (void)K;
-  return (M >= 1 && M <= 64) ? GEMM_PATH_STREAMK : GEMM_PATH_TILE;
+  if (M >= 1 && M <= 64) return GEMM_PATH_STREAMK;
+  const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  return pair_tiles >= 64 ? GEMM_PATH_TILE_PAIR : GEMM_PATH_TILE;
 }
 
 const char* gemm_status_string(int status) {
@@ -268,7 +269,8 @@ int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int
   if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return GEMM_ERR_INVALID_ARG;
   if (relu != 0 && relu != 1) return GEMM_ERR_INVALID_ARG;
-  if (path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE && path != GEMM_PATH_STREAMK)
+  if (path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE && path != GEMM_PATH_STREAMK &&
+      path != GEMM_PATH_TILE_PAIR)
     return GEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return GEMM_OK;
   DeviceCtx d;
@@ -290,6 +292,7 @@ int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int
     if (rc != GEMM_OK) return rc;
     return launch_streamk_gemm(p, d, ws, ws_bytes);
   }
+  if (path == GEMM_PATH_TILE_PAIR) return launch_tile_pair_gemm(p, d);
   return launch_tile_gemm(p, d);
 }
 

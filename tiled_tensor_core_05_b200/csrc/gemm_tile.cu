@@ -56,6 +56,25 @@ struct TileCfg {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
+// The CTA-pair kernel: a 256 x 256 output tile per pair of SMs.  Each CTA
+// stages its own 128 rows of A and its own 128 columns of B per k-block, and
+// keeps its 128 accumulator rows x 256 columns in its TMEM.
+template <int STAGES>
+struct PairCfg {
+  static constexpr int kBN = 256;                 // pair tile columns
+  static constexpr int kABytes = kBM * kBK * 2;   // this CTA's 128 rows
+  static constexpr int kBChunk = kBK * 64 * 2;
+  static constexpr int kBBytes = kBK * 128 * 2;   // this CTA's 128 columns
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiBuf;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
+  static constexpr uint32_t kTmemCols = 512;      // two 256-column accumulators
+  static constexpr uint32_t kIdesc = idesc_f16_f32(2 * kBM, kBN, /*A MN-major*/ false,
+                                                   /*B MN-major*/ true);
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
 // Grouped-panel rasterisation: consecutive tile indices sweep group_m
 // tile-rows of one panel column by column, so the CTAs that run at the same
 // time share A rows and B columns in L2.
@@ -68,6 +87,76 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
   const int r = tile - g * per_group;
   mb = first_m + r % rows;
   nb = r / rows;
+}
+
+// Epilogue of one accumulator tile, run by one warp for its 32 TMEM lanes:
+// tcgen05.ld 64 columns at a time -> ReLU in fp32 -> RNE to fp16 -> 128-byte
+// swizzled staging row per thread -> TMA store of a 32 x 64 box (double
+// buffered per warp).  Columns at and beyond N rounded down to 8 (the TMA
+// store writes whole 16-byte groups) are written with plain stores.
+// `release()` runs once the last TMEM load of the tile has completed.
+template <int BN, bool RELU, class Release>
+__device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uint32_t& chunk_no,
+                                              const CUtensorMap* tmC, __half* C, int64_t ldc,
+                                              int M, int N, int n8, int row0, int col_base,
+                                              int lane, Release release) {
+#pragma unroll 1
+  for (int c = 0; c < BN / kEpiCols; ++c) {
+    uint32_t v0[32], v1[32];
+    tmem_ld_32x32b_x32(t_row + c * kEpiCols, v0);
+    tmem_ld_32x32b_x32(t_row + c * kEpiCols + 32, v1);
+    tmem_wait_ld();
+    if (c == BN / kEpiCols - 1) {
+      // the accumulator has been read: hand it back to the MMA issuer
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) release();
+    }
+    uint32_t h[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float x0 = __uint_as_float(v0[2 * i]), x1 = __uint_as_float(v0[2 * i + 1]);
+      float y0 = __uint_as_float(v1[2 * i]), y1 = __uint_as_float(v1[2 * i + 1]);
+      if (RELU) {
+        x0 = relu_f32(x0);
+        x1 = relu_f32(x1);
+        y0 = relu_f32(y0);
+        y1 = relu_f32(y1);
+      }
+      h[i] = pack_half2(x0, x1);
+      h[16 + i] = pack_half2(y0, y1);
+    }
+    uint8_t* buf = bufs + (chunk_no & 1u) * kEpiBuf;
+    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+    __syncwarp();
+    // row `lane`, 128 bytes = 8 chunks of 16 bytes, chunk j stored at j ^ (row & 7)
+    const uint32_t row_addr = smem_u32(buf) + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), h[4 * j], h[4 * j + 1], h[4 * j + 2],
+                   h[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    const int col0 = col_base + c * kEpiCols;
+    if (lane == 0) {
+      if (row0 < M && col0 < n8) tma_store_2d(tmC, buf, col0, row0);
+      bulk_commit_group();
+    }
+    if (n8 < N && col0 + kEpiCols > n8 && col0 < N && row0 + lane < M) {
+      // ragged tail columns [max(n8, col0), min(N, col0 + 64)) of this row,
+      // read back from this thread's own (swizzled) staging row
+      const int j_end = min(N, col0 + kEpiCols);
+      __half* crow = C + static_cast<int64_t>(row0 + lane) * ldc;
+      for (int j = max(n8, col0); j < j_end; ++j) {
+        const int cc = j - col0;
+        const uint32_t addr = row_addr + ((((cc >> 3) ^ (lane & 7)) << 4) | ((cc & 7) << 1));
+        unsigned short bits;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(bits) : "r"(addr) : "memory");
+        crow[j] = __ushort_as_half(bits);
+      }
+    }
+    ++chunk_no;
+  }
 }
 
 template <int BN, int STAGES, bool RELU>
@@ -239,63 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = mb * kBM + q * kEpiRows;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-#pragma unroll 1
-      for (int c = 0; c < BN / kEpiCols; ++c) {
-        uint32_t v0[32], v1[32];
-        tmem_ld_32x32b_x32(t_row + c * kEpiCols, v0);
-        tmem_ld_32x32b_x32(t_row + c * kEpiCols + 32, v1);
-        tmem_wait_ld();
-        if (c == BN / kEpiCols - 1) {
-          // the accumulator has been read: hand it back to the MMA warp
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        }
-        uint32_t h[32];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0 = __uint_as_float(v0[2 * i]), x1 = __uint_as_float(v0[2 * i + 1]);
-          float y0 = __uint_as_float(v1[2 * i]), y1 = __uint_as_float(v1[2 * i + 1]);
-          if (RELU) {
-            x0 = relu_f32(x0);
-            x1 = relu_f32(x1);
-            y0 = relu_f32(y0);
-            y1 = relu_f32(y1);
-          }
-          h[i] = pack_half2(x0, x1);
-          h[16 + i] = pack_half2(y0, y1);
-        }
-        uint8_t* buf = bufs + (chunk_no & 1u) * kEpiBuf;
-        if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
-        __syncwarp();
-        // row `lane`, 128 bytes = 8 chunks of 16 bytes, chunk j stored at j ^ (row & 7)
-        const uint32_t row_addr = smem_u32(buf) + lane * 128;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), h[4 * j], h[4 * j + 1], h[4 * j + 2],
-                       h[4 * j + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        const int col0 = nb * BN + c * kEpiCols;
-        if (lane == 0) {
-          if (row0 < M && col0 < n8) tma_store_2d(&tmC, buf, col0, row0);
-          bulk_commit_group();
-        }
-        if (n8 < N && col0 + kEpiCols > n8 && col0 < N && row0 + lane < M) {
-          // ragged tail columns [max(n8, col0), min(N, col0 + 64)) of this row,
-          // read back from this thread's own (swizzled) staging row
-          const int j_end = min(N, col0 + kEpiCols);
-          __half* crow = C + static_cast<int64_t>(row0 + lane) * ldc;
-          for (int j = max(n8, col0); j < j_end; ++j) {
-            const int cc = j - col0;
-            const uint32_t addr = row_addr + ((((cc >> 3) ^ (lane & 7)) << 4) | ((cc & 7) << 1));
-            unsigned short bits;
-            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(bits) : "r"(addr) : "memory");
-            crow[j] = __ushort_as_half(bits);
-          }
-        }
-        ++chunk_no;
-      }
+      uint64_t* release_bar = &acc_empty[acc];
+      epilogue_tile<BN, RELU>(t_row, bufs, chunk_no, &tmC, C, ldc, M, N, n8, row0, nb * BN,
+                              lane, [release_bar] { mbar_arrive(release_bar); });
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -312,6 +347,223 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Busy-wait for about `ns` nanoseconds (bounded, used on the abort path only).
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < ns) {
+  }
+}
+
+// CTA-pair kernel.  Launched with clusters of 2 CTAs; cluster rank 0 (the
+// "leader") issues the tcgen05.mma.cta_group::2 for both SMs.
+//   * both producers load their halves into their own shared memory and count
+//     the bytes on the leader's full[stage] barrier (armed by the leader for
+//     both halves);
+//   * the leader's commit frees stage s in both CTAs and tells both epilogues
+//     that an accumulator is ready (multicast arrive);
+//   * each CTA's four epilogue warps drain its own TMEM rows and arrive on the
+//     leader's acc_empty barrier (8 arrivals per accumulator use).
+template <int STAGES, bool RELU>
+__global__ void __launch_bounds__(kThreads, 1)
+    tile_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                          const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
+                          int64_t ldc, int M, int N, int K, int group_m, int* status,
+                          uint64_t timeout_ns) {
+  using Cfg = PairCfg<STAGES>;
+  constexpr int BN = Cfg::kBN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + STAGES * Cfg::kABytes;
+  uint8_t* smEpi = smem + STAGES * Cfg::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smEpi + Cfg::kEpiBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(num_clusters_x());
+  const int num_m = (M + 2 * kBM - 1) / (2 * kBM);
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + kBK - 1) / kBK;
+  const int n8 = N & ~7;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish_alloc_permit_pair();
+  }
+  tc_fence_before_sync();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM of both SMs allocated
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  // the leader's barriers, as addresses this CTA can signal
+  const uint32_t full_leader = map_to_cta(smem_u32(full), 0);
+  const uint32_t acc_empty_leader = map_to_cta(smem_u32(acc_empty), 0);
+
+  if (warp == 0) {
+    // --------------------------------------------- TMA producer (both CTAs) ---
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, group_m, mb, nb);
+        const int a_row = mb * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int b_col = nb * BN + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
+          const uint32_t bar = full_leader + stage * 8;
+          tma_load_2d_pair(&tmA, bar, smA + stage * Cfg::kABytes, kb * kBK, a_row);
+          uint8_t* bdst = smB + stage * Cfg::kBBytes;
+          tma_load_2d_pair(&tmB, bar, bdst, b_col, kb * kBK);
+          tma_load_2d_pair(&tmB, bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleProducer << 4) | 3);
+        if (leader) {
+          for (int s = 0; s < STAGES; ++s)
+            if (armed & (1u << s))
+              (void)mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, timeout_ns);
+        } else {
+          // this CTA's loads complete on the leader's barriers, which it cannot
+          // poll; give loads already issued ample time to land
+          spin_ns(2000000);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer (leader) ---
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      int site = 0;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
+          ok = false;
+          site = 5;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
+            ok = false;
+            site = 6;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_u32(smA + stage * Cfg::kABytes);
+          const uint32_t b_addr = smem_u32(smB + stage * Cfg::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k) {
+            const uint64_t adesc = smem_desc_sw128(a_addr + k * (kUmmaK * 2), 16, 1024);
+            const uint64_t bdesc =
+                smem_desc_sw128(b_addr + k * (kUmmaK * 128), Cfg::kBChunk, 1024);
+            umma_f16_pair(d_tmem, adesc, bdesc, Cfg::kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair(&empty[stage], 0x3);  // stage s free in both CTAs
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&acc_full[acc], 0x3);  // both epilogues may read
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleMma << 4) | site);
+        umma_commit_pair(drain, 0x1);
+        (void)mbar_wait(drain, 0, nullptr, timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (both CTAs) ---
+    const int q = warp & 3;
+    uint8_t* bufs = smEpi + (warp - 2) * 2 * kEpiBuf;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    uint32_t chunk_no = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs) {
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, group_m, mb, nb);
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, timeout_ns) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0)
+          raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleEpilogue << 4) | 3);
+        break;
+      }
+      tc_fence_after_sync();
+      const int row0 = mb * 2 * kBM + static_cast<int>(rank) * kBM + q * kEpiRows;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      const uint32_t release_bar = acc_empty_leader + acc * 8;
+      epilogue_tile<BN, RELU>(t_row, bufs, chunk_no, &tmC, C, ldc, M, N, n8, row0, nb * BN,
+                              lane, [release_bar] { mbar_arrive_cluster(release_bar); });
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before_sync();
+  // no CTA of the pair leaves (or frees TMEM) while the other may still signal
+  // its barriers or use its TMEM
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+  }
+}
+
 // Sets the dynamic shared-memory limit of a kernel once per device.
 bool ensure_smem_attr(const void* func, int bytes, int device, std::atomic<uint64_t>& done) {
   const uint64_t bit = 1ull << (device & 63);
@@ -323,13 +575,19 @@ bool ensure_smem_attr(const void* func, int bytes, int device, std::atomic<uint6
   return true;
 }
 
-int group_m_setting() {
+// Rows of A per raster panel (TTC_GROUP_ROWS overrides it for tuning sweeps).
+int group_rows_setting() {
   static const int g = [] {
-    const char* s = std::getenv("TTC_GROUP_M");
+    const char* s = std::getenv("TTC_GROUP_ROWS");
     const int v = s ? std::atoi(s) : 0;
-    return v > 0 ? v : 8;
+    return v > 0 ? v : 2048;
   }();
   return g;
+}
+
+int group_tiles(int tile_rows) {
+  const int g = group_rows_setting() / tile_rows;
+  return g > 0 ? g : 1;
 }
 
 template <int BN, int STAGES, bool RELU>
@@ -353,8 +611,55 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   kern<<<grid, kThreads, Cfg::kSmemBytes, p.stream>>>(
       tA, tB, tC, static_cast<__half*>(p.C), p.ldc, static_cast<int>(p.M),
       static_cast<int>(p.N), static_cast<int>(p.K),
-      group_m_setting(), d.status, d.timeout_ns);
+      group_tiles(kBM), d.status, d.timeout_ns);
   return cudaGetLastError() == cudaSuccess ? 0 : GEMM_ERR_LAUNCH;
+}
+
+template <int STAGES, bool RELU>
+int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
+  using Cfg = PairCfg<STAGES>;
+  static std::atomic<uint64_t> attr_done{0};
+  static int max_pairs[64] = {};
+  CUtensorMap tA, tB, tC;
+  int rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, kBM);
+  if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
+  const uint64_t n8 = static_cast<uint64_t>(p.N) & ~7ull;
+  if (rc == 0) rc = encode_tmap_f16_2d(&tC, p.C, n8 > 0 ? n8 : 8, p.M, p.ldc, kEpiCols, kEpiRows);
+  if (rc != 0) return rc;
+  auto kern = tile_pair_gemm_kernel<STAGES, RELU>;
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
+                        attr_done))
+    return GEMM_ERR_LAUNCH;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = p.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // pairs that can be resident at once (GPC layout may leave an SM unpaired)
+  int& resident = max_pairs[d.device & 63];
+  if (resident == 0) {
+    cfg.gridDim = dim3(2 * (d.sm_count / 2), 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = d.sm_count / 2;
+    }
+    resident = n;
+  }
+  const int64_t num_tiles = ((p.M + 2 * kBM - 1) / (2 * kBM)) * ((p.N + 255) / 256);
+  const int pairs = static_cast<int>(num_tiles < resident ? num_tiles : resident);
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc, static_cast<int>(p.M),
+      static_cast<int>(p.N), static_cast<int>(p.K), group_tiles(2 * kBM), d.status,
+      d.timeout_ns);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
 }  // namespace
@@ -366,6 +671,10 @@ int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d) {
   const bool wide = tiles256 >= d.sm_count;
   if (wide) return p.relu ? launch_impl<256, 4, true>(p, d) : launch_impl<256, 4, false>(p, d);
   return p.relu ? launch_impl<128, 6, true>(p, d) : launch_impl<128, 6, false>(p, d);
+}
+
+int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d) {
+  return p.relu ? launch_pair_impl<6, true>(p, d) : launch_pair_impl<6, false>(p, d);
 }
 
 }  // namespace ttc

@@ -31,8 +31,11 @@ struct DeviceCtx {
 int encode_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t ld, uint32_t box_inner, uint32_t box_outer);
 
-// Large-shape path: persistent warp-specialised tcgen05 kernel.
+// Large-shape path: persistent warp-specialised tcgen05 kernel, one SM per
+// 128-row tile ...
 int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d);
+// ... or a pair of SMs per 256 x 256 tile (tcgen05.mma.cta_group::2).
+int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d);
 
 // Small-M path: swap-AB stream-K kernel.  `workspace` holds partial tiles and
 // per-tile arrival counters (counters must be zero on entry; the kernel
