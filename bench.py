@@ -38,7 +38,7 @@ NOMINAL_FP16_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["tiled_tensor_core_05_b200/csrc/gemm_tile.cu",
-                  "tiled_tensor_core_05_b200/csrc/gemm_streamk.cu",
+                  "tiled_tensor_core_05_b200/csrc/gemm_skinny.cu",
                   "tiled_tensor_core_05_b200/csrc/sm100.cuh"]
 
 
@@ -204,7 +204,8 @@ def time_launches(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
     return total, sum(per) / len(per)
 
 
-def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True):
+def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
+                     comparator=False):
     import torch
 
     from tiled_tensor_core_05_b200 import ops, workloads
@@ -227,6 +228,13 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True):
     if st != 0:
         raise RuntimeError(f"device reported status {st:#x}")
     res = {"total_ms": total_ms, "launch_ms": launch_ms, "w": w}
+    if comparator:
+        # context only, never on the measured path: cuBLAS through torch on
+        # the same inputs, timed the same way right after our kernel
+        def torch_step():
+            torch.relu_(torch.matmul(a, b, out=c))
+        _, t_ms = time_launches(torch_step, steps, warmup, stream, None, None)
+        res["torch_launch_ms"] = t_ms
     if e2e:
         # end to end through the C ABI: pinned host inputs -> device, the
         # kernel, result -> pinned host, every step
@@ -366,7 +374,7 @@ def run_ours(args):
     sampler = ClockSampler(gpu_id_for(local))
     sampler.wait_first()
     main = measure_workload(args.workload, args.steps, args.warmup, dist, sampler,
-                            e2e=not args.no_e2e)
+                            e2e=not args.no_e2e, comparator=not args.no_comparator)
     sampler.stop()
     clocks = sampler.summary()
     w = main["w"]
@@ -388,7 +396,7 @@ def run_ours(args):
     line["roofline"] = roofline_entry(args.workload, main["launch_ms"], peaks, peak_src,
                                       long_run)
     path = ops.select_path(w.M, w.N, w.K)
-    line["roofline"]["kernel"] = {ops.PATH_STREAMK: "streamk_gemm_kernel",
+    line["roofline"]["kernel"] = {ops.PATH_SKINNY: "skinny_gemm_kernel",
                                   ops.PATH_TILE: "tile_gemm_kernel",
                                   ops.PATH_TILE_PAIR: "tile_pair_gemm_kernel"}[path]
     if "e2e_ms" in main:
@@ -399,18 +407,28 @@ def run_ours(args):
                        "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"],
                        "ms_per_step": round(e_ms, 4)}
     line["clocks"] = clocks
+    if "torch_launch_ms" in main:
+        t_ms = main["torch_launch_ms"]
+        line["context_torch_matmul_relu"] = {
+            "what": "torch.relu(torch.matmul(a, b)) (cuBLAS fp16 + a separate ReLU kernel), "
+                    "same inputs and timing; context only, not on the measured path",
+            "ms_per_call": round(t_ms, 5),
+            "tflops": round(w.flops / (t_ms * 1e-3) / 1e12, 2) if unit == "TFLOP/s" else None,
+            "gbs": round(w.bytes_min / (t_ms * 1e-3) / 1e9, 1) if unit == "GB/s" else None}
     if rank == 0 and not args.no_secondary:
         others = []
         for name in ("mlp_up", "decode", "cube1024", "cube256"):
             if name == args.workload:
                 continue
             r = measure_workload(name, max(args.steps, 20), max(args.warmup, 3), None, None,
-                                 e2e=False)
+                                 e2e=False, comparator=not args.no_comparator)
             ow = r["w"]
             entry = {"workload": name, "M": ow.M, "N": ow.N, "K": ow.K,
                      "ms_per_launch": round(r["launch_ms"], 5),
                      "tflops": round(ow.flops / (r["launch_ms"] * 1e-3) / 1e12, 2),
                      "roofline": roofline_entry(name, r["launch_ms"], peaks, peak_src, False)}
+            if "torch_launch_ms" in r:
+                entry["context_torch_ms_per_call"] = round(r["torch_launch_ms"], 5)
             if name == "decode":
                 entry["gbs"] = round(ow.bytes_min / (r["launch_ms"] * 1e-3) / 1e9, 1)
                 entry["pct_of_nominal_hbm"] = round(100 * entry["gbs"] / NOMINAL_HBM_GBS, 2)
@@ -440,6 +458,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparator", action="store_true",
+                    help="skip timing torch.matmul + relu as a context comparator")
     ap.add_argument("--cpu-budget", type=float, default=10.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     args = ap.parse_args(argv)

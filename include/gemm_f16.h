@@ -30,7 +30,7 @@
  *     a per-device status word, read with gemm_get_device_status().
  *   - Results are deterministic: the same inputs give the same bits on every
  *     run, whatever the scheduling.
- *   - Small-M problems (M <= 64) use a stream-K path whose fp32 partial tiles
+ *   - Small-M problems (M <= 64) use a split-K path whose fp32 partial tiles
  *     and arrival counters live in a workspace the library allocates once per
  *     (device, stream) on first use (cudaMalloc; about 10 MB on a 148-SM GPU)
  *     and keeps until process exit.  Make that first call outside CUDA-graph
@@ -61,16 +61,17 @@ enum gemm_status {
   GEMM_ERR_ALIGNMENT = -2,          /* pointer not 16-byte aligned or ld % 8 != 0 */
   GEMM_ERR_UNSUPPORTED_DEVICE = -3, /* current device is not compute capability 10.0 */
   GEMM_ERR_LAUNCH = -4,             /* a CUDA runtime call or kernel launch failed */
-  GEMM_ERR_WORKSPACE = -5,          /* workspace allocation failed */
+  GEMM_ERR_WORKSPACE = -5,          /* small-M workspace allocation failed */
   GEMM_ERR_DEVICE_TIMEOUT = -6,     /* reported by gemm_get_device_status */
   GEMM_ERR_SCRATCH_LIMIT = -7       /* problem too large for gemm_relu_f16_noalloc's fixed scratch */
 };
 
 enum gemm_path {
-  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> STREAMK; at least 64 tiles of
+  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY; at least 64 tiles of
                               256 x 256 -> TILE_PAIR; otherwise TILE */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile (any shape) */
-  GEMM_PATH_STREAMK = 2,   /* swap-AB stream-K kernel (M <= 64 only) */
+  GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 256 columns of B per CTA streamed
+                              in lock-step, split-K only when tiles < SMs (M <= 64 only) */
   GEMM_PATH_TILE_PAIR = 3  /* persistent kernel, two SMs (a CTA pair) per 256 x 256 tile
                               (any shape) */
 };
@@ -86,14 +87,14 @@ GEMM_API int gemm_f16(const void* A, const void* B, void* C, int64_t M, int64_t 
              int64_t lda, int64_t ldb, int64_t ldc, gemm_stream_t stream);
 
 /* Either of the above with an explicit kernel choice.  relu: 0 or 1.  path:
- * a gemm_path value; GEMM_PATH_STREAMK with M > 64 returns
+ * a gemm_path value; GEMM_PATH_SKINNY with M > 64 returns
  * GEMM_ERR_INVALID_ARG. */
 GEMM_API int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
                 int64_t lda, int64_t ldb, int64_t ldc, int relu, int path,
                 gemm_stream_t stream);
 
-/* The path GEMM_PATH_AUTO takes for this shape (GEMM_PATH_TILE or
- * GEMM_PATH_STREAMK).  Pure host function. */
+/* The path GEMM_PATH_AUTO takes for this shape (GEMM_PATH_TILE,
+ * GEMM_PATH_TILE_PAIR or GEMM_PATH_SKINNY).  Pure host function. */
 GEMM_API int gemm_select_path(int64_t M, int64_t N, int64_t K);
 
 /* Human-readable text for a gemm_status value (static storage). */
@@ -103,7 +104,7 @@ GEMM_API const char* gemm_status_string(int status);
  * current device: *device_status = 0 if every kernel finished normally, else
  * the code of the first bounded wait that gave up (non-zero; the kernel that
  * gave up returned without completing its output).  After a non-zero status
- * the stream-K workspaces of the device are re-zeroed.  Returns GEMM_OK, or
+ * the small-M workspaces of the device are re-zeroed.  Returns GEMM_OK, or
  * GEMM_ERR_LAUNCH if a CUDA call failed. */
 GEMM_API int gemm_get_device_status(gemm_stream_t stream, int* device_status);
 
@@ -119,12 +120,12 @@ GEMM_API int gemm_selftest_wait_timeout(int64_t timeout_ns, gemm_stream_t stream
  *
  * No counterpart in the pages: this is an interface addition, not part of the
  * method.  gemm_relu_f16 lazily cudaMalloc's a workspace for its small-M
- * (stream-K) kernel on the first call per (device, stream).  Some callers
+ * (split-K) kernel on the first call per (device, stream).  Some callers
  * cannot allow that: plugins whose enqueue step is forbidden to allocate,
  * processes whose device memory is owned and accounted for by a pool
  * allocator, and latency-critical loops where cudaMalloc's implicit device
  * synchronisation would stall other work.  This entry point runs the same
- * stream-K kernel, but keeps its scratch (fp32 partial tiles and per-tile
+ * small-M kernel, but keeps its scratch (fp32 partial tiles and per-tile
  * arrival counters) in a fixed array that is part of the library image: every
  * GPU that loads the library holds those 5,243,648 bytes (5 MiB) until the
  * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.

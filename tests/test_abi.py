@@ -54,8 +54,8 @@ def test_status_strings(lib):
 
 def test_path_selection(lib):
     from tiled_tensor_core_05_b200 import ops
-    assert ops.select_path(32, 28672, 8192) == ops.PATH_STREAMK
-    assert ops.select_path(64, 100, 100) == ops.PATH_STREAMK
+    assert ops.select_path(32, 28672, 8192) == ops.PATH_SKINNY
+    assert ops.select_path(64, 100, 100) == ops.PATH_SKINNY
     assert ops.select_path(65, 100, 100) == ops.PATH_TILE
     assert ops.select_path(1024, 1024, 1024) == ops.PATH_TILE
     assert ops.select_path(8192, 8192, 8192) == ops.PATH_TILE_PAIR

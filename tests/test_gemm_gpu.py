@@ -19,7 +19,7 @@ from tiled_tensor_core_05_b200 import ops, workloads
 
 pytestmark = pytest.mark.gpu
 
-TILE, STREAMK, PAIR = ops.PATH_TILE, ops.PATH_STREAMK, ops.PATH_TILE_PAIR
+TILE, SKINNY, PAIR = ops.PATH_TILE, ops.PATH_SKINNY, ops.PATH_TILE_PAIR
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -63,13 +63,13 @@ def test_workload_full(oracle_mod, name, relu, path):
 
 
 @pytest.mark.parametrize("name", ["cube256", "ragged1000"])
-def test_workload_full_streamk_path(oracle_mod, name):
-    """The stream-K kernel on the first 64 / 32 rows of the small workloads."""
+def test_workload_full_skinny_path(oracle_mod, name):
+    """The small-M kernel on the first 64 / 32 rows of the small workloads."""
     a, b = workloads.workload_inputs(name)
     for m in (64, 32, 1):
         ref = oracle_mod.gemm_relu(a[:m], b)
-        c = run(a[:m].contiguous(), b, relu=True, path=STREAMK)
-        check_parity(c, ref, True, f"{name}[:{m}] stream-K")
+        c = run(a[:m].contiguous(), b, relu=True, path=SKINNY)
+        check_parity(c, ref, True, f"{name}[:{m}] small-M")
 
 
 # ------------------------------------------------ ragged shape grid, both paths ---
@@ -98,15 +98,16 @@ def test_pair_kernel_multi_tile(oracle_mod, m, n, k):
 
 
 @pytest.mark.parametrize("m,n,k", [(m, n, k) for (m, n, k) in GRID if m <= 64] +
-                         [(32, 129, 257), (64, 1000, 1000), (7, 4096, 65), (64, 2048, 4099)])
-def test_ragged_grid_streamk(oracle_mod, m, n, k):
+                         [(32, 129, 257), (64, 1000, 1000), (7, 4096, 65), (64, 2048, 4099),
+                          (32, 256, 8192), (5, 600, 3000), (33, 520, 12000), (1, 64, 70000)])
+def test_ragged_grid_skinny(oracle_mod, m, n, k):
     a, b = workloads.make_inputs(m, n, k, seed=2000 + m + 7 * n + 13 * k)
     for relu in (True, False):
         ref = oracle_mod.gemm_relu(a, b) if relu else oracle_mod.gemm(a, b)
-        check_parity(run(a, b, relu=relu, path=STREAMK), ref, relu, f"stream-K {m}x{n}x{k}")
+        check_parity(run(a, b, relu=relu, path=SKINNY), ref, relu, f"small-M {m}x{n}x{k}")
 
 
-@pytest.mark.parametrize("path", [TILE, STREAMK, PAIR])
+@pytest.mark.parametrize("path", [TILE, SKINNY, PAIR])
 def test_padded_leading_dimensions(oracle_mod, path):
     m, n, k = 45, 300, 190
     a, b = workloads.make_inputs(m, n, k, seed=5)
@@ -121,7 +122,7 @@ def gpu_fn_for(path):
     def fn(a, b, relu):
         a = torch.from_numpy(np.ascontiguousarray(np.asarray(a, dtype=np.float16)))
         b = torch.from_numpy(np.ascontiguousarray(np.asarray(b, dtype=np.float16)))
-        if path == STREAMK and a.shape[0] > 64:
+        if path == SKINNY and a.shape[0] > 64:
             p = TILE
         else:
             p = path
@@ -130,7 +131,7 @@ def gpu_fn_for(path):
 
 
 @pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
-@pytest.mark.parametrize("path", [TILE, STREAMK, PAIR], ids=["tile", "streamk", "pair"])
+@pytest.mark.parametrize("path", [TILE, SKINNY, PAIR], ids=["tile", "skinny", "pair"])
 def test_pins_on_gpu(pin, path):
     fails = pin(gpu_fn_for(path), exact=False)
     assert not fails, "\n".join(fails[:5])
@@ -201,7 +202,7 @@ def test_empty_output_is_noop():
 def test_deterministic_bits_both_paths():
     a, b = workloads.make_inputs(64, 3000, 2500, seed=9)
     ad, bd = to_dev(a, round8(2500)), to_dev(b)
-    for path in (TILE, STREAMK, PAIR):
+    for path in (TILE, SKINNY, PAIR):
         outs = []
         for _ in range(3):
             outs.append(ops.gemm_f16_ex(ad, bd, relu=True, path=path).view(torch.int16).cpu())
@@ -209,7 +210,7 @@ def test_deterministic_bits_both_paths():
 
 
 def test_back_to_back_calls_on_two_streams(oracle_mod):
-    """Two streams, each with its own stream-K workspace, interleaved."""
+    """Two streams, each with its own small-M workspace, interleaved."""
     a, b = workloads.make_inputs(32, 5000, 3000, seed=21)
     ref = oracle_mod.gemm_relu(a, b)
     ad, bd = a.cuda(), b.cuda()
@@ -258,11 +259,11 @@ def test_extent_beyond_allocation_rejected():
     assert rc == -1
 
 
-def test_streamk_path_refuses_large_m():
+def test_skinny_path_refuses_large_m():
     a = torch.zeros((65, 16), dtype=torch.float16, device="cuda")
     b = torch.zeros((16, 16), dtype=torch.float16, device="cuda")
     with pytest.raises(RuntimeError, match="invalid argument"):
-        ops.gemm_f16_ex(a, b, path=STREAMK)
+        ops.gemm_f16_ex(a, b, path=SKINNY)
 
 
 # ------------------------------------------------------ failure detection ---

@@ -1,8 +1,8 @@
 // Host side of libttc05: the C ABI declared in include/gemm_f16.h.
 //
 // Argument validation, per-device context (SM count, status word), TMA
-// tensor-map encoding, the choice between the tile kernel and the stream-K
-// kernel, the stream-K workspace cache and the status/self-test entry points.
+// tensor-map encoding, the choice between the tile kernels and the small-M
+// kernel, the small-M workspace cache and the status/self-test entry points.
 // The computation itself is the fused GEMM + ReLU of "Writing high-performance
 // kernels in TileLang" (atlascloud.ai blog), section "Escribamos un GEMM".
 #include <cuda.h>
@@ -137,7 +137,7 @@ int check_matrix(const void* p, int64_t rows, int64_t cols, int64_t ld, int devi
 }
 
 int get_workspace(const DeviceCtx& d, cudaStream_t stream, void** ptr, size_t* bytes) {
-  const size_t need = streamk_workspace_bytes(d.sm_count, 64);
+  const size_t need = skinny_workspace_bytes(d.sm_count, 64);
   std::lock_guard<std::mutex> lock(g_mutex);
   for (const Workspace& w : g_workspaces) {
     if (w.device == d.device && w.stream == stream) {
@@ -196,7 +196,7 @@ int read_and_clear_status(const DeviceCtx& d, cudaStream_t stream, int* out) {
   if (host != 0) {
     if (cudaMemsetAsync(d.status, 0, sizeof(int), stream) != cudaSuccess)
       return GEMM_ERR_LAUNCH;
-    // a kernel that gave up may have left stream-K arrival counters non-zero
+    // a kernel that gave up may have left split-K arrival counters non-zero
     std::lock_guard<std::mutex> lock(g_mutex);
     for (const Workspace& w : g_workspaces)
       if (w.device == d.device && cudaMemsetAsync(w.ptr, 0, w.bytes, stream) != cudaSuccess)
@@ -243,7 +243,7 @@ int gemm_abi_version(void) { return 10000; }
 
 int gemm_select_path(int64_t M, int64_t N, int64_t K) {
   (void)K;
-  if (M >= 1 && M <= 64) return GEMM_PATH_STREAMK;
+  if (M >= 1 && M <= 64) return GEMM_PATH_SKINNY;
   const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
   return pair_tiles >= 64 ? GEMM_PATH_TILE_PAIR : GEMM_PATH_TILE;
 }
@@ -255,7 +255,7 @@ const char* gemm_status_string(int status) {
     case GEMM_ERR_ALIGNMENT: return "pointer not 16-byte aligned or leading dimension not a multiple of 8";
     case GEMM_ERR_UNSUPPORTED_DEVICE: return "current device is not an sm_100 (B200) GPU";
     case GEMM_ERR_LAUNCH: return "CUDA runtime call or kernel launch failed";
-    case GEMM_ERR_WORKSPACE: return "stream-K workspace allocation failed";
+    case GEMM_ERR_WORKSPACE: return "small-M workspace allocation failed";
     case GEMM_ERR_DEVICE_TIMEOUT: return "a device-side wait ran out of time";
     case GEMM_ERR_SCRATCH_LIMIT:
       return "problem too large for the fixed scratch of gemm_relu_f16_noalloc (needs M <= 32)";
@@ -269,7 +269,7 @@ int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int
   if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return GEMM_ERR_INVALID_ARG;
   if (relu != 0 && relu != 1) return GEMM_ERR_INVALID_ARG;
-  if (path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE && path != GEMM_PATH_STREAMK &&
+  if (path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE && path != GEMM_PATH_SKINNY &&
       path != GEMM_PATH_TILE_PAIR)
     return GEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return GEMM_OK;
@@ -284,13 +284,13 @@ int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int
   if (rc == GEMM_OK) rc = check_matrix(B, K, N, ldb, d.device);
   if (rc != GEMM_OK) return rc;
   if (path == GEMM_PATH_AUTO) path = gemm_select_path(M, N, K);
-  if (path == GEMM_PATH_STREAMK) {
-    if (streamk_m_pad(M) == 0) return GEMM_ERR_INVALID_ARG;
+  if (path == GEMM_PATH_SKINNY) {
+    if (skinny_m_pad(M) == 0) return GEMM_ERR_INVALID_ARG;
     void* ws = nullptr;
     size_t ws_bytes = 0;
     rc = get_workspace(d, stream, &ws, &ws_bytes);
     if (rc != GEMM_OK) return rc;
-    return launch_streamk_gemm(p, d, ws, ws_bytes);
+    return launch_skinny_gemm(p, d, ws, ws_bytes);
   }
   if (path == GEMM_PATH_TILE_PAIR) return launch_tile_pair_gemm(p, d);
   return launch_tile_gemm(p, d);
@@ -307,7 +307,7 @@ int gemm_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_
 }
 
 // The allocation-free entry point: the same validation as gemm_f16_ex, then
-// the stream-K kernel with the library's fixed scratch array (see the header).
+// the small-M kernel with the library's fixed scratch array (see the header).
 int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_t M, int64_t N,
                           int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
                           gemm_stream_t stream) {
@@ -325,7 +325,7 @@ int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_t M, int6
   rc = check_matrix(A, M, K, lda, d.device);
   if (rc == GEMM_OK) rc = check_matrix(B, K, N, ldb, d.device);
   if (rc != GEMM_OK) return rc;
-  return launch_streamk_gemm_noalloc(p, d);
+  return launch_skinny_gemm_noalloc(p, d);
 }
 
 int gemm_get_device_status(gemm_stream_t stream, int* device_status) {

@@ -1,0 +1,443 @@
+// Small-M (decode-shaped) path of C = ReLU(A @ B) for sm_100a.
+//
+// With few rows in A the product is bound by reading B from HBM once; the
+// tensor cores are nearly idle and what matters is how fast, and in which
+// order, B streams in.
+//
+//   * swap-AB: the kernel computes C^T = B^T A^T, so a 128-wide slab of B's
+//     columns is the MMA M dimension (B^T is MN-major in shared memory, read
+//     straight from row-major B) and the few rows of A are the MMA N
+//     dimension (MP = M rounded up to 32 or 64; A^T is K-major).  One CTA owns
+//     a 256-column tile of C^T: two MMAs per 16-deep k step into two TMEM
+//     accumulators.
+//   * lock-step streaming: every CTA walks its k-range upward from the same
+//     start at the same time, so at any moment the whole grid reads the same
+//     band of rows of B across all N.  Row-major B then streams in long
+//     contiguous runs, which HBM serves far better than the scattered k
+//     offsets of a stream-K split (measured: 5.3 TB/s with stream-K over
+//     148 SMs, 6.8+ TB/s in lock-step over 112 SMs for M=32, N=28672,
+//     K=8192).
+//   * split-K only when there are fewer tiles than SMs: the k range of each
+//     tile is cut into S equal slices (one CTA each) -- the split-KV /
+//     FlashDecoding idea of "Writing high-performance kernels in TileLang"
+//     (atlascloud.ai blog), section "La parte buena: las optimizaciones son
+//     de una sola línea cada una", applied to the K axis of the GEMM.  Each
+//     slice writes its fp32 partial tile to a workspace and bumps the tile's
+//     arrival counter; whichever slice arrives last sums the S partials in
+//     slice order (deterministic), then applies ReLU -- only after the full K
+//     reduction -- and stores fp16.  No CTA ever waits for another.
+#include <atomic>
+#include <mutex>
+
+#include "../../include/gemm_f16.h"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace ttc {
+namespace {
+
+constexpr int kTW = 256;       // columns of B (rows of C^T) per CTA tile
+constexpr int kSub = 128;      // columns per MMA (MMA M)
+constexpr int kBK = 64;        // k-depth of a stage: one 128-byte swizzle row of A
+constexpr int kUmmaK = 16;
+constexpr int kThreads = 192;  // producer, MMA, 4 epilogue warps
+constexpr int kEpiWarps = 4;
+
+template <int MP, int STAGES>
+struct SkinnyCfg {
+  static constexpr int kBChunk = kBK * 64 * 2;    // 64 columns x 64 k-rows = 8 KiB
+  static constexpr int kBBytes = 4 * kBChunk;     // 256 columns
+  static constexpr int kABytes = MP * kBK * 2;    // MP rows x 128 bytes
+  static constexpr int kStageBytes = kBBytes + kABytes;
+  static constexpr int kNumBars = 2 * STAGES + 3;
+  static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kNumBars * 8 + 16;
+  static constexpr uint32_t kTmemCols = (2 * MP < 32) ? 32 : 2 * MP;
+  static constexpr uint32_t kIdesc = idesc_f16_f32(kSub, MP, /*A MN-major*/ true,
+                                                   /*B MN-major*/ false);
+  static_assert(MP == 32 || MP == 64, "MP");
+  static_assert(kABytes % 1024 == 0, "A tile alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
+  return __ldcg(reinterpret_cast<const float4*>(p));
+}
+
+template <int MP, bool RELU>
+__device__ __forceinline__ void store_column(const float (&v)[MP], __half* C, int M, int N,
+                                             int64_t ldc, int n) {
+  if (n >= N) return;
+#pragma unroll
+  for (int m = 0; m < MP; ++m) {
+    if (m < M) {
+      const float x = RELU ? relu_f32(v[m]) : v[m];
+      C[static_cast<int64_t>(m) * ldc + n] = __float2half_rn(x);
+    }
+  }
+}
+
+// MP fp32 accumulator columns of this thread's TMEM lane.
+template <int MP>
+__device__ __forceinline__ void load_accumulator(uint32_t taddr, float (&v)[MP]) {
+#pragma unroll
+  for (int j = 0; j < MP / 32; ++j) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr + j * 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[j * 32 + i] = __uint_as_float(r[i]);
+  }
+}
+
+// One CTA per (tile, k-slice); blockIdx.x = tile * S + slice.
+template <int MP, int STAGES, bool RELU>
+__global__ void __launch_bounds__(kThreads, 1)
+    skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, __half* __restrict__ C, int M,
+                       int N, int K, int64_t ldc, int S, float* __restrict__ partials,
+                       int* __restrict__ counters, int* status, uint64_t timeout_ns) {
+  using Cfg = SkinnyCfg<MP, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* smB = smem;
+  uint8_t* smA = smem + STAGES * Cfg::kBBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* drain = bars + 2 * STAGES + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tile = blockIdx.x / S;
+  const int slice = blockIdx.x - tile * S;
+  const int KB = (K + kBK - 1) / kBK;
+  const int kb_begin = static_cast<int>(static_cast<int64_t>(slice) * KB / S);
+  const int kb_end = static_cast<int>(static_cast<int64_t>(slice + 1) * KB / S);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer ---
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int kb = kb_begin; kb < kb_end; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+        uint8_t* bdst = smB + stage * Cfg::kBBytes;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tma_load_2d(&tmB, &full[stage], bdst + j * Cfg::kBChunk, tile * kTW + j * 64,
+                      kb * kBK);
+        tma_load_2d(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, 0);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleProducer << 4) | 2);
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s))
+            (void)mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer ---
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = kb_begin; kb < kb_end; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t b_addr = smem_u32(smB + stage * Cfg::kBBytes);
+        const uint32_t a_addr = smem_u32(smA + stage * Cfg::kABytes);
+#pragma unroll
+        for (int k = 0; k < kBK / kUmmaK; ++k) {
+          // MMA B operand = A^T tile (K-major): 32 bytes per 16 k along the row
+          const uint64_t bdesc = smem_desc_sw128(a_addr + k * (kUmmaK * 2), 16, 1024);
+#pragma unroll
+          for (int h = 0; h < kTW / kSub; ++h) {
+            // MMA A operand = B^T sub-tile h (N-major): slabs 2h, 2h+1; 16 k-rows
+            const uint64_t adesc = smem_desc_sw128(
+                b_addr + h * 2 * Cfg::kBChunk + k * (kUmmaK * 128), Cfg::kBChunk, 1024);
+            umma_f16(tmem_base + static_cast<uint32_t>(h * MP), adesc, bdesc, Cfg::kIdesc,
+                     (kb > kb_begin || k > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) {
+        umma_commit(acc_full);
+      } else {
+        raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleMma << 4) | 4);
+        umma_commit(drain);
+        (void)mbar_wait(drain, 0, nullptr, timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue ---
+    const int q = warp & 3;
+    const int row = q * 32 + lane;  // TMEM lane = column of C inside each 128-wide half
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(acc_full, 0, abort_flag, timeout_ns) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    // the four epilogue warps meet at named barriers below: all continue or
+    // all stop
+    ok = named_bar_and(1, kEpiWarps * 32, ok);
+    if (!ok) {
+      if (lane == 0)
+        raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleEpilogue << 4) | 2);
+    } else {
+      tc_fence_after_sync();
+      const int n0 = tile * kTW + row;
+      const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      // one 128-column half at a time keeps only MP accumulators per thread live
+      if (S == 1) {
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float v[MP];
+          load_accumulator<MP>(t_lane + static_cast<uint32_t>(h * MP), v);
+          store_column<MP, RELU>(v, C, M, N, ldc, n0 + h * kSub);
+        }
+      } else {
+        // partial tile of this slice: [item][256 columns][MP]
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float v[MP];
+          load_accumulator<MP>(t_lane + static_cast<uint32_t>(h * MP), v);
+          float* mine =
+              partials + (static_cast<int64_t>(blockIdx.x) * kTW + h * kSub + row) * MP;
+#pragma unroll
+          for (int m = 0; m < MP; m += 4)
+            *reinterpret_cast<float4*>(mine + m) = make_float4(v[m], v[m + 1], v[m + 2], v[m + 3]);
+        }
+        __threadfence();
+        named_bar_sync(1, kEpiWarps * 32);
+        if (threadIdx.x == 64) {
+          const int prev = atomicAdd(&counters[tile], 1);
+          const int is_last = (prev == S - 1) ? 1 : 0;
+          if (is_last) atomicExch(&counters[tile], 0);  // ready for the next call
+          *last_flag = is_last;
+        }
+        named_bar_sync(1, kEpiWarps * 32);
+        if (*last_flag) {
+          __threadfence();
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            float v[MP], acc[MP];
+            load_accumulator<MP>(t_lane + static_cast<uint32_t>(h * MP), v);
+            for (int sl = 0; sl < S; ++sl) {
+              if (sl == slice) {
+#pragma unroll
+                for (int m = 0; m < MP; ++m) acc[m] = (sl == 0) ? v[m] : acc[m] + v[m];
+              } else {
+                const float* src =
+                    partials + ((static_cast<int64_t>(tile) * S + sl) * kTW + h * kSub + row) * MP;
+#pragma unroll
+                for (int m = 0; m < MP; m += 4) {
+                  const float4 p = ld_cg_f4(src + m);
+                  if (sl == 0) {
+                    acc[m] = p.x; acc[m + 1] = p.y; acc[m + 2] = p.z; acc[m + 3] = p.w;
+                  } else {
+                    acc[m] += p.x; acc[m + 1] += p.y; acc[m + 2] += p.z; acc[m + 3] += p.w;
+                  }
+                }
+              }
+            }
+            store_column<MP, RELU>(acc, C, M, N, ldc, n0 + h * kSub);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+bool ensure_smem_attr_skinny(const void* func, int bytes, int device,
+                             std::atomic<uint64_t>& done) {
+  const uint64_t bit = 1ull << (device & 63);
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
+constexpr size_t counter_bytes(int n) {
+  return (static_cast<size_t>(n) * sizeof(int) + 255) & ~static_cast<size_t>(255);
+}
+
+// Number of k-slices per tile: 1 when the tiles already cover the SMs,
+// otherwise as many as fit on the idle SMs, keeping at least 4 k-blocks of 64
+// per slice and at most `max_items` (tile, slice) pairs.
+int choose_slices(int64_t tiles, int64_t KB, int sm_count, int64_t max_items) {
+  if (tiles >= sm_count) return 1;
+  int64_t s = sm_count / tiles;
+  const int64_t by_k = KB / 4;
+  if (s > by_k) s = by_k;
+  if (s * tiles > max_items) s = max_items / tiles;
+  return s < 1 ? 1 : static_cast<int>(s);
+}
+
+template <int MP, int STAGES, bool RELU>
+int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
+                int64_t max_items) {
+  using Cfg = SkinnyCfg<MP, STAGES>;
+  static std::atomic<uint64_t> attr_done{0};
+  const int64_t KB = (p.K + kBK - 1) / kBK;
+  const int64_t tiles = (p.N + kTW - 1) / kTW;
+  const int S = choose_slices(tiles, KB, d.sm_count, max_items);
+  int* counters = nullptr;
+  float* partials = nullptr;
+  if (S > 1) {
+    // counters for the tiles, then one fp32 partial tile per (tile, slice)
+    const size_t need = counter_bytes(static_cast<int>(max_items)) +
+                        static_cast<size_t>(tiles) * S * kTW * MP * sizeof(float);
+    if (ws == nullptr || ws_bytes < need) return GEMM_ERR_WORKSPACE;
+    counters = static_cast<int*>(ws);
+    partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                        counter_bytes(static_cast<int>(max_items)));
+  }
+  CUtensorMap tA, tB;
+  int rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, MP);
+  if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
+  if (rc != 0) return rc;
+  auto kern = skinny_gemm_kernel<MP, STAGES, RELU>;
+  if (!ensure_smem_attr_skinny(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
+                               attr_done))
+    return GEMM_ERR_LAUNCH;
+  const int64_t grid = tiles * S;
+  if (grid > INT32_MAX) return GEMM_ERR_INVALID_ARG;
+  kern<<<static_cast<int>(grid), kThreads, Cfg::kSmemBytes, p.stream>>>(
+      tA, tB, static_cast<__half*>(p.C), static_cast<int>(p.M), static_cast<int>(p.N),
+      static_cast<int>(p.K), p.ldc, S, partials, counters, d.status, d.timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? GEMM_OK : GEMM_ERR_LAUNCH;
+}
+
+}  // namespace
+
+int skinny_m_pad(int64_t M) {
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 0;
+}
+
+size_t skinny_workspace_bytes(int sm_count, int m_pad) {
+  // split-K happens only with fewer tiles than SMs, so at most sm_count
+  // (tile, slice) items carry a partial tile
+  return counter_bytes(sm_count) +
+         static_cast<size_t>(sm_count) * kTW * static_cast<size_t>(m_pad) * sizeof(float);
+}
+
+int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes) {
+  const int mp = skinny_m_pad(p.M);
+  if (mp == 32)
+    return p.relu ? launch_impl<32, 6, true>(p, d, ws, ws_bytes, d.sm_count)
+                  : launch_impl<32, 6, false>(p, d, ws, ws_bytes, d.sm_count);
+  if (mp == 64)
+    return p.relu ? launch_impl<64, 5, true>(p, d, ws, ws_bytes, d.sm_count)
+                  : launch_impl<64, 5, false>(p, d, ws, ws_bytes, d.sm_count);
+  return GEMM_ERR_INVALID_ARG;
+}
+
+// ------------------------------------------------ allocation-free variant ---
+// Scratch of gemm_relu_f16_noalloc: arrival counters for up to
+// kNoAllocMaxItems tiles, then one fp32 partial tile (256 columns x 32) per
+// (tile, slice) item, for at most kNoAllocMaxItems items.  It is part of the
+// library image, so every GPU that loads the library holds it.
+namespace {
+
+constexpr int kNoAllocMP = 32;
+constexpr int kNoAllocMaxItems = 160;
+constexpr size_t kNoAllocCounterBytes = counter_bytes(kNoAllocMaxItems);
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocCounterBytes + static_cast<size_t>(kNoAllocMaxItems) * kTW * kNoAllocMP * sizeof(float);
+static_assert(kNoAllocScratchBytes == 5243648, "documented scratch size");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[64] = {};  // device address of g_noalloc_scratch, per device
+
+// Host code cannot use the array's name as a device address (it names a host
+// stand-in); look the real address up once per device, with it current.
+int noalloc_scratch_address(int device, void** out) {
+  if (device < 0 || device >= 64) return GEMM_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[device] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return GEMM_ERR_LAUNCH;
+    }
+    g_noalloc_addr[device] = p;
+  }
+  *out = g_noalloc_addr[device];
+  return GEMM_OK;
+}
+
+}  // namespace
+
+int launch_skinny_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d) {
+  if (p.M > kNoAllocMP) return GEMM_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  const int rc = noalloc_scratch_address(d.device, &scratch);
+  if (rc != GEMM_OK) return rc;
+  // the array keeps the previous call's contents: the arrival counters must
+  // start at zero (partial tiles are always written before they are read)
+  if (cudaMemsetAsync(scratch, 0, kNoAllocCounterBytes, p.stream) != cudaSuccess)
+    return GEMM_ERR_LAUNCH;
+  const int64_t items = d.sm_count < kNoAllocMaxItems ? d.sm_count : kNoAllocMaxItems;
+  return launch_impl<kNoAllocMP, 6, true>(p, d, scratch, kNoAllocScratchBytes, items);
+}
+
+}  // namespace ttc

@@ -37,17 +37,17 @@ int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d);
 // ... or a pair of SMs per 256 x 256 tile (tcgen05.mma.cta_group::2).
 int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d);
 
-// Small-M path: swap-AB stream-K kernel.  `workspace` holds partial tiles and
-// per-tile arrival counters (counters must be zero on entry; the kernel
-// leaves them zero).
-size_t streamk_workspace_bytes(int sm_count, int m_pad);
-int launch_streamk_gemm(const GemmProblem& p, const DeviceCtx& d, void* workspace,
-                        size_t workspace_bytes);
-int streamk_m_pad(int64_t M);  // MMA N used for M rows (0 if M is too large)
+// Small-M path: swap-AB, lock-step split-K kernel.  `workspace` holds
+// per-tile arrival counters and split-K partial tiles (counters must be zero
+// on entry; the kernel leaves them zero).
+size_t skinny_workspace_bytes(int sm_count, int m_pad);
+int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* workspace,
+                       size_t workspace_bytes);
+int skinny_m_pad(int64_t M);  // MMA N used for M rows (0 if M is too large)
 
-// The stream-K kernel with its scratch in a fixed device array of the
-// library (no allocation); M <= 32.  Returns GEMM_ERR_SCRATCH_LIMIT beyond.
-int launch_streamk_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d);
+// The small-M kernel with its scratch in a fixed device array of the library
+// (no allocation); M <= 32.  Returns GEMM_ERR_SCRATCH_LIMIT beyond.
+int launch_skinny_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d);
 
 // Writes C = 0 (used when K == 0: the empty sum, and ReLU of it, is +0).
 int launch_zero_fill(const GemmProblem& p);
