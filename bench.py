@@ -37,9 +37,16 @@ METRIC = "fused GEMM+ReLU TFLOP/s and % of B200 dense fp16 peak (GB/s % HBM for 
 NOMINAL_FP16_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["tiled_tensor_core_05_b200/csrc/gemm_tile.cu",
-                  "tiled_tensor_core_05_b200/csrc/gemm_skinny.cu",
-                  "tiled_tensor_core_05_b200/csrc/sm100.cuh"]
+# source files that define each timed kernel (the `traffic` figure of a
+# committed ncu capture is reported only while these are unchanged)
+KERNEL_SOURCES = {
+    "tile_pair_gemm_kernel": ["tiled_tensor_core_05_b200/csrc/gemm_tile.cu",
+                              "tiled_tensor_core_05_b200/csrc/sm100.cuh"],
+    "tile_gemm_kernel": ["tiled_tensor_core_05_b200/csrc/gemm_tile.cu",
+                         "tiled_tensor_core_05_b200/csrc/sm100.cuh"],
+    "skinny_gemm_kernel": ["tiled_tensor_core_05_b200/csrc/gemm_skinny.cu",
+                           "tiled_tensor_core_05_b200/csrc/sm100.cuh"],
+}
 
 
 # ------------------------------------------------------------------ utils ---
@@ -58,25 +65,25 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def traffic_for(workload: str):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken on
-    the current kernel sources (else None)."""
+def traffic_for(workload: str, kernel: str):
+    """DRAM bytes (read + write) per launch from a committed ncu capture of
+    `kernel` on `workload`, if it was taken on the current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             table = json.load(f)
     except (OSError, ValueError):
         return None
-    e = table.get(workload)
-    if not e or e.get("kernel_src_sha") != kernel_source_hash():
+    e = table.get(f"{kernel}/{workload}")
+    if not e or e.get("kernel_src_sha") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -260,23 +267,30 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
     return res
 
 
+def kernel_for(w) -> str:
+    from tiled_tensor_core_05_b200 import ops
+    return {ops.PATH_SKINNY: "skinny_gemm_kernel", ops.PATH_TILE: "tile_gemm_kernel",
+            ops.PATH_TILE_PAIR: "tile_pair_gemm_kernel"}[ops.select_path(w.M, w.N, w.K)]
+
+
 def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool):
     from tiled_tensor_core_05_b200 import workloads
     w = workloads.WORKLOADS[name]
+    kernel = kernel_for(w)
     if name == "decode":
         # HBM bound: algorithmic bytes = A, B read once, C written once
         achieved = w.bytes_min / (launch_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_for(name),
-                "algorithmic_bytes_per_launch": w.bytes_min,
+                "frac": round(achieved / peak, 4), "traffic": traffic_for(name, kernel),
+                "kernel": kernel, "algorithmic_bytes_per_launch": w.bytes_min,
                 "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"}
     achieved = w.flops / (launch_ms * 1e-3) / 1e12
     key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
     peak = peaks.get(key, peaks["bf16_tflops"])
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4), "traffic": traffic_for(name),
-            "algorithmic_flops_per_launch": w.flops,
+            "frac": round(achieved / peak, 4), "traffic": traffic_for(name, kernel),
+            "kernel": kernel, "algorithmic_flops_per_launch": w.flops,
             "peak_source": f"{peak_src} {key} (cuBLAS bf16; fp16 has the same nominal rate)"}
 
 
@@ -395,10 +409,6 @@ def run_ours(args):
         line["pct_of_dense_fp16_peak"] = round(100 * value / world / NOMINAL_FP16_TFLOPS, 2)
     line["roofline"] = roofline_entry(args.workload, main["launch_ms"], peaks, peak_src,
                                       long_run)
-    path = ops.select_path(w.M, w.N, w.K)
-    line["roofline"]["kernel"] = {ops.PATH_SKINNY: "skinny_gemm_kernel",
-                                  ops.PATH_TILE: "tile_gemm_kernel",
-                                  ops.PATH_TILE_PAIR: "tile_pair_gemm_kernel"}[path]
     if "e2e_ms" in main:
         e_ms = main["e2e_ms"]
         ev = (w.flops / (e_ms * 1e-3) / 1e12) if unit == "TFLOP/s" else \
