@@ -173,9 +173,15 @@ def gpu_id_for(dev_index: int) -> str:
 
 # ----------------------------------------------------------- measurements ---
 
-def time_launches(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
-    """Warm up, then time `steps` calls with CUDA events on `stream`.
-    Returns (total_ms max over ranks, mean per-launch ms on this rank)."""
+def time_launches(fn, steps: int, warmup: int, stream, dist=None, sampler=None,
+                  per_launch=False):
+    """Warm up, then time exactly `steps` back-to-back calls between two CUDA
+    events on `stream` (barrier + synchronize on both sides).  Returns
+    (total_ms of the timed region, max over ranks; ms per launch).  One step
+    launches one kernel, so the kernel's average duration over the timed region
+    is total / steps (gaps between launches included: a conservative figure).
+    With per_launch=True, `steps` more calls are timed afterwards each between
+    its own pair of events, and their mean is returned instead."""
     import torch
     if sampler:
         sampler.mark("warm0")
@@ -187,15 +193,11 @@ def time_launches(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
     torch.cuda.synchronize()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     if sampler:
         sampler.mark("t0")
     ev0.record(stream)
-    for i in range(steps):
-        starts[i].record(stream)
+    for _ in range(steps):
         fn()
-        ends[i].record(stream)
     ev1.record(stream)
     torch.cuda.synchronize()
     if sampler:
@@ -203,12 +205,22 @@ def time_launches(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
     if dist is not None:
         dist.barrier()
     total = ev0.elapsed_time(ev1)
-    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     if dist is not None:
         t = torch.tensor([total], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total = float(t.item())
-    return total, sum(per) / len(per)
+    per_ms = total / steps
+    if per_launch:
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            starts[i].record(stream)
+            fn()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        per = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+        per_ms = sum(per) / len(per)
+    return total, per_ms
 
 
 def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
@@ -240,7 +252,9 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
         # the same inputs, timed the same way right after our kernel
         def torch_step():
             torch.relu_(torch.matmul(a, b, out=c))
-        _, t_ms = time_launches(torch_step, steps, warmup, stream, None, None)
+        t_total, _ = time_launches(torch_step, steps, warmup, stream, None, None,
+                                   per_launch=False)
+        t_ms = t_total / steps
         res["torch_launch_ms"] = t_ms
     if e2e:
         # end to end through the C ABI: pinned host inputs -> device, the
@@ -256,7 +270,7 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
             c_h.copy_(c, non_blocking=True)
 
         e_steps = max(3, min(steps, 10))
-        e_total, _ = time_launches(e2e_step, e_steps, 1, stream, dist, None)
+        e_total, _ = time_launches(e2e_step, e_steps, 1, stream, dist, None, per_launch=False)
         res["e2e_ms"] = e_total / e_steps
         res["h2d"] = a.numel() * 2 + b.numel() * 2
         res["d2h"] = c.numel() * 2

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstdlib>
 #include <mutex>
 #include <vector>
 
@@ -222,6 +223,21 @@ int encode_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_INVALID_ARG;
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* s = std::getenv("TTC_PDL");
+    return !(s != nullptr && s[0] == '0');
+  }();
+  return on;
+}
+
+int pdl_attribute(cudaLaunchAttribute* attr) {
+  if (!pdl_enabled()) return 0;
+  attr->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr->val.programmaticStreamSerializationAllowed = 1;
+  return 1;
 }
 
 int launch_zero_fill(const GemmProblem& p) {

@@ -218,6 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // the set-up above overlaps the previous kernel of the stream; inputs and
+  // outputs are touched only after it has finished
+  grid_dependency_trigger();
+  grid_dependency_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer ---
@@ -424,6 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();  // barriers of both CTAs initialised, TMEM of both SMs allocated
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_trigger();
+  grid_dependency_wait();
   // the leader's barriers, as addresses this CTA can signal
   const uint32_t full_leader = map_to_cta(smem_u32(full), 0);
   const uint32_t acc_empty_leader = map_to_cta(smem_u32(acc_empty), 0);
@@ -608,11 +614,18 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
     return GEMM_ERR_LAUNCH;
   const int64_t num_tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
   const int grid = static_cast<int>(num_tiles < d.sm_count ? num_tiles : d.sm_count);
-  kern<<<grid, kThreads, Cfg::kSmemBytes, p.stream>>>(
-      tA, tB, tC, static_cast<__half*>(p.C), p.ldc, static_cast<int>(p.M),
-      static_cast<int>(p.N), static_cast<int>(p.K),
-      group_tiles(kBM), d.status, d.timeout_ns);
-  return cudaGetLastError() == cudaSuccess ? 0 : GEMM_ERR_LAUNCH;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = p.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_attribute(&attr[0]);
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc, static_cast<int>(p.M),
+      static_cast<int>(p.N), static_cast<int>(p.K), group_tiles(kBM), d.status, d.timeout_ns);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
 template <int STAGES, bool RELU>
@@ -630,7 +643,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
                         attr_done))
     return GEMM_ERR_LAUNCH;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
@@ -655,6 +668,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   const int64_t num_tiles = ((p.M + 2 * kBM - 1) / (2 * kBM)) * ((p.N + 255) / 256);
   const int pairs = static_cast<int>(num_tiles < resident ? num_tiles : resident);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.numAttrs = 1 + pdl_attribute(&attr[1]);
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc, static_cast<int>(p.M),
       static_cast<int>(p.N), static_cast<int>(p.K), group_tiles(2 * kBM), d.status,

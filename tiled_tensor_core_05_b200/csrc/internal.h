@@ -24,6 +24,15 @@ struct DeviceCtx {
   uint64_t timeout_ns;  // limit for every device-side wait
 };
 
+// Whether kernels are launched with programmatic stream serialisation, so
+// their set-up overlaps the previous kernel of the stream (TTC_PDL=0 turns it
+// off for comparisons).
+bool pdl_enabled();
+
+// Fills `attr` with the programmatic-serialisation attribute when enabled;
+// returns the number of attributes written (0 or 1).
+int pdl_attribute(cudaLaunchAttribute* attr);
+
 // Encode a 2-D row-major fp16 tensor map with 128-byte swizzle.
 //   inner/outer: extents in elements (inner is contiguous)
 //   ld: row stride in elements; box_inner/box_outer: box extents in elements
