@@ -25,7 +25,7 @@ from . import build as _build
 
 __all__ = [
     "gemm_relu", "gemm", "gemm_relu_at", "gemm_at", "gemm_f64_at",
-    "decode_f16", "encode_f16", "max_threads",
+    "gemm_bias_act", "activation_f64", "decode_f16", "encode_f16", "max_threads",
 ]
 
 _lib = None
@@ -50,6 +50,11 @@ def _load():
         lib.oracle_decode_f16.restype = None
         lib.oracle_encode_f16.argtypes = [p, p, i64]
         lib.oracle_encode_f16.restype = None
+        lib.oracle_gemm_bias_act_f16.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64,
+                                                 ctypes.c_int, ctypes.c_int]
+        lib.oracle_gemm_bias_act_f16.restype = ctypes.c_int
+        lib.oracle_activation_f64.argtypes = [p, p, i64, ctypes.c_int]
+        lib.oracle_activation_f64.restype = None
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -175,6 +180,48 @@ def encode_f16(values) -> np.ndarray:
     values = np.ascontiguousarray(values, dtype=np.float64)
     out = np.empty(values.shape, dtype=np.uint16)
     _load().oracle_encode_f16(values.ctypes.data, out.ctypes.data, values.size)
+    return out
+
+
+ACT_NONE, ACT_RELU, ACT_GELU = 0, 1, 2
+_ACTS = {"none": ACT_NONE, "relu": ACT_RELU, "gelu": ACT_GELU}
+
+
+def gemm_bias_act(a, b, bias=None, act="gelu", nthreads=None) -> np.ndarray:
+    """act(A @ B + bias) as an (M, N) float16 array; bias is an fp16 vector of
+    length N (or None); act is "none", "relu" or "gelu" (erf form)."""
+    a, b = _bits(a), _bits(b)
+    M, K = a.shape
+    K2, N = b.shape
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    c = np.zeros((M, N), dtype=np.uint16)
+    if M == 0 or N == 0:
+        return c.view(np.float16)
+    bias_ptr = None
+    if bias is not None:
+        if hasattr(bias, "detach"):  # torch tensor
+            bias = bias.detach().reshape(1, -1)
+        else:
+            bias = np.asarray(bias).reshape(1, -1)
+        bb = np.ascontiguousarray(_bits(bias))
+        if bb.shape[1] != N:
+            raise ValueError("bias must have N elements")
+        bias_ptr = bb.ctypes.data
+    rc = _load().oracle_gemm_bias_act_f16(a.ctypes.data, b.ctypes.data, bias_ptr, c.ctypes.data,
+                                          M, N, K, _ld(a), _ld(b), N, code, _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_gemm_bias_act_f16 failed ({rc})")
+    return c.view(np.float16)
+
+
+def activation_f64(x, act="gelu") -> np.ndarray:
+    """The oracle's activation on float64 values (no rounding)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    _load().oracle_activation_f64(x.ctypes.data, out.ctypes.data, x.size, code)
     return out
 
 

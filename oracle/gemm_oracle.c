@@ -219,4 +219,72 @@ int oracle_gemm_f64_at(const uint16_t* A, const uint16_t* B,
     return 0;
 }
 
+/* ---- fused bias + activation epilogue --------------------------------- */
+/* "TileLang simplifica la creación de kernels GPU de alto rendimiento"
+ * (posicionamiento-web.ar), section "Fusionar operaciones para reducir viajes
+ * a memoria": the bias is added and GELU applied while the accumulator is
+ * still on chip, and the result is written once.  Read here as
+ *   C[i,j] = fp16_RNE( act( sum_k A[i,k] B[k,j] + bias[j] ) )
+ * with bias an fp16 vector over the output columns (absent = 0), the sum
+ * exact as above, and act one of
+ *   0: identity, 1: max(x, 0) (-0 and NaN -> +0),
+ *   2: GELU(x) = x * Phi(x) with Phi the standard normal CDF (the plain
+ *      definition), Phi(x) = 0.5 * erfc(-x / sqrt(2)): the same function as
+ *      0.5 * (1 + erf(x / sqrt(2))) without its cancellation for negative x
+ *      (libm's erfc in fp64). */
+enum { ORACLE_ACT_NONE = 0, ORACLE_ACT_RELU = 1, ORACLE_ACT_GELU = 2 };
+
+static double act64(double x, int act)
+{
+    if (act == ORACLE_ACT_RELU) return relu64(x);
+    if (act == ORACLE_ACT_GELU) return x * (0.5 * erfc(-x / sqrt(2.0)));
+    return x;
+}
+
+int oracle_gemm_bias_act_f16(const uint16_t* A, const uint16_t* B, const uint16_t* bias,
+                             uint16_t* C, int64_t M, int64_t N, int64_t K,
+                             int64_t lda, int64_t ldb, int64_t ldc, int act, int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0 || act < 0 || act > 2) return -1;
+    if (M == 0 || N == 0) return 0;
+    if (lda < K || ldb < N || ldc < N) return -1;
+    double* tab = decode_table();
+    if (!tab) return -1;
+    int failed = 0;
+    const int nt = resolve_threads(nthreads);
+#pragma omp parallel num_threads(nt)
+    {
+        double* acc = (double*)malloc(sizeof(double) * (size_t)N);
+        if (!acc) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < M; ++i) {
+            if (!acc) continue;
+            for (int64_t j = 0; j < N; ++j) acc[j] = 0.0;
+            const uint16_t* arow = A + i * lda;
+            for (int64_t k = 0; k < K; ++k) {
+                const double a = tab[arow[k]];
+                const uint16_t* brow = B + k * ldb;
+                for (int64_t j = 0; j < N; ++j) acc[j] += a * tab[brow[j]];
+            }
+            uint16_t* crow = C + i * ldc;
+            for (int64_t j = 0; j < N; ++j) {
+                const double x = acc[j] + (bias ? tab[bias[j]] : 0.0);
+                crow[j] = oracle_f64_to_f16(act64(x, act));
+            }
+        }
+        free(acc);
+    }
+    free(tab);
+    return failed ? -1 : 0;
+}
+
+/* The activations alone on fp64 inputs (unrounded), for pinning act64. */
+void oracle_activation_f64(const double* in, double* out, int64_t n, int act)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = act64(in[i], act);
+}
+
 int oracle_max_threads(void) { return resolve_threads(0); }

@@ -51,9 +51,11 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+typedef CUresult (*PointerAttrsFn)(unsigned int, CUpointer_attribute*, void**, CUdeviceptr);
 
 EncodeTiledFn g_encode = nullptr;
 AddressRangeFn g_addr_range = nullptr;
+PointerAttrsFn g_ptr_attrs = nullptr;
 std::once_flag g_entry_once;
 
 void load_entry_points() {
@@ -69,6 +71,11 @@ void load_entry_points() {
                                          &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       g_addr_range = reinterpret_cast<AddressRangeFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuPointerGetAttributes", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ptr_attrs = reinterpret_cast<PointerAttrsFn>(fn);
   });
 }
 
@@ -127,13 +134,41 @@ bool extent_in_allocation(const void* p, int64_t rows, int64_t cols, int64_t ld)
   return start >= base && start - base + span <= size;
 }
 
+// One driver query for memory type, owning device and allocation range.
+// Returns -1 when the query itself is unavailable (caller falls back).
+int query_pointer(const void* p, int device, int64_t rows, int64_t cols, int64_t ld) {
+  if (g_ptr_attrs == nullptr) return -1;
+  unsigned int mem_type = 0;
+  int ordinal = -1;
+  unsigned int managed = 0;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  CUpointer_attribute attrs[5] = {CU_POINTER_ATTRIBUTE_MEMORY_TYPE,
+                                  CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL,
+                                  CU_POINTER_ATTRIBUTE_IS_MANAGED,
+                                  CU_POINTER_ATTRIBUTE_RANGE_START_ADDR,
+                                  CU_POINTER_ATTRIBUTE_RANGE_SIZE};
+  void* data[5] = {&mem_type, &ordinal, &managed, &base, &size};
+  if (g_ptr_attrs(5, attrs, data, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS) return 0;
+  const bool on_device = (mem_type == CU_MEMORYTYPE_DEVICE && ordinal == device) || managed != 0;
+  if (!on_device || size == 0) return 0;
+  const uint64_t start = reinterpret_cast<uint64_t>(p);
+  const uint64_t span = (static_cast<uint64_t>(rows - 1) * static_cast<uint64_t>(ld) +
+                         static_cast<uint64_t>(cols)) * 2u;
+  return (start >= base && start - base + span <= size) ? 1 : 0;
+}
+
 int check_matrix(const void* p, int64_t rows, int64_t cols, int64_t ld, int device) {
   if (p == nullptr) return GEMM_ERR_INVALID_ARG;
   if (ld < cols || ld < 1) return GEMM_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0 || (ld & 7) != 0) return GEMM_ERR_ALIGNMENT;
   if (static_cast<uint64_t>(ld) * 2u >= (1ull << 40)) return GEMM_ERR_INVALID_ARG;
-  if (!is_device_pointer(p, device)) return GEMM_ERR_INVALID_ARG;
-  if (!extent_in_allocation(p, rows, cols, ld)) return GEMM_ERR_INVALID_ARG;
+  const int q = query_pointer(p, device, rows, cols, ld);
+  if (q == 0) return GEMM_ERR_INVALID_ARG;
+  if (q < 0) {
+    if (!is_device_pointer(p, device)) return GEMM_ERR_INVALID_ARG;
+    if (!extent_in_allocation(p, rows, cols, ld)) return GEMM_ERR_INVALID_ARG;
+  }
   return GEMM_OK;
 }
 
@@ -292,6 +327,7 @@ int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int
   DeviceCtx d;
   int rc = get_device(&d);
   if (rc != GEMM_OK) return rc;
+  load_entry_points();
   rc = check_matrix(C, M, N, ldc, d.device);
   if (rc != GEMM_OK) return rc;
   GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, relu != 0, stream};
@@ -334,6 +370,7 @@ int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_t M, int6
   DeviceCtx d;
   int rc = get_device(&d);
   if (rc != GEMM_OK) return rc;
+  load_entry_points();
   rc = check_matrix(C, M, N, ldc, d.device);
   if (rc != GEMM_OK) return rc;
   GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, true, stream};
