@@ -76,6 +76,12 @@ enum gemm_path {
                               (any shape) */
 };
 
+enum gemm_activation {
+  GEMM_ACT_NONE = 0,  /* identity */
+  GEMM_ACT_RELU = 1,  /* max(x, 0); -0 and NaN give +0 */
+  GEMM_ACT_GELU = 2   /* x * Phi(x), Phi the standard normal CDF (exact "erf" GELU) */
+};
+
 /* C = ReLU(A @ B).  "Escribamos un GEMM": the tiled fp16 matmul with the
  * max(x, 0) epilogue fused before the fp16 store.  Returns GEMM_OK or a
  * negative gemm_status. */
@@ -92,6 +98,21 @@ GEMM_API int gemm_f16(const void* A, const void* B, void* C, int64_t M, int64_t 
 GEMM_API int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
                 int64_t lda, int64_t ldb, int64_t ldc, int relu, int path,
                 gemm_stream_t stream);
+
+/* C = act(A @ B + bias): the fused epilogue of "TileLang simplifica la
+ * creación de kernels GPU de alto rendimiento" (posicionamiento-web.ar),
+ * section "Fusionar operaciones para reducir viajes a memoria" -- the bias is
+ * added and the activation applied to the fp32 accumulator on chip, and C is
+ * written once.
+ *   bias: device pointer to N fp16 values (one per column of C), 16-byte
+ *         aligned, or NULL for no bias.
+ *   activation: a gemm_activation value.
+ *   path: a gemm_path value (as in gemm_f16_ex).
+ * With K == 0 the result is C = act(bias) (act(0) = +0 without a bias).
+ * Returns GEMM_OK or a negative gemm_status. */
+GEMM_API int gemm_bias_act_f16(const void* A, const void* B, const void* bias, void* C,
+                               int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                               int64_t ldc, int activation, int path, gemm_stream_t stream);
 
 /* The path GEMM_PATH_AUTO takes for this shape (GEMM_PATH_TILE,
  * GEMM_PATH_TILE_PAIR or GEMM_PATH_SKINNY).  Pure host function. */

@@ -207,6 +207,17 @@ __global__ void zero_fill_kernel(__half* C, int64_t M, int64_t N, int64_t ldc) {
   }
 }
 
+template <int ACT>
+__global__ void bias_act_fill_kernel(__half* C, const __half* bias, int64_t M, int64_t N,
+                                     int64_t ldc) {
+  const int64_t total = M * N;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / N, c = i - r * N;
+    C[r * ldc + c] = __float2half_rn(activate<ACT>(__half2float(bias[c])));
+  }
+}
+
 __global__ void wait_probe_kernel(int* status, uint64_t timeout_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -275,6 +286,22 @@ int pdl_attribute(cudaLaunchAttribute* attr) {
   return 1;
 }
 
+int launch_bias_act_fill(const GemmProblem& p) {
+  const int64_t total = p.M * p.N;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  __half* C = static_cast<__half*>(p.C);
+  const __half* bias = static_cast<const __half*>(p.bias);
+  const int g = static_cast<int>(blocks);
+  if (p.act == kActRelu)
+    bias_act_fill_kernel<kActRelu><<<g, 256, 0, p.stream>>>(C, bias, p.M, p.N, p.ldc);
+  else if (p.act == kActGelu)
+    bias_act_fill_kernel<kActGelu><<<g, 256, 0, p.stream>>>(C, bias, p.M, p.N, p.ldc);
+  else
+    bias_act_fill_kernel<kActNone><<<g, 256, 0, p.stream>>>(C, bias, p.M, p.N, p.ldc);
+  return cudaGetLastError() == cudaSuccess ? GEMM_OK : GEMM_ERR_LAUNCH;
+}
+
 int launch_zero_fill(const GemmProblem& p) {
   const int64_t total = p.M * p.N;
   int64_t blocks = (total + 255) / 256;
@@ -314,12 +341,14 @@ const char* gemm_status_string(int status) {
   }
 }
 
-int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
-                int64_t lda, int64_t ldb, int64_t ldc, int relu, int path,
-                gemm_stream_t stream) {
+int gemm_bias_act_f16(const void* A, const void* B, const void* bias, void* C, int64_t M,
+                      int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                      int activation, int path, gemm_stream_t stream) {
   if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return GEMM_ERR_INVALID_ARG;
-  if (relu != 0 && relu != 1) return GEMM_ERR_INVALID_ARG;
+  if (activation != GEMM_ACT_NONE && activation != GEMM_ACT_RELU &&
+      activation != GEMM_ACT_GELU)
+    return GEMM_ERR_INVALID_ARG;
   if (path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE && path != GEMM_PATH_SKINNY &&
       path != GEMM_PATH_TILE_PAIR)
     return GEMM_ERR_INVALID_ARG;
@@ -330,8 +359,16 @@ int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int
   load_entry_points();
   rc = check_matrix(C, M, N, ldc, d.device);
   if (rc != GEMM_OK) return rc;
-  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, relu != 0, stream};
-  if (K == 0) return launch_zero_fill(p);
+  if (bias != nullptr) {
+    // one row of N fp16 values, 16-byte aligned
+    rc = check_matrix(bias, 1, N, (N + 7) / 8 * 8, d.device);
+    if (rc != GEMM_OK) return rc;
+  }
+  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, activation, bias, stream};
+  if (K == 0) {
+    // the empty sum is +0: C = act(bias), or +0 without a bias (act(0) = +0)
+    return bias != nullptr ? launch_bias_act_fill(p) : launch_zero_fill(p);
+  }
   rc = check_matrix(A, M, K, lda, d.device);
   if (rc == GEMM_OK) rc = check_matrix(B, K, N, ldb, d.device);
   if (rc != GEMM_OK) return rc;
@@ -346,6 +383,14 @@ int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int
   }
   if (path == GEMM_PATH_TILE_PAIR) return launch_tile_pair_gemm(p, d);
   return launch_tile_gemm(p, d);
+}
+
+int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                int64_t lda, int64_t ldb, int64_t ldc, int relu, int path,
+                gemm_stream_t stream) {
+  if (relu != 0 && relu != 1) return GEMM_ERR_INVALID_ARG;
+  return gemm_bias_act_f16(A, B, nullptr, C, M, N, K, lda, ldb, ldc,
+                           relu ? GEMM_ACT_RELU : GEMM_ACT_NONE, path, stream);
 }
 
 int gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
@@ -373,7 +418,7 @@ int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_t M, int6
   load_entry_points();
   rc = check_matrix(C, M, N, ldc, d.device);
   if (rc != GEMM_OK) return rc;
-  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, true, stream};
+  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, GEMM_ACT_RELU, nullptr, stream};
   if (K == 0) return launch_zero_fill(p);
   rc = check_matrix(A, M, K, lda, d.device);
   if (rc == GEMM_OK) rc = check_matrix(B, K, N, ldb, d.device);

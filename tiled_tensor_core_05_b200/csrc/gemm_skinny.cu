@@ -27,7 +27,6 @@
 //     slice order (deterministic), then applies ReLU -- only after the full K
 //     reduction -- and stores fp16.  No CTA ever waits for another.
 #include <atomic>
-#include <cstdlib>
 #include <mutex>
 
 #include "../../include/gemm_f16.h"
@@ -64,14 +63,17 @@ __device__ __forceinline__ float4 ld_cg_f4(const float* p) {
   return __ldcg(reinterpret_cast<const float4*>(p));
 }
 
-template <int MP, bool RELU>
+// Column n of C (rows m < M): activation of the fp32 sums plus the column's
+// bias, rounded to fp16.
+template <int MP, int ACT>
 __device__ __forceinline__ void store_column(const float (&v)[MP], __half* C, int M, int N,
-                                             int64_t ldc, int n) {
+                                             int64_t ldc, int n, const __half* bias) {
   if (n >= N) return;
+  const float b = bias != nullptr ? __half2float(bias[n]) : 0.0f;
 #pragma unroll
   for (int m = 0; m < MP; ++m) {
     if (m < M) {
-      const float x = RELU ? relu_f32(v[m]) : v[m];
+      const float x = activate<ACT>(v[m] + b);
       C[static_cast<int64_t>(m) * ldc + n] = __float2half_rn(x);
     }
   }
@@ -90,15 +92,16 @@ __device__ __forceinline__ void load_accumulator(uint32_t taddr, float (&v)[MP])
   }
 }
 
-// One CTA per (tile, k-slice); blockIdx.x = tile * S + slice.  HINT = 1 loads
-// B (streamed once) with an L2 evict-first policy and A (re-read by every
-// CTA) with evict-last.
-template <int MP, int STAGES, int HINT, bool RELU>
+// One CTA per (tile, k-slice); blockIdx.x = tile * S + slice.  B (streamed
+// once) is loaded with an L2 evict-first policy and A (re-read by every CTA)
+// with evict-last.
+template <int MP, int STAGES, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, __half* __restrict__ C, int M,
-                       int N, int K, int64_t ldc, int S, float* __restrict__ partials,
-                       int* __restrict__ counters, int* status, uint64_t timeout_ns) {
+                       int N, int K, int64_t ldc, const __half* __restrict__ bias, int S,
+                       float* __restrict__ partials, int* __restrict__ counters, int* status,
+                       uint64_t timeout_ns) {
   using Cfg = SkinnyCfg<MP, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -155,8 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
-      const uint64_t pol_b = HINT ? l2_policy_evict_first() : 0;
-      const uint64_t pol_a = HINT ? l2_policy_evict_last() : 0;
+      const uint64_t pol_b = l2_policy_evict_first();
+      const uint64_t pol_a = l2_policy_evict_last();
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
           ok = false;
@@ -164,19 +167,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
         uint8_t* bdst = smB + stage * Cfg::kBBytes;
-        if (HINT) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tma_load_2d_hint(&tmB, &full[stage], bdst + j * Cfg::kBChunk, tile * kTW + j * 64,
-                             kb * kBK, pol_b);
-          tma_load_2d_hint(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, 0, pol_a);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tma_load_2d(&tmB, &full[stage], bdst + j * Cfg::kBChunk, tile * kTW + j * 64,
-                        kb * kBK);
-          tma_load_2d(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, 0);
-        }
+        for (int j = 0; j < 4; ++j)
+          tma_load_2d_hint(&tmB, &full[stage], bdst + j * Cfg::kBChunk, tile * kTW + j * 64,
+                           kb * kBK, pol_b);
+        tma_load_2d_hint(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, 0, pol_a);
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) {
@@ -255,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < 2; ++h) {
           float v[MP];
           load_accumulator<MP>(t_lane + static_cast<uint32_t>(h * MP), v);
-          store_column<MP, RELU>(v, C, M, N, ldc, n0 + h * kSub);
+          store_column<MP, ACT>(v, C, M, N, ldc, n0 + h * kSub, bias);
         }
       } else {
         // partial tile of this slice: [item][256 columns][MP]
@@ -302,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-            store_column<MP, RELU>(acc, C, M, N, ldc, n0 + h * kSub);
+            store_column<MP, ACT>(acc, C, M, N, ldc, n0 + h * kSub, bias);
           }
         }
       }
@@ -345,7 +340,7 @@ int choose_slices(int64_t tiles, int64_t KB, int sm_count, int64_t max_items) {
   return s < 1 ? 1 : static_cast<int>(s);
 }
 
-template <int MP, int STAGES, int HINT, bool RELU>
+template <int MP, int STAGES, int ACT>
 int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
                 int64_t max_items) {
   using Cfg = SkinnyCfg<MP, STAGES>;
@@ -368,7 +363,7 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_by
   int rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, MP);
   if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
   if (rc != 0) return rc;
-  auto kern = skinny_gemm_kernel<MP, STAGES, HINT, RELU>;
+  auto kern = skinny_gemm_kernel<MP, STAGES, ACT>;
   if (!ensure_smem_attr_skinny(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
                                attr_done))
     return GEMM_ERR_LAUNCH;
@@ -384,8 +379,8 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_by
   cfg.numAttrs = pdl_attribute(&attr[0]);
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, static_cast<__half*>(p.C), static_cast<int>(p.M),
-      static_cast<int>(p.N), static_cast<int>(p.K), p.ldc, S, partials, counters, d.status,
-      d.timeout_ns);
+      static_cast<int>(p.N), static_cast<int>(p.K), p.ldc, static_cast<const __half*>(p.bias), S,
+      partials, counters, d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? GEMM_OK : GEMM_ERR_LAUNCH;
 }
 
@@ -404,36 +399,21 @@ size_t skinny_workspace_bytes(int sm_count, int m_pad) {
          static_cast<size_t>(sm_count) * kTW * static_cast<size_t>(m_pad) * sizeof(float);
 }
 
-// Small-M configuration for M <= 32 (TTC_SKINNY_CFG selects another one in
-// tuning sweeps): 0 = 5 stages with L2 hints (measured best on the decode
-// shape: 72.7 us vs 75.2 us for 6 stages without hints); 1 = 6 stages with
-// hints; 2 = 6 stages without hints; 3 = 4 stages with hints.
-int skinny_cfg_setting() {
-  static const int c = [] {
-    const char* s = std::getenv("TTC_SKINNY_CFG");
-    const int v = s ? std::atoi(s) : 0;
-    return (v >= 0 && v <= 3) ? v : 0;
-  }();
-  return c;
-}
-
-template <bool RELU>
-int launch_mp32(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes) {
-  switch (skinny_cfg_setting()) {
-    case 1: return launch_impl<32, 6, 1, RELU>(p, d, ws, ws_bytes, d.sm_count);
-    case 2: return launch_impl<32, 6, 0, RELU>(p, d, ws, ws_bytes, d.sm_count);
-    case 3: return launch_impl<32, 4, 1, RELU>(p, d, ws, ws_bytes, d.sm_count);
-    default: return launch_impl<32, 5, 1, RELU>(p, d, ws, ws_bytes, d.sm_count);
+// 5 stages with L2 hints: measured best on the decode shape (72.7 us against
+// 75.2 us for 6 stages without hints, 73.5-75.0 us for 4 or 6 stages with).
+template <int MP>
+int launch_mp(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes) {
+  switch (p.act) {
+    case kActRelu: return launch_impl<MP, 5, kActRelu>(p, d, ws, ws_bytes, d.sm_count);
+    case kActGelu: return launch_impl<MP, 5, kActGelu>(p, d, ws, ws_bytes, d.sm_count);
+    default: return launch_impl<MP, 5, kActNone>(p, d, ws, ws_bytes, d.sm_count);
   }
 }
 
 int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes) {
   const int mp = skinny_m_pad(p.M);
-  if (mp == 32)
-    return p.relu ? launch_mp32<true>(p, d, ws, ws_bytes) : launch_mp32<false>(p, d, ws, ws_bytes);
-  if (mp == 64)
-    return p.relu ? launch_impl<64, 5, 1, true>(p, d, ws, ws_bytes, d.sm_count)
-                  : launch_impl<64, 5, 1, false>(p, d, ws, ws_bytes, d.sm_count);
+  if (mp == 32) return launch_mp<32>(p, d, ws, ws_bytes);
+  if (mp == 64) return launch_mp<64>(p, d, ws, ws_bytes);
   return GEMM_ERR_INVALID_ARG;
 }
 
@@ -485,7 +465,7 @@ int launch_skinny_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d) {
   if (cudaMemsetAsync(scratch, 0, kNoAllocCounterBytes, p.stream) != cudaSuccess)
     return GEMM_ERR_LAUNCH;
   const int64_t items = d.sm_count < kNoAllocMaxItems ? d.sm_count : kNoAllocMaxItems;
-  return launch_impl<kNoAllocMP, 5, 1, true>(p, d, scratch, kNoAllocScratchBytes, items);
+  return launch_impl<kNoAllocMP, 5, kActRelu>(p, d, scratch, kNoAllocScratchBytes, items);
 }
 
 }  // namespace ttc

@@ -95,13 +95,30 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
 // buffered per warp).  Columns at and beyond N rounded down to 8 (the TMA
 // store writes whole 16-byte groups) are written with plain stores.
 // `release()` runs once the last TMEM load of the tile has completed.
-template <int BN, bool RELU, class Release>
+// `bias` (N fp16 values or null) is added per column before the activation.
+template <int BN, int ACT, class Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uint32_t& chunk_no,
                                               const CUtensorMap* tmC, __half* C, int64_t ldc,
-                                              int M, int N, int n8, int row0, int col_base,
-                                              int lane, Release release) {
+                                              const __half* __restrict__ bias, int M, int N,
+                                              int n8, int row0, int col_base, int lane,
+                                              Release release) {
 #pragma unroll 1
   for (int c = 0; c < BN / kEpiCols; ++c) {
+    // the 64 bias values of this chunk as 32 packed pairs (0 past N)
+    uint32_t bb[32];
+    if (bias != nullptr) {
+      const int col0 = col_base + c * kEpiCols;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int col = col0 + 2 * i;
+        if (col + 1 < N) {
+          bb[i] = __ldg(reinterpret_cast<const unsigned int*>(bias + col));
+        } else {
+          const unsigned short lo = col < N ? __ldg(reinterpret_cast<const unsigned short*>(bias + col)) : 0;
+          bb[i] = lo;
+        }
+      }
+    }
     uint32_t v0[32], v1[32];
     tmem_ld_32x32b_x32(t_row + c * kEpiCols, v0);
     tmem_ld_32x32b_x32(t_row + c * kEpiCols + 32, v1);
@@ -117,14 +134,16 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
     for (int i = 0; i < 16; ++i) {
       float x0 = __uint_as_float(v0[2 * i]), x1 = __uint_as_float(v0[2 * i + 1]);
       float y0 = __uint_as_float(v1[2 * i]), y1 = __uint_as_float(v1[2 * i + 1]);
-      if (RELU) {
-        x0 = relu_f32(x0);
-        x1 = relu_f32(x1);
-        y0 = relu_f32(y0);
-        y1 = relu_f32(y1);
+      if (bias != nullptr) {
+        const float2 bx = __half22float2(*reinterpret_cast<const __half2*>(&bb[i]));
+        const float2 by = __half22float2(*reinterpret_cast<const __half2*>(&bb[16 + i]));
+        x0 += bx.x;
+        x1 += bx.y;
+        y0 += by.x;
+        y1 += by.y;
       }
-      h[i] = pack_half2(x0, x1);
-      h[16 + i] = pack_half2(y0, y1);
+      h[i] = pack_half2(activate<ACT>(x0), activate<ACT>(x1));
+      h[16 + i] = pack_half2(activate<ACT>(y0), activate<ACT>(y1));
     }
     uint8_t* buf = bufs + (chunk_no & 1u) * kEpiBuf;
     if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
@@ -159,13 +178,13 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
   }
 }
 
-template <int BN, int STAGES, bool RELU>
+template <int BN, int STAGES, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
-                     int64_t ldc, int M, int N, int K, int group_m, int* status,
-                     uint64_t timeout_ns) {
+                     int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
+                     int group_m, int* status, uint64_t timeout_ns) {
   using Cfg = TileCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -333,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       uint64_t* release_bar = &acc_empty[acc];
-      epilogue_tile<BN, RELU>(t_row, bufs, chunk_no, &tmC, C, ldc, M, N, n8, row0, nb * BN,
-                              lane, [release_bar] { mbar_arrive(release_bar); });
+      epilogue_tile<BN, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
+                             nb * BN, lane, [release_bar] { mbar_arrive(release_bar); });
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -367,13 +386,13 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 //     that an accumulator is ready (multicast arrive);
 //   * each CTA's four epilogue warps drain its own TMEM rows and arrive on the
 //     leader's acc_empty barrier (8 arrivals per accumulator use).
-template <int STAGES, bool RELU>
+template <int STAGES, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
-                          int64_t ldc, int M, int N, int K, int group_m, int* status,
-                          uint64_t timeout_ns) {
+                          int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
+                          int group_m, int* status, uint64_t timeout_ns) {
   using Cfg = PairCfg<STAGES>;
   constexpr int BN = Cfg::kBN;
   extern __shared__ uint8_t smem_raw[];
@@ -550,8 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       const uint32_t release_bar = acc_empty_leader + acc * 8;
-      epilogue_tile<BN, RELU>(t_row, bufs, chunk_no, &tmC, C, ldc, M, N, n8, row0, nb * BN,
-                              lane, [release_bar] { mbar_arrive_cluster(release_bar); });
+      epilogue_tile<BN, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
+                             nb * BN, lane, [release_bar] { mbar_arrive_cluster(release_bar); });
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -596,7 +615,7 @@ int group_tiles(int tile_rows) {
   return g > 0 ? g : 1;
 }
 
-template <int BN, int STAGES, bool RELU>
+template <int BN, int STAGES, int ACT>
 int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   using Cfg = TileCfg<BN, STAGES>;
   static std::atomic<uint64_t> attr_done{0};
@@ -608,7 +627,7 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   const uint64_t n8 = static_cast<uint64_t>(p.N) & ~7ull;
   if (rc == 0) rc = encode_tmap_f16_2d(&tC, p.C, n8 > 0 ? n8 : 8, p.M, p.ldc, kEpiCols, kEpiRows);
   if (rc != 0) return rc;
-  auto kern = tile_gemm_kernel<BN, STAGES, RELU>;
+  auto kern = tile_gemm_kernel<BN, STAGES, ACT>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
                         attr_done))
     return GEMM_ERR_LAUNCH;
@@ -623,12 +642,13 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   cfg.attrs = attr;
   cfg.numAttrs = pdl_attribute(&attr[0]);
   const cudaError_t e = cudaLaunchKernelEx(
-      &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc, static_cast<int>(p.M),
-      static_cast<int>(p.N), static_cast<int>(p.K), group_tiles(kBM), d.status, d.timeout_ns);
+      &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
+      static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
+      static_cast<int>(p.K), group_tiles(kBM), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
-template <int STAGES, bool RELU>
+template <int STAGES, int ACT>
 int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   using Cfg = PairCfg<STAGES>;
   static std::atomic<uint64_t> attr_done{0};
@@ -639,7 +659,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   const uint64_t n8 = static_cast<uint64_t>(p.N) & ~7ull;
   if (rc == 0) rc = encode_tmap_f16_2d(&tC, p.C, n8 > 0 ? n8 : 8, p.M, p.ldc, kEpiCols, kEpiRows);
   if (rc != 0) return rc;
-  auto kern = tile_pair_gemm_kernel<STAGES, RELU>;
+  auto kern = tile_pair_gemm_kernel<STAGES, ACT>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
                         attr_done))
     return GEMM_ERR_LAUNCH;
@@ -670,9 +690,9 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.numAttrs = 1 + pdl_attribute(&attr[1]);
   const cudaError_t e = cudaLaunchKernelEx(
-      &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc, static_cast<int>(p.M),
-      static_cast<int>(p.N), static_cast<int>(p.K), group_tiles(2 * kBM), d.status,
-      d.timeout_ns);
+      &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
+      static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
+      static_cast<int>(p.K), group_tiles(2 * kBM), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
@@ -683,12 +703,22 @@ int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d) {
   // 128 x 128 tiles (twice as many CTAs for small problems).
   const int64_t tiles256 = ((p.M + kBM - 1) / kBM) * ((p.N + 255) / 256);
   const bool wide = tiles256 >= d.sm_count;
-  if (wide) return p.relu ? launch_impl<256, 4, true>(p, d) : launch_impl<256, 4, false>(p, d);
-  return p.relu ? launch_impl<128, 6, true>(p, d) : launch_impl<128, 6, false>(p, d);
+  switch (p.act) {
+    case kActRelu:
+      return wide ? launch_impl<256, 4, kActRelu>(p, d) : launch_impl<128, 6, kActRelu>(p, d);
+    case kActGelu:
+      return wide ? launch_impl<256, 4, kActGelu>(p, d) : launch_impl<128, 6, kActGelu>(p, d);
+    default:
+      return wide ? launch_impl<256, 4, kActNone>(p, d) : launch_impl<128, 6, kActNone>(p, d);
+  }
 }
 
 int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d) {
-  return p.relu ? launch_pair_impl<6, true>(p, d) : launch_pair_impl<6, false>(p, d);
+  switch (p.act) {
+    case kActRelu: return launch_pair_impl<6, kActRelu>(p, d);
+    case kActGelu: return launch_pair_impl<6, kActGelu>(p, d);
+    default: return launch_pair_impl<6, kActNone>(p, d);
+  }
 }
 
 }  // namespace ttc

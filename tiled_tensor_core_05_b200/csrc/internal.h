@@ -13,7 +13,8 @@ struct GemmProblem {
   void* C;
   int64_t M, N, K;
   int64_t lda, ldb, ldc;
-  bool relu;
+  int act;             // kActNone / kActRelu / kActGelu (sm100.cuh), = gemm_activation
+  const void* bias;    // N fp16 values added per column before the activation, or null
   cudaStream_t stream;
 };
 
@@ -60,5 +61,7 @@ int launch_skinny_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d);
 
 // Writes C = 0 (used when K == 0: the empty sum, and ReLU of it, is +0).
 int launch_zero_fill(const GemmProblem& p);
+// Writes C[i, j] = act(bias[j]) (K == 0 with a bias).
+int launch_bias_act_fill(const GemmProblem& p);
 
 }  // namespace ttc

@@ -285,6 +285,21 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 // max(x, 0) that maps -0 and NaN to +0.
 __device__ __forceinline__ float relu_f32(float x) { return x > 0.0f ? x : 0.0f; }
 
+// Epilogue activations: kActRelu as above; kActGelu is x * Phi(x) with the
+// standard normal CDF Phi(x) = erfc(-x / sqrt(2)) / 2 (CUDA's erfcf).
+enum : int { kActNone = 0, kActRelu = 1, kActGelu = 2 };
+
+template <int ACT>
+__device__ __forceinline__ float activate(float x) {
+  if constexpr (ACT == kActRelu) {
+    return relu_f32(x);
+  } else if constexpr (ACT == kActGelu) {
+    return x * (0.5f * erfcf(x * -0.7071067811865476f));
+  } else {
+    return x;
+  }
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),

@@ -20,6 +20,8 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libttc05.so")
 
 PATH_AUTO, PATH_TILE, PATH_SKINNY, PATH_TILE_PAIR = 0, 1, 2, 3
+ACT_NONE, ACT_RELU, ACT_GELU = 0, 1, 2
+_ACTS = {"none": ACT_NONE, "relu": ACT_RELU, "gelu": ACT_GELU}
 
 _lib = None
 
@@ -30,6 +32,8 @@ _SIGNATURES = {
                  ctypes.c_int),
     "gemm_f16_ex": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 +
                     [ctypes.c_int, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
+    "gemm_bias_act_f16": ([ctypes.c_void_p] * 4 + [ctypes.c_int64] * 6 +
+                          [ctypes.c_int, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
     "gemm_select_path": ([ctypes.c_int64] * 3, ctypes.c_int),
     "gemm_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "gemm_get_device_status": ([ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -110,6 +114,35 @@ def gemm_f16_ex(a: torch.Tensor, b: torch.Tensor, out: torch.Tensor | None = Non
                                _ld_padded(a), _ld_padded(b), _ld_padded(out), int(bool(relu)),
                                int(path), _stream_handle(stream, dev))
     _check(rc, "gemm_f16_ex")
+    return out
+
+
+def gemm_bias_act_f16(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None,
+                      act: str | int = "gelu", out: torch.Tensor | None = None, *,
+                      path: int = PATH_AUTO, stream=None) -> torch.Tensor:
+    """C = act(A @ B + bias) with a per-column fp16 bias (or None) and act in
+    "none" / "relu" / "gelu" (exact GELU), fused into the GEMM epilogue."""
+    if a.dtype != torch.float16 or b.dtype != torch.float16:
+        raise TypeError("a and b must be torch.float16")
+    M, K = a.shape
+    K2, N = b.shape
+    if K != K2:
+        raise ValueError(f"shape mismatch {tuple(a.shape)} @ {tuple(b.shape)}")
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    if bias is not None:
+        if bias.dtype != torch.float16 or bias.numel() != N or not bias.is_cuda:
+            raise ValueError("bias must be a CUDA fp16 tensor with N elements")
+        if bias.dim() != 1 and not bias.is_contiguous():
+            raise ValueError("bias must be contiguous")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
+    dev = a.device
+    with torch.cuda.device(dev):
+        rc = lib().gemm_bias_act_f16(a.data_ptr(), b.data_ptr(),
+                                     None if bias is None else bias.data_ptr(), out.data_ptr(),
+                                     M, N, K, _ld_padded(a), _ld_padded(b), _ld_padded(out),
+                                     code, int(path), _stream_handle(stream, dev))
+    _check(rc, "gemm_bias_act_f16")
     return out
 
 
