@@ -25,7 +25,8 @@ from . import build as _build
 
 __all__ = [
     "gemm_relu", "gemm", "gemm_relu_at", "gemm_at", "gemm_f64_at",
-    "gemm_bias_act", "activation_f64", "decode_f16", "encode_f16", "max_threads",
+    "gemm_bias_act", "gemm_general", "activation_f64", "decode_f16", "encode_f16",
+    "max_threads",
 ]
 
 _lib = None
@@ -53,6 +54,10 @@ def _load():
         lib.oracle_gemm_bias_act_f16.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64,
                                                  ctypes.c_int, ctypes.c_int]
         lib.oracle_gemm_bias_act_f16.restype = ctypes.c_int
+        lib.oracle_gemm_general_f16.argtypes = [p, p, p, p, i64, i64, i64, i64, i64, i64,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int]
+        lib.oracle_gemm_general_f16.restype = ctypes.c_int
         lib.oracle_activation_f64.argtypes = [p, p, i64, ctypes.c_int]
         lib.oracle_activation_f64.restype = None
         lib.oracle_max_threads.argtypes = []
@@ -213,6 +218,34 @@ def gemm_bias_act(a, b, bias=None, act="gelu", nthreads=None) -> np.ndarray:
                                           M, N, K, _ld(a), _ld(b), N, code, _threads(nthreads))
     if rc != 0:
         raise RuntimeError(f"oracle_gemm_bias_act_f16 failed ({rc})")
+    return c.view(np.float16)
+
+
+def gemm_general(a, b, bias=None, act="relu", trans_a=False, trans_b=False,
+                 nthreads=None) -> np.ndarray:
+    """act(op(A) @ op(B) + bias): with trans_a the stored ``a`` is K x M and
+    op(A) = a.T; with trans_b the stored ``b`` is N x K and op(B) = b.T."""
+    a, b = _bits(a), _bits(b)
+    M, K = (a.shape[1], a.shape[0]) if trans_a else a.shape
+    K2, N = (b.shape[1], b.shape[0]) if trans_b else b.shape
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    c = np.zeros((M, N), dtype=np.uint16)
+    if M == 0 or N == 0:
+        return c.view(np.float16)
+    bias_ptr = None
+    if bias is not None:
+        bias = bias.detach().reshape(1, -1) if hasattr(bias, "detach") else np.asarray(bias).reshape(1, -1)
+        bb = np.ascontiguousarray(_bits(bias))
+        if bb.shape[1] != N:
+            raise ValueError("bias must have N elements")
+        bias_ptr = bb.ctypes.data
+    rc = _load().oracle_gemm_general_f16(a.ctypes.data, b.ctypes.data, bias_ptr, c.ctypes.data,
+                                         M, N, K, _ld(a), _ld(b), N, int(bool(trans_a)),
+                                         int(bool(trans_b)), code, _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_gemm_general_f16 failed ({rc})")
     return c.view(np.float16)
 
 

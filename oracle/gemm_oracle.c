@@ -281,6 +281,43 @@ int oracle_gemm_bias_act_f16(const uint16_t* A, const uint16_t* B, const uint16_
     return failed ? -1 : 0;
 }
 
+/* ---- operand layouts ----------------------------------------------------- */
+/* T.gemm's transpose_A / transpose_B options ("Writing high-performance
+ * kernels in TileLang", atlascloud.ai blog, section "Escribamos un GEMM"):
+ * op(A) is M x K and op(B) is K x N, with
+ *   trans_a = 0: A stored M x K row-major (A[i,k] at A + i*lda + k)
+ *   trans_a = 1: A stored K x M row-major (op(A)[i,k] at A + k*lda + i)
+ *   trans_b = 0: B stored K x N row-major (B[k,j] at B + k*ldb + j)
+ *   trans_b = 1: B stored N x K row-major (op(B)[k,j] at B + j*ldb + k)
+ * C = fp16_RNE(act(sum_k op(A)[i,k] op(B)[k,j] + bias[j])), ascending k in
+ * fp64, one element at a time. */
+int oracle_gemm_general_f16(const uint16_t* A, const uint16_t* B, const uint16_t* bias,
+                            uint16_t* C, int64_t M, int64_t N, int64_t K,
+                            int64_t lda, int64_t ldb, int64_t ldc,
+                            int trans_a, int trans_b, int act, int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0 || act < 0 || act > 2) return -1;
+    if (M == 0 || N == 0) return 0;
+    if (lda < (trans_a ? M : K) || ldb < (trans_b ? K : N) || ldc < N) return -1;
+    double* tab = decode_table();
+    if (!tab) return -1;
+    const int64_t sa_i = trans_a ? 1 : lda, sa_k = trans_a ? lda : 1;
+    const int64_t sb_k = trans_b ? 1 : ldb, sb_j = trans_b ? ldb : 1;
+    const int nt = resolve_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (int64_t i = 0; i < M; ++i) {
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += tab[A[i * sa_i + k * sa_k]] * tab[B[k * sb_k + j * sb_j]];
+            const double x = acc + (bias ? tab[bias[j]] : 0.0);
+            C[i * ldc + j] = oracle_f64_to_f16(act64(x, act));
+        }
+    }
+    free(tab);
+    return 0;
+}
+
 /* The activations alone on fp64 inputs (unrounded), for pinning act64. */
 void oracle_activation_f64(const double* in, double* out, int64_t n, int act)
 {
