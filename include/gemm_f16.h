@@ -114,6 +114,20 @@ GEMM_API int gemm_bias_act_f16(const void* A, const void* B, const void* bias, v
                                int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
                                int64_t ldc, int activation, int path, gemm_stream_t stream);
 
+/* C = act(op(A) @ op(B) + bias) with T.gemm's transpose_A / transpose_B
+ * options ("Writing high-performance kernels in TileLang", atlascloud.ai
+ * blog, section "Escribamos un GEMM"):
+ *   trans_a = 0: A stored M x K row-major, lda >= K;
+ *   trans_a = 1: A stored K x M row-major (M contiguous), lda >= M, op(A) = A^T;
+ *   trans_b = 0: B stored K x N row-major, ldb >= N;
+ *   trans_b = 1: B stored N x K row-major (K contiguous, the layout of a
+ *                linear layer's weight), ldb >= K, op(B) = B^T.
+ * Everything else as in gemm_bias_act_f16 (which is trans_a = trans_b = 0). */
+GEMM_API int gemm_f16_general(const void* A, const void* B, const void* bias, void* C,
+                              int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                              int64_t ldc, int trans_a, int trans_b, int activation, int path,
+                              gemm_stream_t stream);
+
 /* The path GEMM_PATH_AUTO takes for this shape (GEMM_PATH_TILE,
  * GEMM_PATH_TILE_PAIR or GEMM_PATH_SKINNY).  Pure host function. */
 GEMM_API int gemm_select_path(int64_t M, int64_t N, int64_t K);

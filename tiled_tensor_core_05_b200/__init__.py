@@ -10,7 +10,8 @@ used on machines without a GPU); the first call does.
 """
 from __future__ import annotations
 
-__all__ = ["gemm_relu_f16", "gemm_f16", "gemm_f16_ex", "gemm_bias_act_f16", "lib"]
+__all__ = ["gemm_relu_f16", "gemm_f16", "gemm_f16_ex", "gemm_bias_act_f16", "gemm_general",
+           "lib"]
 
 
 def __getattr__(name):

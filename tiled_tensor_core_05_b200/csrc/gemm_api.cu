@@ -341,10 +341,12 @@ const char* gemm_status_string(int status) {
   }
 }
 
-int gemm_bias_act_f16(const void* A, const void* B, const void* bias, void* C, int64_t M,
-                      int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
-                      int activation, int path, gemm_stream_t stream) {
+int gemm_f16_general(const void* A, const void* B, const void* bias, void* C, int64_t M,
+                     int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int trans_a,
+                     int trans_b, int activation, int path, gemm_stream_t stream) {
   if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
+  if ((trans_a != 0 && trans_a != 1) || (trans_b != 0 && trans_b != 1))
+    return GEMM_ERR_INVALID_ARG;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return GEMM_ERR_INVALID_ARG;
   if (activation != GEMM_ACT_NONE && activation != GEMM_ACT_RELU &&
       activation != GEMM_ACT_GELU)
@@ -364,13 +366,16 @@ int gemm_bias_act_f16(const void* A, const void* B, const void* bias, void* C, i
     rc = check_matrix(bias, 1, N, (N + 7) / 8 * 8, d.device);
     if (rc != GEMM_OK) return rc;
   }
-  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, activation, bias, stream};
+  const int layout = (trans_a ? kLayoutTransA : 0) | (trans_b ? kLayoutTransB : 0);
+  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, activation, bias, layout, stream};
   if (K == 0) {
     // the empty sum is +0: C = act(bias), or +0 without a bias (act(0) = +0)
     return bias != nullptr ? launch_bias_act_fill(p) : launch_zero_fill(p);
   }
-  rc = check_matrix(A, M, K, lda, d.device);
-  if (rc == GEMM_OK) rc = check_matrix(B, K, N, ldb, d.device);
+  // stored shapes: A is K x M when transposed, B is N x K when transposed
+  rc = trans_a ? check_matrix(A, K, M, lda, d.device) : check_matrix(A, M, K, lda, d.device);
+  if (rc == GEMM_OK)
+    rc = trans_b ? check_matrix(B, N, K, ldb, d.device) : check_matrix(B, K, N, ldb, d.device);
   if (rc != GEMM_OK) return rc;
   if (path == GEMM_PATH_AUTO) path = gemm_select_path(M, N, K);
   if (path == GEMM_PATH_SKINNY) {
@@ -383,6 +388,13 @@ int gemm_bias_act_f16(const void* A, const void* B, const void* bias, void* C, i
   }
   if (path == GEMM_PATH_TILE_PAIR) return launch_tile_pair_gemm(p, d);
   return launch_tile_gemm(p, d);
+}
+
+int gemm_bias_act_f16(const void* A, const void* B, const void* bias, void* C, int64_t M,
+                      int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                      int activation, int path, gemm_stream_t stream) {
+  return gemm_f16_general(A, B, bias, C, M, N, K, lda, ldb, ldc, 0, 0, activation, path,
+                          stream);
 }
 
 int gemm_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
@@ -418,7 +430,7 @@ int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_t M, int6
   load_entry_points();
   rc = check_matrix(C, M, N, ldc, d.device);
   if (rc != GEMM_OK) return rc;
-  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, GEMM_ACT_RELU, nullptr, stream};
+  GemmProblem p{A, B, C, M, N, K, lda, ldb, ldc, GEMM_ACT_RELU, nullptr, 0, stream};
   if (K == 0) return launch_zero_fill(p);
   rc = check_matrix(A, M, K, lda, d.device);
   if (rc == GEMM_OK) rc = check_matrix(B, K, N, ldb, d.device);

@@ -47,13 +47,14 @@ template <int MP, int STAGES>
 struct SkinnyCfg {
   static constexpr int kBChunk = kBK * 64 * 2;    // 64 columns x 64 k-rows = 8 KiB
   static constexpr int kBBytes = 4 * kBChunk;     // 256 columns
-  static constexpr int kABytes = MP * kBK * 2;    // MP rows x 128 bytes
+  // A^T: MP rows x 128 bytes (A stored M x K), or one 64-column slab of 64
+  // k-rows (A stored K x M): room for the larger
+  static constexpr int kABytesK = MP * kBK * 2;
+  static constexpr int kABytes = kABytesK > 8192 ? kABytesK : 8192;
   static constexpr int kStageBytes = kBBytes + kABytes;
   static constexpr int kNumBars = 2 * STAGES + 3;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kNumBars * 8 + 16;
   static constexpr uint32_t kTmemCols = (2 * MP < 32) ? 32 : 2 * MP;
-  static constexpr uint32_t kIdesc = idesc_f16_f32(kSub, MP, /*A MN-major*/ true,
-                                                   /*B MN-major*/ false);
   static_assert(MP == 32 || MP == 64, "MP");
   static_assert(kABytes % 1024 == 0, "A tile alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -100,9 +101,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, __half* __restrict__ C, int M,
                        int N, int K, int64_t ldc, const __half* __restrict__ bias, int S,
-                       float* __restrict__ partials, int* __restrict__ counters, int* status,
-                       uint64_t timeout_ns) {
+                       int layout, float* __restrict__ partials, int* __restrict__ counters,
+                       int* status, uint64_t timeout_ns) {
   using Cfg = SkinnyCfg<MP, STAGES>;
+  const bool ta = (layout & kLayoutTransA) != 0;
+  const bool tb = (layout & kLayoutTransB) != 0;
+  // bytes of one stage: 256 columns of B, and A^T as stored
+  const uint32_t stage_bytes = Cfg::kBBytes + (ta ? 8192u : static_cast<uint32_t>(Cfg::kABytesK));
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* smB = smem;
@@ -165,13 +170,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+        mbar_arrive_expect_tx(&full[stage], stage_bytes);
         uint8_t* bdst = smB + stage * Cfg::kBBytes;
+        if (!tb) {  // row-major B: four 64-column slabs of 64 k-rows
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          tma_load_2d_hint(&tmB, &full[stage], bdst + j * Cfg::kBChunk, tile * kTW + j * 64,
-                           kb * kBK, pol_b);
-        tma_load_2d_hint(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, 0, pol_a);
+          for (int j = 0; j < 4; ++j)
+            tma_load_2d_hint(&tmB, &full[stage], bdst + j * Cfg::kBChunk, tile * kTW + j * 64,
+                             kb * kBK, pol_b);
+        } else {  // B stored N x K: 256 rows of 64 k
+          tma_load_2d_hint(&tmB, &full[stage], bdst, kb * kBK, tile * kTW, pol_b);
+        }
+        if (!ta)  // A stored M x K: MP rows of 64 k
+          tma_load_2d_hint(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, 0, pol_a);
+        else  // A stored K x M: 64 k-rows of 64 m
+          tma_load_2d_hint(&tmA, &full[stage], smA + stage * Cfg::kABytes, 0, kb * kBK, pol_a);
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) {
@@ -192,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      const uint32_t idesc = idesc_f16_f32(kSub, MP, /*B^T MN-major*/ !tb, /*A^T MN-major*/ ta);
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
           ok = false;
@@ -203,13 +216,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < kBK / kUmmaK; ++k) {
           // MMA B operand = A^T tile (K-major): 32 bytes per 16 k along the row
-          const uint64_t bdesc = smem_desc_sw128(a_addr + k * (kUmmaK * 2), 16, 1024);
+          // (A^T is K-major when A is stored M x K, MN-major when stored K x M)
+          const uint64_t bdesc = operand_desc(a_addr, k, ta, Cfg::kBChunk);
 #pragma unroll
           for (int h = 0; h < kTW / kSub; ++h) {
-            // MMA A operand = B^T sub-tile h (N-major): slabs 2h, 2h+1; 16 k-rows
-            const uint64_t adesc = smem_desc_sw128(
-                b_addr + h * 2 * Cfg::kBChunk + k * (kUmmaK * 128), Cfg::kBChunk, 1024);
-            umma_f16(tmem_base + static_cast<uint32_t>(h * MP), adesc, bdesc, Cfg::kIdesc,
+            // MMA A operand = B^T sub-tile h (columns 128h..128h+127 of the
+            // tile; 16 KiB into the stage in both layouts): N-major slabs of
+            // row-major B, or K-major rows of B stored N x K
+            const uint64_t adesc = operand_desc(b_addr + h * 2 * Cfg::kBChunk, k, !tb,
+                                                Cfg::kBChunk);
+            umma_f16(tmem_base + static_cast<uint32_t>(h * MP), adesc, bdesc, idesc,
                      (kb > kb_begin || k > 0) ? 1u : 0u);
           }
         }
@@ -360,8 +376,16 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_by
                                         counter_bytes(static_cast<int>(max_items)));
   }
   CUtensorMap tA, tB;
-  int rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, MP);
-  if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
+  int rc;
+  if (p.layout & kLayoutTransA)  // stored K x M: 64 k-rows of 64 m (rows >= M read as 0)
+    rc = encode_tmap_f16_2d(&tA, p.A, p.M, p.K, p.lda, 64, kBK);
+  else  // stored M x K: MP rows of 64 k
+    rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, MP);
+  if (rc != 0) return rc;
+  if (p.layout & kLayoutTransB)  // stored N x K: 256 rows of 64 k
+    rc = encode_tmap_f16_2d(&tB, p.B, p.K, p.N, p.ldb, kBK, kTW);
+  else  // row-major: slabs of 64 columns by 64 k-rows
+    rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
   if (rc != 0) return rc;
   auto kern = skinny_gemm_kernel<MP, STAGES, ACT>;
   if (!ensure_smem_attr_skinny(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
@@ -380,7 +404,7 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_by
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, static_cast<__half*>(p.C), static_cast<int>(p.M),
       static_cast<int>(p.N), static_cast<int>(p.K), p.ldc, static_cast<const __half*>(p.bias), S,
-      partials, counters, d.status, d.timeout_ns);
+      p.layout, partials, counters, d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? GEMM_OK : GEMM_ERR_LAUNCH;
 }
 

@@ -49,8 +49,6 @@ struct TileCfg {
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
   static constexpr uint32_t kTmemCols = 2 * BN;
-  static constexpr uint32_t kIdesc = idesc_f16_f32(kBM, BN, /*A MN-major*/ false,
-                                                   /*B MN-major*/ true);
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -70,8 +68,6 @@ struct PairCfg {
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
   static constexpr uint32_t kTmemCols = 512;      // two 256-column accumulators
-  static constexpr uint32_t kIdesc = idesc_f16_f32(2 * kBM, kBN, /*A MN-major*/ false,
-                                                   /*B MN-major*/ true);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -184,8 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
                      int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
-                     int group_m, int* status, uint64_t timeout_ns) {
+                     int layout, int group_m, int* status, uint64_t timeout_ns) {
   using Cfg = TileCfg<BN, STAGES>;
+  const bool ta = (layout & kLayoutTransA) != 0;
+  const bool tb = (layout & kLayoutTransB) != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* smA = smem;
@@ -257,11 +255,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
-          tma_load_2d(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, mb * kBM);
+          uint8_t* adst = smA + stage * Cfg::kABytes;
+          if (!ta) {
+            tma_load_2d(&tmA, &full[stage], adst, kb * kBK, mb * kBM);
+          } else {  // two 64-row slabs of the M-contiguous storage
+            tma_load_2d(&tmA, &full[stage], adst, mb * kBM, kb * kBK);
+            tma_load_2d(&tmA, &full[stage], adst + Cfg::kBChunk, mb * kBM + 64, kb * kBK);
+          }
           uint8_t* bdst = smB + stage * Cfg::kBBytes;
+          if (!tb) {
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j)
-            tma_load_2d(&tmB, &full[stage], bdst + j * Cfg::kBChunk, nb * BN + j * 64, kb * kBK);
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(&tmB, &full[stage], bdst + j * Cfg::kBChunk, nb * BN + j * 64,
+                          kb * kBK);
+          } else {  // BN rows of the K-contiguous storage
+            tma_load_2d(&tmB, &full[stage], bdst, kb * kBK, nb * BN);
+          }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -286,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       int site = 0;
+      const uint32_t idesc = idesc_f16_f32(kBM, BN, ta, !tb);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
           ok = false;
@@ -305,12 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = smem_u32(smB + stage * Cfg::kBBytes);
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
-            // A: K-major, advance 16 fp16 = 32 bytes along the swizzled row.
-            const uint64_t adesc = smem_desc_sw128(a_addr + k * (kUmmaK * 2), 16, 1024);
-            // B: N-major, advance 16 k-rows of 128 bytes.
-            const uint64_t bdesc =
-                smem_desc_sw128(b_addr + k * (kUmmaK * 128), Cfg::kBChunk, 1024);
-            umma_f16(d_tmem, adesc, bdesc, Cfg::kIdesc, (kb | k) != 0 ? 1u : 0u);
+            // row-major A is K-major, row-major B is N-major (and the reverse
+            // for the transposed storages)
+            const uint64_t adesc = operand_desc(a_addr, k, ta, Cfg::kBChunk);
+            const uint64_t bdesc = operand_desc(b_addr, k, !tb, Cfg::kBChunk);
+            umma_f16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
           if (++stage == STAGES) {
@@ -392,8 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
                           int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
-                          int group_m, int* status, uint64_t timeout_ns) {
+                          int layout, int group_m, int* status, uint64_t timeout_ns) {
   using Cfg = PairCfg<STAGES>;
+  const bool ta = (layout & kLayoutTransA) != 0;
+  const bool tb = (layout & kLayoutTransB) != 0;
   constexpr int BN = Cfg::kBN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -471,10 +482,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
           const uint32_t bar = full_leader + stage * 8;
-          tma_load_2d_pair(&tmA, bar, smA + stage * Cfg::kABytes, kb * kBK, a_row);
+          uint8_t* adst = smA + stage * Cfg::kABytes;
+          if (!ta) {
+            tma_load_2d_pair(&tmA, bar, adst, kb * kBK, a_row);
+          } else {
+            tma_load_2d_pair(&tmA, bar, adst, a_row, kb * kBK);
+            tma_load_2d_pair(&tmA, bar, adst + Cfg::kBChunk, a_row + 64, kb * kBK);
+          }
           uint8_t* bdst = smB + stage * Cfg::kBBytes;
-          tma_load_2d_pair(&tmB, bar, bdst, b_col, kb * kBK);
-          tma_load_2d_pair(&tmB, bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
+          if (!tb) {
+            tma_load_2d_pair(&tmB, bar, bdst, b_col, kb * kBK);
+            tma_load_2d_pair(&tmB, bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
+          } else {
+            tma_load_2d_pair(&tmB, bar, bdst, kb * kBK, b_col);
+          }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -505,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       int site = 0;
+      const uint32_t idesc = idesc_f16_f32(2 * kBM, BN, ta, !tb);
       for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
           ok = false;
@@ -524,10 +546,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = smem_u32(smB + stage * Cfg::kBBytes);
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
-            const uint64_t adesc = smem_desc_sw128(a_addr + k * (kUmmaK * 2), 16, 1024);
-            const uint64_t bdesc =
-                smem_desc_sw128(b_addr + k * (kUmmaK * 128), Cfg::kBChunk, 1024);
-            umma_f16_pair(d_tmem, adesc, bdesc, Cfg::kIdesc, (kb | k) != 0 ? 1u : 0u);
+            const uint64_t adesc = operand_desc(a_addr, k, ta, Cfg::kBChunk);
+            const uint64_t bdesc = operand_desc(b_addr, k, !tb, Cfg::kBChunk);
+            umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit_pair(&empty[stage], 0x3);  // stage s free in both CTAs
           if (++stage == STAGES) {
@@ -600,6 +621,21 @@ bool ensure_smem_attr(const void* func, int bytes, int device, std::atomic<uint6
   return true;
 }
 
+// TMA maps of A (tile of `a_rows` rows of op(A) by 64 k) and B (64 k by
+// `b_cols` columns of op(B)) for the operand layouts of `p`.
+int encode_operand_maps(const GemmProblem& p, int a_rows, int b_cols, CUtensorMap* tA,
+                        CUtensorMap* tB) {
+  int rc;
+  if (p.layout & kLayoutTransA)  // stored K x M: boxes of 64 m by 64 k
+    rc = encode_tmap_f16_2d(tA, p.A, p.M, p.K, p.lda, 64, kBK);
+  else  // stored M x K: boxes of 64 k by a_rows m
+    rc = encode_tmap_f16_2d(tA, p.A, p.K, p.M, p.lda, kBK, a_rows);
+  if (rc != 0) return rc;
+  if (p.layout & kLayoutTransB)  // stored N x K: boxes of 64 k by b_cols n
+    return encode_tmap_f16_2d(tB, p.B, p.K, p.N, p.ldb, kBK, b_cols);
+  return encode_tmap_f16_2d(tB, p.B, p.N, p.K, p.ldb, 64, kBK);  // 64 n by 64 k
+}
+
 // Rows of A per raster panel (TTC_GROUP_ROWS overrides it for tuning sweeps).
 int group_rows_setting() {
   static const int g = [] {
@@ -620,8 +656,7 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   using Cfg = TileCfg<BN, STAGES>;
   static std::atomic<uint64_t> attr_done{0};
   CUtensorMap tA, tB, tC;
-  int rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, kBM);
-  if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
+  int rc = encode_operand_maps(p, kBM, BN, &tA, &tB);
   // inner extent N rounded down to 8 columns (see the kernel's ragged tail);
   // the map is never used when that is 0
   const uint64_t n8 = static_cast<uint64_t>(p.N) & ~7ull;
@@ -644,7 +679,7 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
-      static_cast<int>(p.K), group_tiles(kBM), d.status, d.timeout_ns);
+      static_cast<int>(p.K), p.layout, group_tiles(kBM), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
@@ -654,8 +689,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   static std::atomic<uint64_t> attr_done{0};
   static int max_pairs[64] = {};
   CUtensorMap tA, tB, tC;
-  int rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, kBM);
-  if (rc == 0) rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
+  int rc = encode_operand_maps(p, kBM, 128, &tA, &tB);  // this CTA's half: 128 columns
   const uint64_t n8 = static_cast<uint64_t>(p.N) & ~7ull;
   if (rc == 0) rc = encode_tmap_f16_2d(&tC, p.C, n8 > 0 ? n8 : 8, p.M, p.ldc, kEpiCols, kEpiRows);
   if (rc != 0) return rc;
@@ -692,7 +726,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
-      static_cast<int>(p.K), group_tiles(2 * kBM), d.status, d.timeout_ns);
+      static_cast<int>(p.K), p.layout, group_tiles(2 * kBM), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 

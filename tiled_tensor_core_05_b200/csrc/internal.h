@@ -15,6 +15,7 @@ struct GemmProblem {
   int64_t lda, ldb, ldc;
   int act;             // kActNone / kActRelu / kActGelu (sm100.cuh), = gemm_activation
   const void* bias;    // N fp16 values added per column before the activation, or null
+  int layout;          // kLayoutTransA | kLayoutTransB (sm100.cuh): transposed storages
   cudaStream_t stream;
 };
 

@@ -266,6 +266,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Descriptor of the 16-deep k step `k` of a 64-deep operand stage at `base`
+// that is either K-major (one 128-byte row of 64 k per M/N index) or MN-major
+// (64-wide M/N slabs of 64 k-rows, `slab_bytes` apart).
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k, bool mn_major,
+                                                 uint32_t slab_bytes) {
+  return mn_major ? smem_desc_sw128(base + k * (16 * 128), slab_bytes, 1024)
+                  : smem_desc_sw128(base + k * (16 * 2), 16, 1024);
+}
+
+// Operand layouts as passed to the kernels: bit 0 = A stored K x M (op(A) =
+// A^T, M contiguous), bit 1 = B stored N x K (op(B) = B^T, K contiguous).
+enum : int { kLayoutTransA = 1, kLayoutTransB = 2 };
+
 // Instruction descriptor for kind::f16 with fp16 A and B, fp32 D.
 //   bits 4-5 D format (1 = f32); 7-9 A format (0 = f16); 10-12 B format (0 = f16)
 //   bit 15 A major (1 = MN-major); bit 16 B major (1 = MN-major)

@@ -34,6 +34,8 @@ _SIGNATURES = {
                     [ctypes.c_int, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
     "gemm_bias_act_f16": ([ctypes.c_void_p] * 4 + [ctypes.c_int64] * 6 +
                           [ctypes.c_int, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
+    "gemm_f16_general": ([ctypes.c_void_p] * 4 + [ctypes.c_int64] * 6 +
+                         [ctypes.c_int] * 4 + [ctypes.c_void_p], ctypes.c_int),
     "gemm_select_path": ([ctypes.c_int64] * 3, ctypes.c_int),
     "gemm_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "gemm_get_device_status": ([ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -143,6 +145,35 @@ def gemm_bias_act_f16(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | Non
                                      M, N, K, _ld_padded(a), _ld_padded(b), _ld_padded(out),
                                      code, int(path), _stream_handle(stream, dev))
     _check(rc, "gemm_bias_act_f16")
+    return out
+
+
+def gemm_general(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None,
+                 act: str | int = "relu", out: torch.Tensor | None = None, *,
+                 trans_a: bool = False, trans_b: bool = False, path: int = PATH_AUTO,
+                 stream=None) -> torch.Tensor:
+    """C = act(op(A) @ op(B) + bias).  With trans_a the stored ``a`` is K x M
+    (op(A) = a.T); with trans_b the stored ``b`` is N x K (op(B) = b.T, the
+    layout of a linear layer's weight)."""
+    if a.dtype != torch.float16 or b.dtype != torch.float16:
+        raise TypeError("a and b must be torch.float16")
+    M, K = (a.shape[1], a.shape[0]) if trans_a else tuple(a.shape)
+    K2, N = (b.shape[1], b.shape[0]) if trans_b else tuple(b.shape)
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    if bias is not None and (bias.dtype != torch.float16 or bias.numel() != N):
+        raise ValueError("bias must be fp16 with N elements")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
+    dev = a.device
+    with torch.cuda.device(dev):
+        rc = lib().gemm_f16_general(a.data_ptr(), b.data_ptr(),
+                                    None if bias is None else bias.data_ptr(), out.data_ptr(),
+                                    M, N, K, _ld_padded(a), _ld_padded(b), _ld_padded(out),
+                                    int(bool(trans_a)), int(bool(trans_b)), code, int(path),
+                                    _stream_handle(stream, dev))
+    _check(rc, "gemm_f16_general")
     return out
 
 
