@@ -238,7 +238,10 @@ def time_launches(fn, steps: int, warmup: int, stream, dist=None, sampler=None,
 
 
 def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
-                     comparator=False):
+                     comparator=False, variant="relu", path=0):
+    """Time one workload.  variant: "relu" (gemm_relu_f16, the measured path),
+    "bias_gelu" (gemm_bias_act_f16 with a per-column bias and GELU) or "wT"
+    (gemm_f16_general with B stored N x K, ReLU)."""
     import torch
 
     from tiled_tensor_core_05_b200 import ops, workloads
@@ -249,12 +252,32 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
     stream = torch.cuda.current_stream()
     lib = ops.lib()
     h = int(stream.cuda_stream)
-    args = (a.data_ptr(), b.data_ptr(), c.data_ptr(), w.M, w.N, w.K, w.K, w.N, w.N, h)
+    bias = None
+    if variant == "relu" and path == 0:
+        fn, args = lib.gemm_relu_f16, (a.data_ptr(), b.data_ptr(), c.data_ptr(), w.M, w.N, w.K,
+                                       w.K, w.N, w.N, h)
+    elif variant == "relu":  # an explicitly chosen kernel
+        fn, args = lib.gemm_f16_ex, (a.data_ptr(), b.data_ptr(), c.data_ptr(), w.M, w.N, w.K,
+                                     w.K, w.N, w.N, 1, path, h)
+    elif variant == "bias_gelu":
+        g = torch.Generator(device="cpu")
+        g.manual_seed(w.seed + 100)
+        bias = (torch.randn(w.N, generator=g) * 0.5).half().cuda()
+        fn, args = lib.gemm_bias_act_f16, (a.data_ptr(), b.data_ptr(), bias.data_ptr(),
+                                           c.data_ptr(), w.M, w.N, w.K, w.K, w.N, w.N,
+                                           ops.ACT_GELU, ops.PATH_AUTO, h)
+    elif variant == "wT":
+        b = b.t().contiguous()  # stored N x K
+        fn, args = lib.gemm_f16_general, (a.data_ptr(), b.data_ptr(), None, c.data_ptr(), w.M,
+                                          w.N, w.K, w.K, w.K, w.N, 0, 1, ops.ACT_RELU,
+                                          ops.PATH_AUTO, h)
+    else:
+        raise ValueError(variant)
 
     def step():
-        rc = lib.gemm_relu_f16(*args)
+        rc = fn(*args)
         if rc != 0:
-            raise RuntimeError(f"gemm_relu_f16 failed: {ops.status_string(rc)}")
+            raise RuntimeError(f"{variant} call failed: {ops.status_string(rc)}")
 
     total_ms, launch_ms = time_launches(step, steps, warmup, stream, dist, sampler)
     st = ops.device_status()
@@ -264,8 +287,15 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
     if comparator:
         # context only, never on the measured path: cuBLAS through torch on
         # the same inputs, timed the same way right after our kernel
-        def torch_step():
-            torch.relu_(torch.matmul(a, b, out=c))
+        if variant == "bias_gelu":
+            def torch_step():
+                torch.nn.functional.gelu(torch.addmm(bias, a, b, out=c))
+        elif variant == "wT":
+            def torch_step():
+                torch.relu_(torch.matmul(a, b.t(), out=c))
+        else:
+            def torch_step():
+                torch.relu_(torch.matmul(a, b, out=c))
         t_total, _ = time_launches(torch_step, steps, warmup, stream, None, None,
                                    per_launch=False)
         t_ms = t_total / steps
@@ -298,7 +328,8 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
 def kernel_for(w) -> str:
     from tiled_tensor_core_05_b200 import ops
     return {ops.PATH_SKINNY: "skinny_gemm_kernel", ops.PATH_TILE: "tile_gemm_kernel",
-            ops.PATH_TILE_PAIR: "tile_pair_gemm_kernel"}[ops.select_path(w.M, w.N, w.K)]
+            ops.PATH_TILE_PAIR: "tile_pair_gemm_kernel",
+            ops.PATH_TILE_PAIR_TALL: "tile_pair_gemm_kernel"}[ops.select_path(w.M, w.N, w.K)]
 
 
 def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool):
@@ -416,7 +447,8 @@ def run_ours(args):
     sampler = ClockSampler(gpu_id_for(local))
     sampler.wait_first()
     main = measure_workload(args.workload, args.steps, args.warmup, dist, sampler,
-                            e2e=not args.no_e2e, comparator=not args.no_comparator)
+                            e2e=not args.no_e2e, comparator=not args.no_comparator,
+                            path=args.path)
     sampler.stop()
     clocks = sampler.summary()
     w = main["w"]
@@ -455,13 +487,14 @@ def run_ours(args):
             "gbs": round(w.bytes_min / (t_ms * 1e-3) / 1e9, 1) if unit == "GB/s" else None}
     if rank == 0 and not args.no_secondary:
         others = []
-        for name in ("mlp_up", "decode", "cube1024", "cube256"):
-            if name == args.workload:
+        for name, variant in (("mlp_up", "relu"), ("decode", "relu"), ("cube1024", "relu"),
+                              ("cube256", "relu"), ("mlp_up", "bias_gelu"), ("decode", "wT")):
+            if name == args.workload and variant == "relu":
                 continue
             r = measure_workload(name, max(args.steps, 20), max(args.warmup, 3), None, None,
-                                 e2e=False, comparator=not args.no_comparator)
+                                 e2e=False, comparator=not args.no_comparator, variant=variant)
             ow = r["w"]
-            entry = {"workload": name, "M": ow.M, "N": ow.N, "K": ow.K,
+            entry = {"workload": name, "variant": variant, "M": ow.M, "N": ow.N, "K": ow.K,
                      "ms_per_launch": round(r["launch_ms"], 5),
                      "tflops": round(ow.flops / (r["launch_ms"] * 1e-3) / 1e12, 2),
                      "roofline": roofline_entry(name, r["launch_ms"], peaks, peak_src, False)}
@@ -496,6 +529,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", type=int, default=0,
+                    help="kernel for the main workload: 0 = chosen by shape (gemm_relu_f16), "
+                         "1 tile, 2 small-M, 3 CTA pair, 4 CTA pair with 512-row tiles")
     ap.add_argument("--no-comparator", action="store_true",
                     help="skip timing torch.matmul + relu as a context comparator")
     ap.add_argument("--cpu-budget", type=float, default=10.0,

@@ -67,13 +67,16 @@ enum gemm_status {
 };
 
 enum gemm_path {
-  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY; at least 64 tiles of
-                              256 x 256 -> TILE_PAIR; otherwise TILE */
+  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY; fewer than 64 tiles of
+                              256 x 256 -> TILE; otherwise TILE_PAIR_TALL, or TILE_PAIR
+                              when the 512-row tiles leave a much emptier last wave */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile (any shape) */
   GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 256 columns of B per CTA streamed
                               in lock-step, split-K only when tiles < SMs (M <= 64 only) */
-  GEMM_PATH_TILE_PAIR = 3  /* persistent kernel, two SMs (a CTA pair) per 256 x 256 tile
+  GEMM_PATH_TILE_PAIR = 3, /* persistent kernel, two SMs (a CTA pair) per 256 x 256 tile
                               (any shape) */
+  GEMM_PATH_TILE_PAIR_TALL = 4 /* persistent kernel, a CTA pair per 512 x 256 tile: fewer
+                                  bytes staged per MAC, epilogue not overlapped */
 };
 
 enum gemm_activation {
@@ -128,8 +131,8 @@ GEMM_API int gemm_f16_general(const void* A, const void* B, const void* bias, vo
                               int64_t ldc, int trans_a, int trans_b, int activation, int path,
                               gemm_stream_t stream);
 
-/* The path GEMM_PATH_AUTO takes for this shape (GEMM_PATH_TILE,
- * GEMM_PATH_TILE_PAIR or GEMM_PATH_SKINNY).  Pure host function. */
+/* The path GEMM_PATH_AUTO takes for this shape on a 148-SM B200 (pure host
+ * function; GEMM_PATH_AUTO itself uses the SM count of the current device). */
 GEMM_API int gemm_select_path(int64_t M, int64_t N, int64_t K);
 
 /* Human-readable text for a gemm_status value (static storage). */

@@ -19,7 +19,7 @@ from tiled_tensor_core_05_b200 import ops, workloads
 
 pytestmark = pytest.mark.gpu
 
-TILE, SKINNY, PAIR = ops.PATH_TILE, ops.PATH_SKINNY, ops.PATH_TILE_PAIR
+TILE, SKINNY, PAIR, TALL = ops.PATH_TILE, ops.PATH_SKINNY, ops.PATH_TILE_PAIR, ops.PATH_TILE_PAIR_TALL
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -54,7 +54,8 @@ def run(a_cpu, b_cpu, relu=True, path=ops.PATH_AUTO, lda=None, ldb=None, ldc=Non
 
 @pytest.mark.parametrize("name", ["cube256", "cube1024", "ragged1000"])
 @pytest.mark.parametrize("relu", [True, False])
-@pytest.mark.parametrize("path", [ops.PATH_AUTO, TILE, PAIR], ids=["auto", "tile", "pair"])
+@pytest.mark.parametrize("path", [ops.PATH_AUTO, TILE, PAIR, TALL],
+                         ids=["auto", "tile", "pair", "tall"])
 def test_workload_full(oracle_mod, name, relu, path):
     a, b = workloads.workload_inputs(name)
     ref = oracle_mod.gemm_relu(a, b) if relu else oracle_mod.gemm(a, b)
@@ -80,7 +81,7 @@ GRID = [(m, n, k) for m in EDGE for n in EDGE for k in EDGE
 
 
 @pytest.mark.parametrize("m,n,k", GRID)
-@pytest.mark.parametrize("path", [TILE, PAIR], ids=["tile", "pair"])
+@pytest.mark.parametrize("path", [TILE, PAIR, TALL], ids=["tile", "pair", "tall"])
 def test_ragged_grid_tile(oracle_mod, m, n, k, path):
     a, b = workloads.make_inputs(m, n, k, seed=1000 + m + 7 * n + 13 * k)
     ref = oracle_mod.gemm_relu(a, b)
@@ -90,11 +91,12 @@ def test_ragged_grid_tile(oracle_mod, m, n, k, path):
 @pytest.mark.parametrize("m,n,k", [(600, 1100, 700), (513, 257, 1030), (2048, 2048, 512),
                                    (4000, 300, 96)])
 def test_pair_kernel_multi_tile(oracle_mod, m, n, k):
-    """Several 256 x 256 pair tiles per CTA pair, ragged in every dimension."""
+    """Several pair tiles per CTA pair, ragged in every dimension."""
     a, b = workloads.make_inputs(m, n, k, seed=3000 + m + n + k)
     for relu in (True, False):
         ref = oracle_mod.gemm_relu(a, b) if relu else oracle_mod.gemm(a, b)
-        check_parity(run(a, b, relu=relu, path=PAIR), ref, relu, f"pair {m}x{n}x{k}")
+        for path in (PAIR, TALL):
+            check_parity(run(a, b, relu=relu, path=path), ref, relu, f"{path} {m}x{n}x{k}")
 
 
 @pytest.mark.parametrize("m,n,k", [(m, n, k) for (m, n, k) in GRID if m <= 64] +
@@ -107,7 +109,7 @@ def test_ragged_grid_skinny(oracle_mod, m, n, k):
         check_parity(run(a, b, relu=relu, path=SKINNY), ref, relu, f"small-M {m}x{n}x{k}")
 
 
-@pytest.mark.parametrize("path", [TILE, SKINNY, PAIR])
+@pytest.mark.parametrize("path", [TILE, SKINNY, PAIR, TALL])
 def test_padded_leading_dimensions(oracle_mod, path):
     m, n, k = 45, 300, 190
     a, b = workloads.make_inputs(m, n, k, seed=5)
@@ -131,7 +133,8 @@ def gpu_fn_for(path):
 
 
 @pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
-@pytest.mark.parametrize("path", [TILE, SKINNY, PAIR], ids=["tile", "skinny", "pair"])
+@pytest.mark.parametrize("path", [TILE, SKINNY, PAIR, TALL],
+                         ids=["tile", "skinny", "pair", "tall"])
 def test_pins_on_gpu(pin, path):
     fails = pin(gpu_fn_for(path), exact=False)
     assert not fails, "\n".join(fails[:5])
@@ -181,7 +184,7 @@ def test_workload_fullsize_sampled(oracle_mod, name):
 
 # ------------------------------------------------------------ special cases ---
 
-@pytest.mark.parametrize("path", [ops.PATH_AUTO, TILE, PAIR])
+@pytest.mark.parametrize("path", [ops.PATH_AUTO, TILE, PAIR, TALL])
 def test_k_zero_writes_zeros(path):
     a = torch.empty((5, 0), dtype=torch.float16, device="cuda")
     b = torch.empty((0, 9), dtype=torch.float16, device="cuda")
@@ -202,7 +205,7 @@ def test_empty_output_is_noop():
 def test_deterministic_bits_both_paths():
     a, b = workloads.make_inputs(64, 3000, 2500, seed=9)
     ad, bd = to_dev(a, round8(2500)), to_dev(b)
-    for path in (TILE, SKINNY, PAIR):
+    for path in (TILE, SKINNY, PAIR, TALL):
         outs = []
         for _ in range(3):
             outs.append(ops.gemm_f16_ex(ad, bd, relu=True, path=path).view(torch.int16).cpu())

@@ -11,7 +11,8 @@ from tiled_tensor_core_05_b200 import ops, workloads
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"tile": ops.PATH_TILE, "pair": ops.PATH_TILE_PAIR, "skinny": ops.PATH_SKINNY}
+PATHS = {"tile": ops.PATH_TILE, "pair": ops.PATH_TILE_PAIR, "tall": ops.PATH_TILE_PAIR_TALL,
+         "skinny": ops.PATH_SKINNY}
 LAYOUTS = [(False, False), (True, False), (False, True), (True, True)]
 
 

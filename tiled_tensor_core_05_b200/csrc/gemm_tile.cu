@@ -54,20 +54,30 @@ struct TileCfg {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-// The CTA-pair kernel: a 256 x 256 output tile per pair of SMs.  Each CTA
-// stages its own 128 rows of A and its own 128 columns of B per k-block, and
-// keeps its 128 accumulator rows x 256 columns in its TMEM.
-template <int STAGES>
+// The CTA-pair kernel: a (256 * SLABS) x 256 output tile per pair of SMs.
+// Each CTA stages SLABS slabs of 128 rows of A and its own 128 columns of B
+// per k-block; slab s of CTA r holds tile rows 256 s + 128 r .. + 127, and one
+// pair MMA (M = 256) per slab and 16-deep k step covers tile rows
+// 256 s .. 256 s + 255.  Each CTA keeps SLABS accumulators of 128 rows x 256
+// columns in TMEM: two buffers of one slab (the epilogue of tile i overlaps
+// the main loop of tile i+1), or the two slabs of one tile (25 % fewer bytes
+// staged per MAC, the epilogue not overlapped).
+template <int STAGES, int SLABS>
 struct PairCfg {
-  static constexpr int kBN = 256;                 // pair tile columns
-  static constexpr int kABytes = kBM * kBK * 2;   // this CTA's 128 rows
+  static constexpr int kBN = 256;                         // pair tile columns
+  static constexpr int kTileM = 2 * kBM * SLABS;          // pair tile rows
+  static constexpr int kSlabBytes = kBM * kBK * 2;        // 128 rows of A, 64 k
+  static constexpr int kABytes = SLABS * kSlabBytes;
   static constexpr int kBChunk = kBK * 64 * 2;
-  static constexpr int kBBytes = kBK * 128 * 2;   // this CTA's 128 columns
+  static constexpr int kBBytes = kBK * 128 * 2;           // this CTA's 128 columns
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiBuf;
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
-  static constexpr uint32_t kTmemCols = 512;      // two 256-column accumulators
+  static constexpr int kNBuf = SLABS == 1 ? 2 : 1;        // accumulator buffers
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(SLABS == 1 || SLABS == 2, "SLABS");
+  static_assert(kNBuf * SLABS * kBN == 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -395,17 +405,18 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 //     that an accumulator is ready (multicast arrive);
 //   * each CTA's four epilogue warps drain its own TMEM rows and arrive on the
 //     leader's acc_empty barrier (8 arrivals per accumulator use).
-template <int STAGES, int ACT>
+template <int STAGES, int SLABS, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
                           int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
                           int layout, int group_m, int* status, uint64_t timeout_ns) {
-  using Cfg = PairCfg<STAGES>;
+  using Cfg = PairCfg<STAGES, SLABS>;
   const bool ta = (layout & kLayoutTransA) != 0;
   const bool tb = (layout & kLayoutTransB) != 0;
   constexpr int BN = Cfg::kBN;
+  constexpr int NBUF = Cfg::kNBuf;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* smA = smem;
@@ -426,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = (rank == 0);
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(num_clusters_x());
-  const int num_m = (M + 2 * kBM - 1) / (2 * kBM);
+  const int num_m = (M + Cfg::kTileM - 1) / Cfg::kTileM;
   const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + kBK - 1) / kBK;
@@ -473,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
         int mb, nb;
         tile_coords(tile, num_m, num_n, group_m, mb, nb);
-        const int a_row = mb * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int a_row = mb * Cfg::kTileM + static_cast<int>(rank) * kBM;  // slab 0
         const int b_col = nb * BN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
@@ -482,12 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
           const uint32_t bar = full_leader + stage * 8;
-          uint8_t* adst = smA + stage * Cfg::kABytes;
-          if (!ta) {
-            tma_load_2d_pair(&tmA, bar, adst, kb * kBK, a_row);
-          } else {
-            tma_load_2d_pair(&tmA, bar, adst, a_row, kb * kBK);
-            tma_load_2d_pair(&tmA, bar, adst + Cfg::kBChunk, a_row + 64, kb * kBK);
+#pragma unroll
+          for (int s = 0; s < SLABS; ++s) {
+            uint8_t* adst = smA + stage * Cfg::kABytes + s * Cfg::kSlabBytes;
+            const int row = a_row + s * 2 * kBM;
+            if (!ta) {
+              tma_load_2d_pair(&tmA, bar, adst, kb * kBK, row);
+            } else {
+              tma_load_2d_pair(&tmA, bar, adst, row, kb * kBK);
+              tma_load_2d_pair(&tmA, bar, adst + Cfg::kBChunk, row + 64, kb * kBK);
+            }
           }
           uint8_t* bdst = smB + stage * Cfg::kBBytes;
           if (!tb) {
@@ -534,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * SLABS * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
             ok = false;
@@ -546,9 +561,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = smem_u32(smB + stage * Cfg::kBBytes);
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
-            const uint64_t adesc = operand_desc(a_addr, k, ta, Cfg::kBChunk);
             const uint64_t bdesc = operand_desc(b_addr, k, !tb, Cfg::kBChunk);
-            umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int s = 0; s < SLABS; ++s) {
+              const uint64_t adesc =
+                  operand_desc(a_addr + s * Cfg::kSlabBytes, k, ta, Cfg::kBChunk);
+              umma_f16_pair(d_tmem + static_cast<uint32_t>(s * BN), adesc, bdesc, idesc,
+                            (kb | k) != 0 ? 1u : 0u);
+            }
           }
           umma_commit_pair(&empty[stage], 0x3);  // stage s free in both CTAs
           if (++stage == STAGES) {
@@ -558,8 +578,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         umma_commit_pair(&acc_full[acc], 0x3);  // both epilogues may read
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == NBUF) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       if (!ok) {
         raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleMma << 4) | site);
@@ -586,14 +608,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const int row0 = mb * 2 * kBM + static_cast<int>(rank) * kBM + q * kEpiRows;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
       const uint32_t release_bar = acc_empty_leader + acc * 8;
-      epilogue_tile<BN, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
-                             nb * BN, lane, [release_bar] { mbar_arrive_cluster(release_bar); });
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+#pragma unroll 1
+      for (int s = 0; s < SLABS; ++s) {
+        const int row0 =
+            mb * Cfg::kTileM + s * 2 * kBM + static_cast<int>(rank) * kBM + q * kEpiRows;
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>((acc * SLABS + s) * BN);
+        const bool last = (s == SLABS - 1);
+        // the accumulator buffer is handed back after its last slab is read
+        epilogue_tile<BN, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
+                               nb * BN, lane, [release_bar, last] {
+                                 if (last) mbar_arrive_cluster(release_bar);
+                               });
+      }
+      if (++acc == NBUF) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
     if (lane == 0) bulk_wait_group<0>();
     __syncwarp();
@@ -683,9 +715,9 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
-template <int STAGES, int ACT>
+template <int STAGES, int SLABS, int ACT>
 int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
-  using Cfg = PairCfg<STAGES>;
+  using Cfg = PairCfg<STAGES, SLABS>;
   static std::atomic<uint64_t> attr_done{0};
   static int max_pairs[64] = {};
   CUtensorMap tA, tB, tC;
@@ -693,7 +725,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   const uint64_t n8 = static_cast<uint64_t>(p.N) & ~7ull;
   if (rc == 0) rc = encode_tmap_f16_2d(&tC, p.C, n8 > 0 ? n8 : 8, p.M, p.ldc, kEpiCols, kEpiRows);
   if (rc != 0) return rc;
-  auto kern = tile_pair_gemm_kernel<STAGES, ACT>;
+  auto kern = tile_pair_gemm_kernel<STAGES, SLABS, ACT>;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
                         attr_done))
     return GEMM_ERR_LAUNCH;
@@ -719,14 +751,14 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
     }
     resident = n;
   }
-  const int64_t num_tiles = ((p.M + 2 * kBM - 1) / (2 * kBM)) * ((p.N + 255) / 256);
+  const int64_t num_tiles = ((p.M + Cfg::kTileM - 1) / Cfg::kTileM) * ((p.N + 255) / 256);
   const int pairs = static_cast<int>(num_tiles < resident ? num_tiles : resident);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.numAttrs = 1 + pdl_attribute(&attr[1]);
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
-      static_cast<int>(p.K), p.layout, group_tiles(2 * kBM), d.status, d.timeout_ns);
+      static_cast<int>(p.K), p.layout, group_tiles(Cfg::kTileM), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
@@ -747,11 +779,18 @@ int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d) {
   }
 }
 
-int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d) {
+int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d, int slabs) {
+  if (slabs == 2) {
+    switch (p.act) {
+      case kActRelu: return launch_pair_impl<4, 2, kActRelu>(p, d);
+      case kActGelu: return launch_pair_impl<4, 2, kActGelu>(p, d);
+      default: return launch_pair_impl<4, 2, kActNone>(p, d);
+    }
+  }
   switch (p.act) {
-    case kActRelu: return launch_pair_impl<6, kActRelu>(p, d);
-    case kActGelu: return launch_pair_impl<6, kActGelu>(p, d);
-    default: return launch_pair_impl<6, kActNone>(p, d);
+    case kActRelu: return launch_pair_impl<6, 1, kActRelu>(p, d);
+    case kActGelu: return launch_pair_impl<6, 1, kActGelu>(p, d);
+    default: return launch_pair_impl<6, 1, kActNone>(p, d);
   }
 }
 

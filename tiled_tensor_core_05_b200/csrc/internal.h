@@ -45,8 +45,9 @@ int encode_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
 // Large-shape path: persistent warp-specialised tcgen05 kernel, one SM per
 // 128-row tile ...
 int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d);
-// ... or a pair of SMs per 256 x 256 tile (tcgen05.mma.cta_group::2).
-int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d);
+// ... or a pair of SMs per (256 * slabs) x 256 tile (tcgen05.mma.cta_group::2),
+// slabs = 1 or 2.
+int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d, int slabs);
 
 // Small-M path: swap-AB, lock-step split-K kernel.  `workspace` holds
 // per-tile arrival counters and split-K partial tiles (counters must be zero

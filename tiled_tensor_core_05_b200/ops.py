@@ -19,7 +19,7 @@ import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libttc05.so")
 
-PATH_AUTO, PATH_TILE, PATH_SKINNY, PATH_TILE_PAIR = 0, 1, 2, 3
+PATH_AUTO, PATH_TILE, PATH_SKINNY, PATH_TILE_PAIR, PATH_TILE_PAIR_TALL = 0, 1, 2, 3, 4
 ACT_NONE, ACT_RELU, ACT_GELU = 0, 1, 2
 _ACTS = {"none": ACT_NONE, "relu": ACT_RELU, "gelu": ACT_GELU}
 
