@@ -265,12 +265,13 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
         bias = (torch.randn(w.N, generator=g) * 0.5).half().cuda()
         fn, args = lib.gemm_bias_act_f16, (a.data_ptr(), b.data_ptr(), bias.data_ptr(),
                                            c.data_ptr(), w.M, w.N, w.K, w.K, w.N, w.N,
-                                           ops.ACT_GELU, ops.PATH_AUTO, h)
+                                           ops.ACT_GELU, path, h)
     elif variant == "wT":
         b = b.t().contiguous()  # stored N x K
+        b_cpu = b_cpu.t().contiguous()
         fn, args = lib.gemm_f16_general, (a.data_ptr(), b.data_ptr(), None, c.data_ptr(), w.M,
                                           w.N, w.K, w.K, w.K, w.N, 0, 1, ops.ACT_RELU,
-                                          ops.PATH_AUTO, h)
+                                          path, h)
     else:
         raise ValueError(variant)
 
@@ -448,7 +449,7 @@ def run_ours(args):
     sampler.wait_first()
     main = measure_workload(args.workload, args.steps, args.warmup, dist, sampler,
                             e2e=not args.no_e2e, comparator=not args.no_comparator,
-                            path=args.path)
+                            path=args.path, variant=args.variant)
     sampler.stop()
     clocks = sampler.summary()
     w = main["w"]
@@ -532,6 +533,8 @@ def main(argv=None):
     ap.add_argument("--path", type=int, default=0,
                     help="kernel for the main workload: 0 = chosen by shape (gemm_relu_f16), "
                          "1 tile, 2 small-M, 3 CTA pair, 4 CTA pair with 512-row tiles")
+    ap.add_argument("--variant", default="relu", choices=["relu", "bias_gelu", "wT"],
+                    help="operation of the main workload (default: the fused ReLU GEMM)")
     ap.add_argument("--no-comparator", action="store_true",
                     help="skip timing torch.matmul + relu as a context comparator")
     ap.add_argument("--cpu-budget", type=float, default=10.0,

@@ -131,8 +131,10 @@ GEMM_API int gemm_f16_general(const void* A, const void* B, const void* bias, vo
                               int64_t ldc, int trans_a, int trans_b, int activation, int path,
                               gemm_stream_t stream);
 
-/* The path GEMM_PATH_AUTO takes for this shape on a 148-SM B200 (pure host
- * function; GEMM_PATH_AUTO itself uses the SM count of the current device). */
+/* The path GEMM_PATH_AUTO takes for this shape with ReLU (or no activation) on
+ * a 148-SM B200 (pure host function; GEMM_PATH_AUTO itself uses the SM count
+ * of the current device, and takes GEMM_PATH_TILE_PAIR rather than
+ * GEMM_PATH_TILE_PAIR_TALL for GELU, whose epilogue it then overlaps). */
 GEMM_API int gemm_select_path(int64_t M, int64_t N, int64_t K);
 
 /* Human-readable text for a gemm_status value (static storage). */
@@ -186,6 +188,13 @@ GEMM_API int gemm_selftest_wait_timeout(int64_t timeout_ns, gemm_stream_t stream
 GEMM_API int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_t M, int64_t N,
                                    int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
                                    gemm_stream_t stream);
+
+/* y[i] = act(x[i]) for n fp32 values in device memory, with the exact code
+ * the GEMM epilogues use (GELU: x * Phi(x), Phi from Abramowitz & Stegun
+ * 7.1.26, |Phi error| <= 1e-6).  For checking the activations on their own.
+ * Asynchronous on `stream`. */
+GEMM_API int gemm_activation_f32(const void* x, void* y, int64_t n, int activation,
+                                 gemm_stream_t stream);
 
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
 GEMM_API int gemm_abi_version(void);

@@ -119,3 +119,22 @@ def test_bias_must_be_aligned():
     bias = torch.zeros(17, dtype=torch.float16, device="cuda")[1:]
     with pytest.raises(RuntimeError, match="aligned"):
         ops.gemm_bias_act_f16(a, b, bias, "gelu")
+
+
+def test_gelu_activation_accuracy():
+    """The epilogue's GELU (Phi from Abramowitz & Stegun 7.1.26) against fp64
+    and against CUDA's erfc-based GELU in fp32: |Phi error| within 1e-6."""
+    x64 = torch.linspace(-12, 12, 200001, dtype=torch.float64)
+    x = x64.float().cuda()
+    y = ops.activation_f32(x, "gelu").double().cpu()
+    xf = x.double().cpu()
+    ref = xf * 0.5 * torch.special.erfc(-xf / np.sqrt(2.0))
+    err = (y - ref).abs()
+    assert float((err / xf.abs().clamp(min=1.0)).max()) < 1e-6
+    cuda_ref = torch.nn.functional.gelu(x, approximate="none").double().cpu()
+    assert float((y - cuda_ref).abs().max()) < 2e-6 * 12
+    zero = ops.activation_f32(torch.zeros(4).cuda(), "gelu").cpu()
+    assert (zero == 0).all()
+    relu = ops.activation_f32(torch.tensor([-1.0, -0.0, 0.0, 2.5, float("nan")]).cuda(), "relu")
+    assert relu.cpu().tolist()[:4] == [0.0, 0.0, 0.0, 2.5] and relu.cpu()[4].item() == 0.0
+    assert not torch.signbit(relu.cpu()[1])

@@ -42,6 +42,8 @@ _SIGNATURES = {
     "gemm_selftest_wait_timeout": ([ctypes.c_int64, ctypes.c_void_p,
                                     ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
     "gemm_abi_version": ([], ctypes.c_int),
+    "gemm_activation_f32": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                             ctypes.c_void_p], ctypes.c_int),
     "gemm_relu_f16_noalloc": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
                               ctypes.c_int),
 }
@@ -185,6 +187,19 @@ def gemm_relu_f16(a, b, out=None, *, stream=None):
 def gemm_f16(a, b, out=None, *, stream=None):
     """C = A @ B; see :func:`gemm_f16_ex`."""
     return gemm_f16_ex(a, b, out, relu=False, stream=stream)
+
+
+def activation_f32(x: torch.Tensor, act: str | int = "gelu", stream=None) -> torch.Tensor:
+    """The epilogue activation applied elementwise to a CUDA fp32 tensor."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        _check(lib().gemm_activation_f32(x.data_ptr(), y.data_ptr(), x.numel(), code,
+                                         _stream_handle(stream, x.device)),
+               "gemm_activation_f32")
+    return y
 
 
 def select_path(M: int, N: int, K: int) -> int:
