@@ -86,8 +86,7 @@ __device__ __forceinline__ void load_accumulator(uint32_t taddr, float (&v)[MP])
 #pragma unroll
   for (int j = 0; j < MP / 32; ++j) {
     uint32_t r[32];
-    tmem_ld_32x32b_x32(taddr + j * 32, r);
-    tmem_wait_ld();
+    tmem_load_32x32b_x32(taddr + j * 32, r);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[j * 32 + i] = __uint_as_float(r[i]);
   }

@@ -125,10 +125,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
         }
       }
     }
-    uint32_t v0[32], v1[32];
-    tmem_ld_32x32b_x32(t_row + c * kEpiCols, v0);
-    tmem_ld_32x32b_x32(t_row + c * kEpiCols + 32, v1);
-    tmem_wait_ld();
+    uint32_t v[64];
+    tmem_load_32x32b_x64(t_row + c * kEpiCols, v);
     if (c == BN / kEpiCols - 1) {
       // the accumulator has been read: hand it back to the MMA issuer
       tc_fence_before_sync();
@@ -138,8 +136,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
     uint32_t h[32];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      float x0 = __uint_as_float(v0[2 * i]), x1 = __uint_as_float(v0[2 * i + 1]);
-      float y0 = __uint_as_float(v1[2 * i]), y1 = __uint_as_float(v1[2 * i + 1]);
+      float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
+      float y0 = __uint_as_float(v[32 + 2 * i]), y1 = __uint_as_float(v[32 + 2 * i + 1]);
       if (bias != nullptr) {
         const float2 bx = __half22float2(*reinterpret_cast<const __half2*>(&bb[i]));
         const float2 by = __half22float2(*reinterpret_cast<const __half2*>(&bb[16 + i]));
