@@ -24,14 +24,14 @@ import datetime
 import hashlib
 import json
 import os
-import statistics
 import sys
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+
+from tiled_tensor_core_05_b200.clocks import ClockSampler, gpu_id_for  # noqa: E402
 
 METRIC = "fused GEMM+ReLU TFLOP/s and % of B200 dense fp16 peak (GB/s % HBM for skinny)"
 NOMINAL_FP16_TFLOPS = 2250.0
@@ -86,89 +86,6 @@ def traffic_for(workload: str, kernel: str):
     if not e or e.get("kernel_src_sha") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
-
-
-class ClockSampler:
-    """SM clock, power and clock-event reasons polled through NVML (read-only
-    queries) every ~1 ms from a background thread while the GPU works."""
-
-    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
-               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
-               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
-               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
-               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
-
-    def __init__(self, gpu_uuid: str, interval_s: float = 0.001):
-        self.samples = []
-        self.marks = {}
-        self.ok = False
-        self._stop = threading.Event()
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-            self.bits = [(name, getattr(pynvml, attr)) for name, attr in self.REASONS]
-            self.ok = True
-        except Exception as e:  # no NVML: report that instead of clocks
-            self.err = repr(e)
-            return
-        self.interval = interval_s
-        self.thread = threading.Thread(target=self._run, daemon=True)
-        self.thread.start()
-
-    def _run(self):
-        nv, h = self.nv, self.h
-        while not self._stop.is_set():
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                self.samples.append((time.monotonic(), sm, rs, pw))
-            except Exception:
-                pass
-            time.sleep(self.interval)
-
-    def wait_first(self, timeout=5.0):
-        t0 = time.monotonic()
-        while self.ok and not self.samples and time.monotonic() - t0 < timeout:
-            time.sleep(0.005)
-
-    def mark(self, name):
-        self.marks[name] = time.monotonic()
-
-    def stop(self):
-        self._stop.set()
-        if self.ok:
-            self.thread.join(timeout=2)
-
-    def summary(self, start="t0", end="t1"):
-        if not self.ok:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
-                    "note": "NVML unavailable: " + getattr(self, "err", "")}
-        t0, t1 = self.marks.get(start, 0.0), self.marks.get(end, 1e30)
-        inside = [s for s in self.samples if t0 <= s[0] <= t1]
-        note = "NVML samples taken during the timed region"
-        if len(inside) < 3:
-            w0 = self.marks.get("warm0", t0)
-            inside = [s for s in self.samples if w0 <= s[0] <= t1]
-            note = "timed region too short for 3 samples; warm-up + timed samples"
-        if not inside:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
-                    "note": "no sample during the busy period"}
-        reasons = sorted({name for s in inside for name, bit in self.bits if s[2] & bit})
-        return {"sm_mhz": statistics.median(s[1] for s in inside),
-                "sm_mhz_min": min(s[1] for s in inside),
-                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
-                "power_w_max": round(max(s[3] for s in inside), 1), "note": note}
-
-
-def gpu_id_for(dev_index: int) -> str:
-    """NVML UUID string ("GPU-...") of a torch device index."""
-    import torch
-    s = str(torch.cuda.get_device_properties(dev_index).uuid)
-    return s if s.startswith("GPU-") else "GPU-" + s
 
 
 def max_over_ranks(value: float, dist=None) -> float:
@@ -354,16 +271,23 @@ def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool):
             "peak_source": f"{peak_src} {key} (cuBLAS bf16; fp16 has the same nominal rate)"}
 
 
+def oracle_seconds_per_row(oracle, a, b) -> float:
+    """Host time per row of C for the oracle, measured on a block of rows
+    large enough to occupy every thread it uses (it parallelises over rows)."""
+    oracle.gemm_relu(a[:1], b)  # thread pool and page faults out of the way
+    rows = min(int(a.shape[0]), 2 * oracle.max_threads())
+    t0 = time.perf_counter()
+    oracle.gemm_relu(a[:rows], b)
+    return max(time.perf_counter() - t0, 1e-6) / rows
+
+
 def cpu_baseline(name, budget_s=10.0):
     """The oracle timed on a bounded sample (leading rows) of the workload."""
     import oracle
     from tiled_tensor_core_05_b200 import workloads
     w = workloads.WORKLOADS[name]
     a, b = workloads.workload_inputs(name)
-    t0 = time.perf_counter()
-    oracle.gemm_relu(a[:1], b)
-    t_row = max(time.perf_counter() - t0, 1e-4)
-    rows = int(max(1, min(w.M, budget_s / t_row)))
+    rows = int(max(1, min(w.M, budget_s / oracle_seconds_per_row(oracle, a, b))))
     t0 = time.perf_counter()
     oracle.gemm_relu(a[:rows], b)
     dt = time.perf_counter() - t0
@@ -390,10 +314,7 @@ def run_reference(args):
     w = workloads.WORKLOADS[args.workload]
     a, b = workloads.workload_inputs(args.workload)
     # size one step to about a second of host work
-    t0 = time.perf_counter()
-    oracle.gemm_relu(a[:1], b)
-    t_row = max(time.perf_counter() - t0, 1e-4)
-    rows = int(max(1, min(w.M, 1.0 / t_row)))
+    rows = int(max(1, min(w.M, 1.0 / oracle_seconds_per_row(oracle, a, b))))
     for _ in range(args.warmup):
         oracle.gemm_relu(a[:rows], b)
     t0 = time.perf_counter()

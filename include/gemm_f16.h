@@ -63,7 +63,9 @@ enum gemm_status {
   GEMM_ERR_LAUNCH = -4,             /* a CUDA runtime call or kernel launch failed */
   GEMM_ERR_WORKSPACE = -5,          /* small-M workspace allocation failed */
   GEMM_ERR_DEVICE_TIMEOUT = -6,     /* reported by gemm_get_device_status */
-  GEMM_ERR_SCRATCH_LIMIT = -7       /* problem too large for gemm_relu_f16_noalloc's fixed scratch */
+  GEMM_ERR_SCRATCH_LIMIT = -7,      /* problem too large for gemm_relu_f16_noalloc's fixed scratch */
+  GEMM_ERR_CONFIG = -8              /* gemm_f16_config: configuration not built or not valid
+                                       for this problem */
 };
 
 enum gemm_path {
@@ -130,6 +132,55 @@ GEMM_API int gemm_f16_general(const void* A, const void* B, const void* bias, vo
                               int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
                               int64_t ldc, int trans_a, int trans_b, int activation, int path,
                               gemm_stream_t stream);
+
+/* One kernel configuration, for choosing configurations offline: the tuning
+ * workflow of "TileLang simplifica la creación de kernels GPU de alto
+ * rendimiento" (posicionamiento-web.ar) and "TileLang explicado: kernels de IA
+ * escritos por mosaicos" (easyairoute.com), sections on tuning tile sizes,
+ * pipeline stages and L2 ordering per GPU, done as a sweep outside the library
+ * (the library itself never times or chooses among these at run time).
+ * A field left at 0 takes the value GEMM_PATH_AUTO would use. */
+typedef struct gemm_config {
+  int32_t kernel;     /* GEMM_PATH_TILE, _TILE_PAIR, _TILE_PAIR_TALL or _SKINNY (not AUTO) */
+  int32_t block_n;    /* output columns per tile: 128 or 256 for GEMM_PATH_TILE; 256 (the
+                         only width) for the other kernels */
+  int32_t stages;     /* depth of the shared-memory operand ring (k-blocks of 64 in flight) */
+  int32_t group_rows; /* tile kernels: rows of op(A) per raster panel, the L2 grouping of
+                         the tile order; 0 = 2048.  Must be 0 for GEMM_PATH_SKINNY */
+  int32_t splits;     /* GEMM_PATH_SKINNY: k-slices per 256-column tile, 1 <= splits <=
+                         ceil(K / 64) and splits * ceil(N / 256) <= the SM count when > 1;
+                         0 = chosen from the shape.  Must be 0 for the tile kernels */
+} gemm_config;
+
+/* gemm_f16_general with the kernel configuration `cfg` instead of a path.
+ * Results are the same operation: every configuration meets the same
+ * accuracy, though fp32 sums in another order may differ in the last bits.
+ * Returns GEMM_ERR_CONFIG (and launches nothing) when `cfg` names no compiled
+ * kernel (see gemm_config_list) or does not fit the problem (GEMM_PATH_SKINNY
+ * with M > 64, a splits value out of range), GEMM_ERR_INVALID_ARG for a null
+ * `cfg`; otherwise as gemm_f16_general. */
+GEMM_API int gemm_f16_config(const void* A, const void* B, const void* bias, void* C, int64_t M,
+                             int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                             int trans_a, int trans_b, int activation, const gemm_config* cfg,
+                             gemm_stream_t stream);
+
+/* Dynamic shared memory per CTA (bytes) that the kernel, block_n and stages of
+ * `cfg` need, whether or not that configuration is compiled (stages 0 = the
+ * default).  A configuration fits a B200 when this is <= 232448.  Returns
+ * GEMM_ERR_CONFIG when kernel / block_n name no kernel.  Pure host function. */
+GEMM_API int gemm_config_smem_bytes(const gemm_config* cfg);
+
+/* The compiled configurations (kernel, block_n, stages; group_rows and
+ * splits 0, free at call time): every stage count from 3 up to the shared
+ * memory budget of each tile shape.  Writes up to `capacity` of them to `out`
+ * (may be null when capacity is 0) and returns how many there are.  Pure host
+ * function. */
+GEMM_API int gemm_config_list(gemm_config* out, int capacity);
+
+/* The configuration GEMM_PATH_AUTO takes for this problem on the current
+ * device (all fields resolved).  Returns GEMM_OK, or a negative gemm_status
+ * (invalid sizes or activation, no sm_100 device). */
+GEMM_API int gemm_auto_config(int64_t M, int64_t N, int64_t K, int activation, gemm_config* out);
 
 /* The path GEMM_PATH_AUTO takes for this shape with ReLU (or no activation) on
  * a 148-SM B200 (pure host function; GEMM_PATH_AUTO itself uses the SM count

@@ -46,7 +46,7 @@ def test_only_the_api_is_exported():
 
 def test_status_strings(lib):
     from tiled_tensor_core_05_b200 import ops
-    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
         s = ops.status_string(code)
         assert s and s != "unknown status", code
     assert ops.status_string(12345) == "unknown status"

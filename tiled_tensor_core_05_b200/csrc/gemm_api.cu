@@ -324,7 +324,7 @@ using namespace ttc;
 
 extern "C" {
 
-int gemm_abi_version(void) { return 10000; }
+int gemm_abi_version(void) { return 10100; }
 
 namespace ttc {
 namespace {
@@ -358,32 +358,55 @@ int select_path_for(int64_t M, int64_t N, int sm_count, int activation) {
              : GEMM_PATH_TILE_PAIR;
 }
 
-}  // namespace
-}  // namespace ttc
-
-int gemm_select_path(int64_t M, int64_t N, int64_t K) {
-  (void)K;
-  return select_path_for(M, N, 148, GEMM_ACT_RELU);  // a B200 has 148 SMs
-}
-
-const char* gemm_status_string(int status) {
-  switch (status) {
-    case GEMM_OK: return "ok";
-    case GEMM_ERR_INVALID_ARG: return "invalid argument (size, leading dimension or pointer)";
-    case GEMM_ERR_ALIGNMENT: return "pointer not 16-byte aligned or leading dimension not a multiple of 8";
-    case GEMM_ERR_UNSUPPORTED_DEVICE: return "current device is not an sm_100 (B200) GPU";
-    case GEMM_ERR_LAUNCH: return "CUDA runtime call or kernel launch failed";
-    case GEMM_ERR_WORKSPACE: return "small-M workspace allocation failed";
-    case GEMM_ERR_DEVICE_TIMEOUT: return "a device-side wait ran out of time";
-    case GEMM_ERR_SCRATCH_LIMIT:
-      return "problem too large for the fixed scratch of gemm_relu_f16_noalloc (needs M <= 32)";
-    default: return "unknown status";
+int default_stages(int kernel, int block_n) {
+  switch (kernel) {
+    case GEMM_PATH_TILE: return block_n == 256 ? kDefaultStagesTile256 : kDefaultStagesTile128;
+    case GEMM_PATH_TILE_PAIR: return kDefaultStagesPair;
+    case GEMM_PATH_TILE_PAIR_TALL: return kDefaultStagesTall;
+    case GEMM_PATH_SKINNY: return kDefaultStagesSkinny;
+    default: return 0;
   }
 }
 
-int gemm_f16_general(const void* A, const void* B, const void* bias, void* C, int64_t M,
-                     int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int trans_a,
-                     int trans_b, int activation, int path, gemm_stream_t stream) {
+// Fills the fields of `c` left at 0 with what GEMM_PATH_AUTO would use for an
+// M x N output and checks the rest (the stage count is checked against the
+// compiled kernels at launch).  Returns GEMM_OK or GEMM_ERR_CONFIG.
+int resolve_config(KernelConfig& c, int64_t M, int64_t N, int sm_count) {
+  if (c.stages < 0 || c.group_rows < 0 || c.splits < 0) return GEMM_ERR_CONFIG;
+  switch (c.kernel) {
+    case GEMM_PATH_TILE:
+      if (c.block_n == 0) {
+        // 128 x 256 tiles when there are enough of them to fill the GPU,
+        // otherwise 128 x 128 tiles (twice as many CTAs for small problems)
+        const int64_t tiles256 = ((M + 127) / 128) * ((N + 255) / 256);
+        c.block_n = tiles256 >= sm_count ? 256 : 128;
+      }
+      if (c.block_n != 128 && c.block_n != 256) return GEMM_ERR_CONFIG;
+      break;
+    case GEMM_PATH_TILE_PAIR:
+    case GEMM_PATH_TILE_PAIR_TALL:
+    case GEMM_PATH_SKINNY:
+      if (c.block_n == 0) c.block_n = 256;
+      if (c.block_n != 256) return GEMM_ERR_CONFIG;
+      break;
+    default:
+      return GEMM_ERR_CONFIG;
+  }
+  if (c.stages == 0) c.stages = default_stages(c.kernel, c.block_n);
+  if (c.kernel == GEMM_PATH_SKINNY) {
+    if (c.group_rows != 0 || skinny_m_pad(M) == 0) return GEMM_ERR_CONFIG;
+  } else {
+    if (c.splits != 0) return GEMM_ERR_CONFIG;
+    if (c.group_rows == 0) c.group_rows = kDefaultGroupRows;
+  }
+  return GEMM_OK;
+}
+
+// The entry points' common body: validation, then the kernel of `cfg`, or of
+// `path` when `cfg` is null.
+int run_gemm(const void* A, const void* B, const void* bias, void* C, int64_t M, int64_t N,
+             int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int trans_a, int trans_b,
+             int activation, int path, const gemm_config* cfg, gemm_stream_t stream) {
   if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
   if ((trans_a != 0 && trans_a != 1) || (trans_b != 0 && trans_b != 1))
     return GEMM_ERR_INVALID_ARG;
@@ -391,13 +414,24 @@ int gemm_f16_general(const void* A, const void* B, const void* bias, void* C, in
   if (activation != GEMM_ACT_NONE && activation != GEMM_ACT_RELU &&
       activation != GEMM_ACT_GELU)
     return GEMM_ERR_INVALID_ARG;
-  if (path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE && path != GEMM_PATH_SKINNY &&
-      path != GEMM_PATH_TILE_PAIR && path != GEMM_PATH_TILE_PAIR_TALL)
+  if (cfg == nullptr && path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE &&
+      path != GEMM_PATH_SKINNY && path != GEMM_PATH_TILE_PAIR &&
+      path != GEMM_PATH_TILE_PAIR_TALL)
     return GEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return GEMM_OK;
   DeviceCtx d;
   int rc = get_device(&d);
   if (rc != GEMM_OK) return rc;
+  KernelConfig kc{};
+  if (cfg != nullptr) {
+    kc = KernelConfig{cfg->kernel, cfg->block_n, cfg->stages, cfg->group_rows, cfg->splits};
+    rc = resolve_config(kc, M, N, d.sm_count);
+    if (rc != GEMM_OK) return rc;
+  } else {
+    if (path == GEMM_PATH_AUTO) path = select_path_for(M, N, d.sm_count, activation);
+    kc = KernelConfig{path, 0, 0, 0, 0};
+    if (resolve_config(kc, M, N, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
+  }
   load_entry_points();
   rc = check_matrix(C, M, N, ldc, d.device);
   if (rc != GEMM_OK) return rc;
@@ -417,18 +451,92 @@ int gemm_f16_general(const void* A, const void* B, const void* bias, void* C, in
   if (rc == GEMM_OK)
     rc = trans_b ? check_matrix(B, N, K, ldb, d.device) : check_matrix(B, K, N, ldb, d.device);
   if (rc != GEMM_OK) return rc;
-  if (path == GEMM_PATH_AUTO) path = select_path_for(M, N, d.sm_count, activation);
-  if (path == GEMM_PATH_SKINNY) {
-    if (skinny_m_pad(M) == 0) return GEMM_ERR_INVALID_ARG;
+  if (kc.kernel == GEMM_PATH_SKINNY) {
     void* ws = nullptr;
     size_t ws_bytes = 0;
     rc = get_workspace(d, stream, &ws, &ws_bytes);
     if (rc != GEMM_OK) return rc;
-    return launch_skinny_gemm(p, d, ws, ws_bytes);
+    return launch_skinny_gemm(p, d, ws, ws_bytes, kc);
   }
-  if (path == GEMM_PATH_TILE_PAIR) return launch_tile_pair_gemm(p, d, 1);
-  if (path == GEMM_PATH_TILE_PAIR_TALL) return launch_tile_pair_gemm(p, d, 2);
-  return launch_tile_gemm(p, d);
+  return launch_tile_gemm(p, d, kc);
+}
+
+}  // namespace
+}  // namespace ttc
+
+int gemm_select_path(int64_t M, int64_t N, int64_t K) {
+  (void)K;
+  return select_path_for(M, N, 148, GEMM_ACT_RELU);  // a B200 has 148 SMs
+}
+
+const char* gemm_status_string(int status) {
+  switch (status) {
+    case GEMM_OK: return "ok";
+    case GEMM_ERR_INVALID_ARG: return "invalid argument (size, leading dimension or pointer)";
+    case GEMM_ERR_ALIGNMENT: return "pointer not 16-byte aligned or leading dimension not a multiple of 8";
+    case GEMM_ERR_UNSUPPORTED_DEVICE: return "current device is not an sm_100 (B200) GPU";
+    case GEMM_ERR_LAUNCH: return "CUDA runtime call or kernel launch failed";
+    case GEMM_ERR_WORKSPACE: return "small-M workspace allocation failed";
+    case GEMM_ERR_DEVICE_TIMEOUT: return "a device-side wait ran out of time";
+    case GEMM_ERR_SCRATCH_LIMIT:
+      return "problem too large for the fixed scratch of gemm_relu_f16_noalloc (needs M <= 32)";
+    case GEMM_ERR_CONFIG:
+      return "kernel configuration not compiled, or not valid for this problem";
+    default: return "unknown status";
+  }
+}
+
+int gemm_f16_general(const void* A, const void* B, const void* bias, void* C, int64_t M,
+                     int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int trans_a,
+                     int trans_b, int activation, int path, gemm_stream_t stream) {
+  return run_gemm(A, B, bias, C, M, N, K, lda, ldb, ldc, trans_a, trans_b, activation, path,
+                  nullptr, stream);
+}
+
+int gemm_f16_config(const void* A, const void* B, const void* bias, void* C, int64_t M,
+                    int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int trans_a,
+                    int trans_b, int activation, const gemm_config* cfg, gemm_stream_t stream) {
+  if (cfg == nullptr) return GEMM_ERR_INVALID_ARG;
+  return run_gemm(A, B, bias, C, M, N, K, lda, ldb, ldc, trans_a, trans_b, activation,
+                  GEMM_PATH_AUTO, cfg, stream);
+}
+
+int gemm_config_smem_bytes(const gemm_config* cfg) {
+  if (cfg == nullptr) return GEMM_ERR_INVALID_ARG;
+  int block_n = cfg->block_n;
+  if (block_n == 0 && cfg->kernel != GEMM_PATH_TILE) block_n = 256;
+  const int stages = cfg->stages != 0 ? cfg->stages : default_stages(cfg->kernel, block_n);
+  int bytes = -1;
+  if (cfg->kernel == GEMM_PATH_SKINNY)
+    bytes = block_n == 256 ? skinny_config_smem_bytes(stages) : -1;
+  else
+    bytes = tile_config_smem_bytes(cfg->kernel, block_n, stages);
+  return bytes > 0 ? bytes : GEMM_ERR_CONFIG;
+}
+
+int gemm_config_list(gemm_config* out, int capacity) {
+  KernelConfig all[64];
+  int n = tile_configs_built(all, 64);
+  n += skinny_configs_built(all + n, 64 - n);
+  for (int i = 0; i < n && i < capacity && out != nullptr; ++i)
+    out[i] = gemm_config{all[i].kernel, all[i].block_n, all[i].stages, 0, 0};
+  return n;
+}
+
+int gemm_auto_config(int64_t M, int64_t N, int64_t K, int activation, gemm_config* out) {
+  if (out == nullptr || M < 1 || N < 1 || K < 0 || M > INT32_MAX || N > INT32_MAX ||
+      K > INT32_MAX)
+    return GEMM_ERR_INVALID_ARG;
+  if (activation != GEMM_ACT_NONE && activation != GEMM_ACT_RELU &&
+      activation != GEMM_ACT_GELU)
+    return GEMM_ERR_INVALID_ARG;
+  DeviceCtx d;
+  const int rc = get_device(&d);
+  if (rc != GEMM_OK) return rc;
+  KernelConfig c{select_path_for(M, N, d.sm_count, activation), 0, 0, 0, 0};
+  if (resolve_config(c, M, N, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
+  *out = gemm_config{c.kernel, c.block_n, c.stages, c.group_rows, c.splits};
+  return GEMM_OK;
 }
 
 int gemm_bias_act_f16(const void* A, const void* B, const void* bias, void* C, int64_t M,

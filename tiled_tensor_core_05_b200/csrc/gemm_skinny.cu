@@ -43,6 +43,14 @@ constexpr int kUmmaK = 16;
 constexpr int kThreads = 192;  // producer, MMA, 4 epilogue warps
 constexpr int kEpiWarps = 4;
 
+// Dynamic shared memory of the small-M kernel: 1 KiB of alignment slack, the
+// ring (256 columns of B and room for A^T per stage), the mbarriers (full
+// and empty per stage, accumulator-full, drain, one spare) and the TMEM
+// address slot.  A^T takes 8 KiB per stage for either MP.
+constexpr int skinny_smem_formula(int stages) {
+  return 1024 + stages * (4 * kBK * 64 * 2 + 8192) + (2 * stages + 3) * 8 + 16;
+}
+
 template <int MP, int STAGES>
 struct SkinnyCfg {
   static constexpr int kBChunk = kBK * 64 * 2;    // 64 columns x 64 k-rows = 8 KiB
@@ -57,8 +65,24 @@ struct SkinnyCfg {
   static constexpr uint32_t kTmemCols = (2 * MP < 32) ? 32 : 2 * MP;
   static_assert(MP == 32 || MP == 64, "MP");
   static_assert(kABytes % 1024 == 0, "A tile alignment");
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kSmemBytes == skinny_smem_formula(STAGES), "layout");
+  static_assert(kSmemBytes <= kMaxDynamicSmem, "shared memory budget");
 };
+
+// Ring depths compiled (for MP 32 and 64 and every activation): 3 up to what
+// fits the shared-memory budget.
+constexpr int kSkinnyStages[] = {3, 4, 5};
+constexpr int kNumSkinnyStages = sizeof(kSkinnyStages) / sizeof(kSkinnyStages[0]);
+
+constexpr bool skinny_variants_complete() {
+  for (int st = 3; st <= 16; ++st) {
+    bool built = false;
+    for (int v : kSkinnyStages) built = built || v == st;
+    if ((skinny_smem_formula(st) <= kMaxDynamicSmem) != built) return false;
+  }
+  return true;
+}
+static_assert(skinny_variants_complete(), "built skinny configurations != those within the budget");
 
 __device__ __forceinline__ float4 ld_cg_f4(const float* p) {
   return __ldcg(reinterpret_cast<const float4*>(p));
@@ -355,14 +379,18 @@ int choose_slices(int64_t tiles, int64_t KB, int sm_count, int64_t max_items) {
   return s < 1 ? 1 : static_cast<int>(s);
 }
 
+// `splits` = 0 chooses the k-slices from the shape; otherwise exactly that
+// many (1 <= splits <= k-blocks, and splits * tiles <= max_items when > 1).
 template <int MP, int STAGES, int ACT>
 int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
-                int64_t max_items) {
+                int64_t max_items, int splits) {
   using Cfg = SkinnyCfg<MP, STAGES>;
   static std::atomic<uint64_t> attr_done{0};
   const int64_t KB = (p.K + kBK - 1) / kBK;
   const int64_t tiles = (p.N + kTW - 1) / kTW;
-  const int S = choose_slices(tiles, KB, d.sm_count, max_items);
+  if (splits < 0 || splits > KB || (splits > 1 && splits * tiles > max_items))
+    return GEMM_ERR_CONFIG;
+  const int S = splits > 0 ? splits : choose_slices(tiles, KB, d.sm_count, max_items);
   int* counters = nullptr;
   float* partials = nullptr;
   if (S > 1) {
@@ -422,22 +450,48 @@ size_t skinny_workspace_bytes(int sm_count, int m_pad) {
          static_cast<size_t>(sm_count) * kTW * static_cast<size_t>(m_pad) * sizeof(float);
 }
 
-// 5 stages with L2 hints: measured best on the decode shape (72.7 us against
-// 75.2 us for 6 stages without hints, 73.5-75.0 us for 4 or 6 stages with).
-template <int MP>
-int launch_mp(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes) {
+namespace {
+
+template <int MP, int STAGES>
+int launch_act(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes, int splits) {
   switch (p.act) {
-    case kActRelu: return launch_impl<MP, 5, kActRelu>(p, d, ws, ws_bytes, d.sm_count);
-    case kActGelu: return launch_impl<MP, 5, kActGelu>(p, d, ws, ws_bytes, d.sm_count);
-    default: return launch_impl<MP, 5, kActNone>(p, d, ws, ws_bytes, d.sm_count);
+    case kActRelu: return launch_impl<MP, STAGES, kActRelu>(p, d, ws, ws_bytes, d.sm_count, splits);
+    case kActGelu: return launch_impl<MP, STAGES, kActGelu>(p, d, ws, ws_bytes, d.sm_count, splits);
+    default: return launch_impl<MP, STAGES, kActNone>(p, d, ws, ws_bytes, d.sm_count, splits);
   }
 }
 
-int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes) {
+template <int MP, int I = 0>
+int dispatch_stages(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
+                    const KernelConfig& c) {
+  if constexpr (I == kNumSkinnyStages) {
+    return GEMM_ERR_CONFIG;
+  } else {
+    if (c.stages == kSkinnyStages[I])
+      return launch_act<MP, kSkinnyStages[I]>(p, d, ws, ws_bytes, c.splits);
+    return dispatch_stages<MP, I + 1>(p, d, ws, ws_bytes, c);
+  }
+}
+
+}  // namespace
+
+int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
+                       const KernelConfig& c) {
   const int mp = skinny_m_pad(p.M);
-  if (mp == 32) return launch_mp<32>(p, d, ws, ws_bytes);
-  if (mp == 64) return launch_mp<64>(p, d, ws, ws_bytes);
+  if (mp == 32) return dispatch_stages<32>(p, d, ws, ws_bytes, c);
+  if (mp == 64) return dispatch_stages<64>(p, d, ws, ws_bytes, c);
   return GEMM_ERR_INVALID_ARG;
+}
+
+int skinny_config_smem_bytes(int stages) {
+  if (stages < 1 || stages > 64) return -1;
+  return skinny_smem_formula(stages);
+}
+
+int skinny_configs_built(KernelConfig* out, int cap) {
+  for (int i = 0; i < kNumSkinnyStages && i < cap; ++i)
+    out[i] = KernelConfig{GEMM_PATH_SKINNY, kTW, kSkinnyStages[i], 0, 0};
+  return kNumSkinnyStages;
 }
 
 // ------------------------------------------------ allocation-free variant ---
@@ -488,7 +542,8 @@ int launch_skinny_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d) {
   if (cudaMemsetAsync(scratch, 0, kNoAllocCounterBytes, p.stream) != cudaSuccess)
     return GEMM_ERR_LAUNCH;
   const int64_t items = d.sm_count < kNoAllocMaxItems ? d.sm_count : kNoAllocMaxItems;
-  return launch_impl<kNoAllocMP, 5, kActRelu>(p, d, scratch, kNoAllocScratchBytes, items);
+  return launch_impl<kNoAllocMP, kDefaultStagesSkinny, kActRelu>(p, d, scratch,
+                                                             kNoAllocScratchBytes, items, 0);
 }
 
 }  // namespace ttc

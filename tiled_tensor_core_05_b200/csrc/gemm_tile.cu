@@ -21,7 +21,6 @@
 // Out-of-range A/B elements (M, N or K not a multiple of the tile) are
 // zero-filled by TMA and so contribute nothing to the sum.
 #include <atomic>
-#include <cstdlib>
 
 #include "../../include/gemm_f16.h"
 #include "internal.h"
@@ -39,6 +38,18 @@ constexpr int kEpiRows = 32;    // rows per epilogue warp
 constexpr int kEpiCols = 64;    // columns per epilogue chunk (128 bytes of fp16)
 constexpr int kEpiBuf = kEpiRows * kEpiCols * 2;
 
+// Dynamic shared memory of a tile kernel: 1 KiB of alignment slack, the
+// operand ring, two 32 x 64 fp16 staging boxes per epilogue warp, the
+// mbarriers (full and empty per stage, two accumulator handshakes per
+// buffer, one spare) and the TMEM address slot.
+constexpr int tile_smem_formula(int stage_bytes, int stages) {
+  return 1024 + stages * stage_bytes + kEpiWarps * 2 * kEpiBuf + (2 * stages + 5) * 8 + 16;
+}
+// One ring stage: A (128 rows x 64 k) and B (64 k x bn columns) ...
+constexpr int single_stage_bytes(int bn) { return kBM * kBK * 2 + kBK * bn * 2; }
+// ... or, per CTA of a pair, `slabs` slabs of 128 rows of A and 128 columns of B.
+constexpr int pair_stage_bytes(int slabs) { return slabs * kBM * kBK * 2 + kBK * 128 * 2; }
+
 template <int BN, int STAGES>
 struct TileCfg {
   static constexpr int kABytes = kBM * kBK * 2;
@@ -51,7 +62,8 @@ struct TileCfg {
   static constexpr uint32_t kTmemCols = 2 * BN;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kSmemBytes == tile_smem_formula(single_stage_bytes(BN), STAGES), "layout");
+  static_assert(kSmemBytes <= kMaxDynamicSmem, "shared memory budget");
 };
 
 // The CTA-pair kernel: a (256 * SLABS) x 256 output tile per pair of SMs.
@@ -78,8 +90,54 @@ struct PairCfg {
   static constexpr uint32_t kTmemCols = 512;
   static_assert(SLABS == 1 || SLABS == 2, "SLABS");
   static_assert(kNBuf * SLABS * kBN == 512, "TMEM columns");
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kSmemBytes == tile_smem_formula(pair_stage_bytes(SLABS), STAGES), "layout");
+  static_assert(kSmemBytes <= kMaxDynamicSmem, "shared memory budget");
 };
+
+// Configurations compiled (for every activation): each tile shape with every
+// ring depth from 3 up to what fits the shared-memory budget.  A ring of 2
+// cannot keep a load in flight while the MMA reads the other stage and the
+// next load waits, so it is not built.
+struct TileVariant {
+  int kernel;  // GEMM_PATH_TILE / _TILE_PAIR / _TILE_PAIR_TALL
+  int block_n;
+  int stages;
+};
+constexpr TileVariant kTileVariants[] = {
+    {GEMM_PATH_TILE, 128, 3},      {GEMM_PATH_TILE, 128, 4},      {GEMM_PATH_TILE, 128, 5},
+    {GEMM_PATH_TILE, 128, 6},      {GEMM_PATH_TILE, 256, 3},      {GEMM_PATH_TILE, 256, 4},
+    {GEMM_PATH_TILE_PAIR, 256, 3}, {GEMM_PATH_TILE_PAIR, 256, 4}, {GEMM_PATH_TILE_PAIR, 256, 5},
+    {GEMM_PATH_TILE_PAIR, 256, 6}, {GEMM_PATH_TILE_PAIR_TALL, 256, 3},
+    {GEMM_PATH_TILE_PAIR_TALL, 256, 4}};
+constexpr int kNumTileVariants = sizeof(kTileVariants) / sizeof(kTileVariants[0]);
+
+constexpr int variant_smem_bytes(int kernel, int block_n, int stages) {
+  return kernel == GEMM_PATH_TILE
+             ? (block_n == 128 || block_n == 256
+                    ? tile_smem_formula(single_stage_bytes(block_n), stages)
+                    : -1)
+         : block_n != 256                       ? -1
+         : kernel == GEMM_PATH_TILE_PAIR        ? tile_smem_formula(pair_stage_bytes(1), stages)
+         : kernel == GEMM_PATH_TILE_PAIR_TALL   ? tile_smem_formula(pair_stage_bytes(2), stages)
+                                                : -1;
+}
+
+// The table holds exactly the depths from 3 to the budget's limit.
+constexpr bool variants_complete() {
+  const int kinds[4][2] = {{GEMM_PATH_TILE, 128}, {GEMM_PATH_TILE, 256},
+                           {GEMM_PATH_TILE_PAIR, 256}, {GEMM_PATH_TILE_PAIR_TALL, 256}};
+  for (const auto& k : kinds) {
+    for (int st = 3; st <= 16; ++st) {
+      const bool fits = variant_smem_bytes(k[0], k[1], st) <= kMaxDynamicSmem;
+      bool built = false;
+      for (const auto& v : kTileVariants)
+        built = built || (v.kernel == k[0] && v.block_n == k[1] && v.stages == st);
+      if (fits != built) return false;
+    }
+  }
+  return true;
+}
+static_assert(variants_complete(), "built tile configurations != those within the budget");
 
 // Grouped-panel rasterisation: consecutive tile indices sweep group_m
 // tile-rows of one panel column by column, so the CTAs that run at the same
@@ -666,23 +724,14 @@ int encode_operand_maps(const GemmProblem& p, int a_rows, int b_cols, CUtensorMa
   return encode_tmap_f16_2d(tB, p.B, p.N, p.K, p.ldb, 64, kBK);  // 64 n by 64 k
 }
 
-// Rows of A per raster panel (TTC_GROUP_ROWS overrides it for tuning sweeps).
-int group_rows_setting() {
-  static const int g = [] {
-    const char* s = std::getenv("TTC_GROUP_ROWS");
-    const int v = s ? std::atoi(s) : 0;
-    return v > 0 ? v : 2048;
-  }();
-  return g;
-}
-
-int group_tiles(int tile_rows) {
-  const int g = group_rows_setting() / tile_rows;
+// Tile-rows per raster panel for `group_rows` rows of A.
+int group_tiles(int group_rows, int tile_rows) {
+  const int g = group_rows / tile_rows;
   return g > 0 ? g : 1;
 }
 
 template <int BN, int STAGES, int ACT>
-int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
+int launch_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
   using Cfg = TileCfg<BN, STAGES>;
   static std::atomic<uint64_t> attr_done{0};
   CUtensorMap tA, tB, tC;
@@ -709,12 +758,12 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d) {
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
-      static_cast<int>(p.K), p.layout, group_tiles(kBM), d.status, d.timeout_ns);
+      static_cast<int>(p.K), p.layout, group_tiles(group_rows, kBM), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
 template <int STAGES, int SLABS, int ACT>
-int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
+int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
   using Cfg = PairCfg<STAGES, SLABS>;
   static std::atomic<uint64_t> attr_done{0};
   static int max_pairs[64] = {};
@@ -756,40 +805,54 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d) {
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
-      static_cast<int>(p.K), p.layout, group_tiles(Cfg::kTileM), d.status, d.timeout_ns);
+      static_cast<int>(p.K), p.layout, group_tiles(group_rows, Cfg::kTileM), d.status,
+      d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
+}
+
+template <int KERNEL, int BN, int STAGES, int ACT>
+int launch_variant(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
+  if constexpr (KERNEL == GEMM_PATH_TILE)
+    return launch_impl<BN, STAGES, ACT>(p, d, group_rows);
+  else
+    return launch_pair_impl<STAGES, KERNEL == GEMM_PATH_TILE_PAIR_TALL ? 2 : 1, ACT>(p, d,
+                                                                                  group_rows);
+}
+
+// Finds the table entry of `c` at compile-time-unrolled depth I and launches
+// its kernel for the problem's activation.
+template <int I = 0>
+int dispatch_variant(const GemmProblem& p, const DeviceCtx& d, const KernelConfig& c) {
+  if constexpr (I == kNumTileVariants) {
+    return GEMM_ERR_CONFIG;
+  } else {
+    constexpr TileVariant v = kTileVariants[I];
+    if (c.kernel != v.kernel || c.block_n != v.block_n || c.stages != v.stages)
+      return dispatch_variant<I + 1>(p, d, c);
+    switch (p.act) {
+      case kActRelu: return launch_variant<v.kernel, v.block_n, v.stages, kActRelu>(p, d, c.group_rows);
+      case kActGelu: return launch_variant<v.kernel, v.block_n, v.stages, kActGelu>(p, d, c.group_rows);
+      default: return launch_variant<v.kernel, v.block_n, v.stages, kActNone>(p, d, c.group_rows);
+    }
+  }
 }
 
 }  // namespace
 
-int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d) {
-  // 128 x 256 tiles when there are enough of them to fill the GPU, otherwise
-  // 128 x 128 tiles (twice as many CTAs for small problems).
-  const int64_t tiles256 = ((p.M + kBM - 1) / kBM) * ((p.N + 255) / 256);
-  const bool wide = tiles256 >= d.sm_count;
-  switch (p.act) {
-    case kActRelu:
-      return wide ? launch_impl<256, 4, kActRelu>(p, d) : launch_impl<128, 6, kActRelu>(p, d);
-    case kActGelu:
-      return wide ? launch_impl<256, 4, kActGelu>(p, d) : launch_impl<128, 6, kActGelu>(p, d);
-    default:
-      return wide ? launch_impl<256, 4, kActNone>(p, d) : launch_impl<128, 6, kActNone>(p, d);
-  }
+int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d, const KernelConfig& c) {
+  return dispatch_variant(p, d, c);
 }
 
-int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d, int slabs) {
-  if (slabs == 2) {
-    switch (p.act) {
-      case kActRelu: return launch_pair_impl<4, 2, kActRelu>(p, d);
-      case kActGelu: return launch_pair_impl<4, 2, kActGelu>(p, d);
-      default: return launch_pair_impl<4, 2, kActNone>(p, d);
-    }
-  }
-  switch (p.act) {
-    case kActRelu: return launch_pair_impl<6, 1, kActRelu>(p, d);
-    case kActGelu: return launch_pair_impl<6, 1, kActGelu>(p, d);
-    default: return launch_pair_impl<6, 1, kActNone>(p, d);
-  }
+int tile_config_smem_bytes(int kernel, int block_n, int stages) {
+  if (stages < 1 || stages > 64) return -1;
+  return variant_smem_bytes(kernel, block_n, stages);
+}
+
+int tile_configs_built(KernelConfig* out, int cap) {
+  for (int i = 0; i < kNumTileVariants && i < cap; ++i)
+    out[i] = KernelConfig{kTileVariants[i].kernel, kTileVariants[i].block_n,
+                          kTileVariants[i].stages, 0, 0};
+  return kNumTileVariants;
 }
 
 }  // namespace ttc

@@ -19,6 +19,27 @@ struct GemmProblem {
   cudaStream_t stream;
 };
 
+// One kernel configuration, resolved (no zero "default" fields left): the
+// validated form of the public gemm_config.
+struct KernelConfig {
+  int kernel;      // GEMM_PATH_TILE / _TILE_PAIR / _TILE_PAIR_TALL / _SKINNY
+  int block_n;     // output columns per CTA (TILE: 128 or 256) or per pair / tile (256)
+  int stages;      // depth of the shared-memory operand ring
+  int group_rows;  // tile kernels: rows of A per raster panel
+  int splits;      // SKINNY: k-slices per tile, 0 = chosen from the shape
+};
+
+// Largest dynamic shared memory a CTA may opt into on sm_100.
+constexpr int kMaxDynamicSmem = 232448;
+
+// Defaults used by GEMM_PATH_AUTO and by a gemm_config field left at 0.
+constexpr int kDefaultGroupRows = 2048;
+constexpr int kDefaultStagesTile128 = 6;
+constexpr int kDefaultStagesTile256 = 4;
+constexpr int kDefaultStagesPair = 6;
+constexpr int kDefaultStagesTall = 4;
+constexpr int kDefaultStagesSkinny = 5;
+
 struct DeviceCtx {
   int device;
   int sm_count;
@@ -43,19 +64,27 @@ int encode_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
                        uint64_t ld, uint32_t box_inner, uint32_t box_outer);
 
 // Large-shape path: persistent warp-specialised tcgen05 kernel, one SM per
-// 128-row tile ...
-int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d);
-// ... or a pair of SMs per (256 * slabs) x 256 tile (tcgen05.mma.cta_group::2),
-// slabs = 1 or 2.
-int launch_tile_pair_gemm(const GemmProblem& p, const DeviceCtx& d, int slabs);
+// 128 x block_n tile (GEMM_PATH_TILE), or a pair of SMs per 256 x 256
+// (GEMM_PATH_TILE_PAIR) or 512 x 256 (GEMM_PATH_TILE_PAIR_TALL) tile
+// (tcgen05.mma.cta_group::2).  Returns GEMM_ERR_CONFIG when no kernel was
+// compiled for (kernel, block_n, stages).
+int launch_tile_gemm(const GemmProblem& p, const DeviceCtx& d, const KernelConfig& c);
+// Dynamic shared memory per CTA of a tile-kernel configuration (built or
+// not), or -1 when (kernel, block_n) names no tile kernel.
+int tile_config_smem_bytes(int kernel, int block_n, int stages);
+// Tile-kernel configurations with a compiled kernel: writes up to `cap` of
+// them to `out` (group_rows and splits 0) and returns how many there are.
+int tile_configs_built(KernelConfig* out, int cap);
 
 // Small-M path: swap-AB, lock-step split-K kernel.  `workspace` holds
 // per-tile arrival counters and split-K partial tiles (counters must be zero
 // on entry; the kernel leaves them zero).
 size_t skinny_workspace_bytes(int sm_count, int m_pad);
 int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* workspace,
-                       size_t workspace_bytes);
+                       size_t workspace_bytes, const KernelConfig& c);
 int skinny_m_pad(int64_t M);  // MMA N used for M rows (0 if M is too large)
+int skinny_config_smem_bytes(int stages);
+int skinny_configs_built(KernelConfig* out, int cap);
 
 // The small-M kernel with its scratch in a fixed device array of the library
 // (no allocation); M <= 32.  Returns GEMM_ERR_SCRATCH_LIMIT beyond.

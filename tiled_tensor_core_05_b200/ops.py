@@ -25,6 +25,20 @@ _ACTS = {"none": ACT_NONE, "relu": ACT_RELU, "gelu": ACT_GELU}
 
 _lib = None
 
+
+class GemmConfig(ctypes.Structure):
+    """``gemm_config`` of the C ABI: one kernel configuration (0 = default)."""
+    _fields_ = [("kernel", ctypes.c_int32), ("block_n", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("group_rows", ctypes.c_int32),
+                ("splits", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {f: int(getattr(self, f)) for f, _ in self._fields_}
+
+    def __repr__(self):
+        return "GemmConfig(" + ", ".join(f"{k}={v}" for k, v in self.as_dict().items()) + ")"
+
+
 _SIGNATURES = {
     "gemm_relu_f16": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
                       ctypes.c_int),
@@ -36,6 +50,12 @@ _SIGNATURES = {
                           [ctypes.c_int, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
     "gemm_f16_general": ([ctypes.c_void_p] * 4 + [ctypes.c_int64] * 6 +
                          [ctypes.c_int] * 4 + [ctypes.c_void_p], ctypes.c_int),
+    "gemm_f16_config": ([ctypes.c_void_p] * 4 + [ctypes.c_int64] * 6 + [ctypes.c_int] * 3 +
+                        [ctypes.POINTER(GemmConfig), ctypes.c_void_p], ctypes.c_int),
+    "gemm_config_smem_bytes": ([ctypes.POINTER(GemmConfig)], ctypes.c_int),
+    "gemm_config_list": ([ctypes.POINTER(GemmConfig), ctypes.c_int], ctypes.c_int),
+    "gemm_auto_config": ([ctypes.c_int64] * 3 + [ctypes.c_int, ctypes.POINTER(GemmConfig)],
+                         ctypes.c_int),
     "gemm_select_path": ([ctypes.c_int64] * 3, ctypes.c_int),
     "gemm_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "gemm_get_device_status": ([ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -176,6 +196,65 @@ def gemm_general(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = N
                                     int(bool(trans_a)), int(bool(trans_b)), code, int(path),
                                     _stream_handle(stream, dev))
     _check(rc, "gemm_f16_general")
+    return out
+
+
+def _as_config(cfg) -> GemmConfig:
+    if isinstance(cfg, GemmConfig):
+        return cfg
+    return GemmConfig(**{k: int(v) for k, v in dict(cfg).items()})
+
+
+def gemm_config_run(a: torch.Tensor, b: torch.Tensor, cfg, bias: torch.Tensor | None = None,
+                    act: str | int = "relu", out: torch.Tensor | None = None, *,
+                    trans_a: bool = False, trans_b: bool = False,
+                    stream=None) -> torch.Tensor:
+    """:func:`gemm_general` with an explicit kernel configuration ``cfg`` (a
+    :class:`GemmConfig` or a dict of its fields) instead of a path."""
+    if a.dtype != torch.float16 or b.dtype != torch.float16:
+        raise TypeError("a and b must be torch.float16")
+    M, K = (a.shape[1], a.shape[0]) if trans_a else tuple(a.shape)
+    K2, N = (b.shape[1], b.shape[0]) if trans_b else tuple(b.shape)
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    if bias is not None and (bias.dtype != torch.float16 or bias.numel() != N):
+        raise ValueError("bias must be fp16 with N elements")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
+    c = _as_config(cfg)
+    dev = a.device
+    with torch.cuda.device(dev):
+        rc = lib().gemm_f16_config(a.data_ptr(), b.data_ptr(),
+                                   None if bias is None else bias.data_ptr(), out.data_ptr(),
+                                   M, N, K, _ld_padded(a), _ld_padded(b), _ld_padded(out),
+                                   int(bool(trans_a)), int(bool(trans_b)), code,
+                                   ctypes.byref(c), _stream_handle(stream, dev))
+    _check(rc, f"gemm_f16_config {c!r}")
+    return out
+
+
+def config_smem_bytes(cfg) -> int:
+    """Shared memory per CTA that ``cfg`` needs (negative status if it names
+    no kernel)."""
+    return int(lib().gemm_config_smem_bytes(ctypes.byref(_as_config(cfg))))
+
+
+def config_list() -> list[GemmConfig]:
+    """The compiled kernel configurations (kernel, block_n, stages)."""
+    n = int(lib().gemm_config_list(None, 0))
+    arr = (GemmConfig * n)()
+    lib().gemm_config_list(arr, n)
+    return [GemmConfig(**c.as_dict()) for c in arr]
+
+
+def auto_config(M: int, N: int, K: int, act: str | int = "relu", device=None) -> GemmConfig:
+    """The configuration GEMM_PATH_AUTO takes for this problem on the device."""
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    out = GemmConfig()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        _check(lib().gemm_auto_config(M, N, K, code, ctypes.byref(out)), "gemm_auto_config")
     return out
 
 

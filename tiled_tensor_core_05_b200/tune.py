@@ -1,0 +1,350 @@
+"""Offline sweep of kernel configurations (tile shape, ring depth, CTA pairing,
+raster panel, split-K) for the fused fp16 GEMM + activation.
+
+    python -m tiled_tensor_core_05_b200.tune [--workloads cube8192,mlp_up,...]
+                                             [--steps 30] [--out table.md] [--json out.json]
+
+The tuning workflow of "TileLang simplifica la creación de kernels GPU de alto
+rendimiento" (posicionamiento-web.ar) and "TileLang explicado: kernels de IA
+escritos por mosaicos" (easyairoute.com), in their sections on tuning tile
+sizes, pipeline stages and L2 ordering for each GPU and validating every
+candidate before trusting its time, done once, offline: the library never
+times or picks among configurations at run time.  Its GEMM_PATH_AUTO rules and
+defaults are set from the table this script writes.
+
+For each workload:
+  1. the candidate space: every tile shape (128 x 128 and 128 x 256 on one SM,
+     256 x 256 and 512 x 256 on a CTA pair, the 256-column small-M kernel when
+     M <= 64) x ring depths 3..8 x raster panels (1, 2, 4, ... tile-rows, up to
+     all of them) or k-slices;
+  2. pruning: depths whose shared memory (gemm_config_smem_bytes) exceeds the
+     227 KiB a CTA can opt into, duplicate panels (a panel of more tile-rows
+     than the problem has is the whole column), k-slice counts the split-K
+     workspace or K cannot hold;
+  3. validation of each survivor against torch's fp32 product, activated, with
+     the pages' check |c - ref| <= 1e-2 + 1e-2 |ref| plus c > 0 wherever
+     ref > 1e-2 (ReLU); a candidate that fails is reported and never ranked;
+  4. timing: `steps` back-to-back launches between two CUDA events after 3
+     warm-up launches (operands larger than L2 for the large workloads; the
+     small ones run L2-warm);
+  5. the leaders (and the AUTO configuration) re-timed in interleaved rounds
+     (a fresh random order each round), because the power-capped SM clock
+     drifts by more than the differences between neighbouring candidates; the
+     median of the rounds is ranked, the spread of the rounds and the median
+     SM clock (NVML, sampled during each block) are reported beside it, and
+     ms x MHz (thousands of SM cycles) separates a faster kernel from a
+     higher clock.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import random
+import statistics
+import sys
+import time
+
+from . import ops
+from .workloads import WORKLOADS, Workload, make_inputs
+
+SMEM_BUDGET = 232448  # bytes of dynamic shared memory a CTA may opt into (sm_100)
+STAGE_RANGE = range(3, 9)
+TILE_KINDS = [(ops.PATH_TILE, 128), (ops.PATH_TILE, 256), (ops.PATH_TILE_PAIR, 256),
+              (ops.PATH_TILE_PAIR_TALL, 256)]
+TILE_ROWS = {ops.PATH_TILE: 128, ops.PATH_TILE_PAIR: 256, ops.PATH_TILE_PAIR_TALL: 512}
+KERNEL_NAMES = {ops.PATH_TILE: "tile", ops.PATH_SKINNY: "skinny",
+                ops.PATH_TILE_PAIR: "pair", ops.PATH_TILE_PAIR_TALL: "pair-tall"}
+SKINNY_WIDTH = 256
+
+# extra shapes of the sweep beside the named workloads: a small-M product
+# with few column tiles, where split-K has room to act
+EXTRA = {w.name: w for w in [
+    Workload("decode_n4096", 32, 4096, 8192, 5, 1.0, 0.02,
+             "M=32, K=8192, N=4096; A ~ N(0,1), B ~ N(0, 0.02^2), seed 5"),
+    Workload("decode_m16_n8192_k4096", 16, 8192, 4096, 6, 1.0, 0.02,
+             "M=16, K=4096, N=8192; A ~ N(0,1), B ~ N(0, 0.02^2), seed 6"),
+    Workload("decode_m64_n2048_k8192", 64, 2048, 8192, 7, 1.0, 0.02,
+             "M=64, K=8192, N=2048; A ~ N(0,1), B ~ N(0, 0.02^2), seed 7"),
+    Workload("decode_n1024_k16384", 32, 1024, 16384, 8, 1.0, 0.02,
+             "M=32, K=16384, N=1024; A ~ N(0,1), B ~ N(0, 0.02^2), seed 8"),
+    Workload("decode_n14336_k4096", 32, 14336, 4096, 9, 1.0, 0.02,
+             "M=32, K=4096, N=14336; A ~ N(0,1), B ~ N(0, 0.02^2), seed 9"),
+]}
+
+
+def describe(cfg: dict) -> str:
+    k = cfg["kernel"]
+    if k == ops.PATH_SKINNY:
+        s = cfg["splits"]
+        return f"skinny st{cfg['stages']} splits={'auto' if s == 0 else s}"
+    rows = TILE_ROWS[k]
+    return (f"{KERNEL_NAMES[k]} {rows}x{cfg['block_n']} st{cfg['stages']} "
+            f"panel={cfg['group_rows']}")
+
+
+def candidates(M: int, N: int, K: int, sm_count: int, smem_fn, budget: int = SMEM_BUDGET):
+    """(kept, pruned): kept is a list of config dicts; pruned a list of
+    (config dict, reason).  `smem_fn(cfg) -> bytes` is the library's formula."""
+    kept, pruned = [], []
+    kinds = list(TILE_KINDS)
+    if M <= 64:
+        kinds.append((ops.PATH_SKINNY, SKINNY_WIDTH))
+    for kernel, bn in kinds:
+        for st in STAGE_RANGE:
+            base = {"kernel": kernel, "block_n": bn, "stages": st, "group_rows": 0,
+                    "splits": 0}
+            smem = smem_fn(base)
+            if smem > budget:
+                pruned.append((base, f"shared memory {smem} > {budget}"))
+                continue
+            if kernel == ops.PATH_SKINNY:
+                tiles = -(-N // SKINNY_WIDTH)
+                kb = -(-K // 64)
+                seen = set()
+                for s in (0, 1, 2, 3, 4, 6, 8, 12, 16, 24, 32):
+                    if s > kb or (s > 1 and s * tiles > sm_count):
+                        pruned.append(({**base, "splits": s}, "k-slices do not fit"))
+                        continue
+                    if s in seen:
+                        continue
+                    seen.add(s)
+                    kept.append({**base, "splits": s})
+            else:
+                rows = TILE_ROWS[kernel]
+                tile_rows = -(-M // rows)
+                seen = set()
+                g = 1
+                while True:
+                    eff = min(g, tile_rows)
+                    if eff not in seen:
+                        seen.add(eff)
+                        kept.append({**base, "group_rows": eff * rows})
+                    if g >= tile_rows:
+                        break
+                    g *= 2
+    return kept, pruned
+
+
+# ------------------------------------------------------------ measurement ---
+
+def _reference(a, b, bias, act):
+    import torch
+    ref = torch.matmul(a.float(), b.float())
+    if bias is not None:
+        ref += bias.float()[None, :]
+    if act == "relu":
+        ref.clamp_(min=0.0)
+    elif act == "gelu":
+        ref = torch.nn.functional.gelu(ref)
+    return ref
+
+
+def check(c, ref, act) -> tuple[bool, float]:
+    """The pages' tolerance (and, after ReLU, the sign/zero pattern)."""
+    import torch
+    cf = c.float()
+    err = (cf - ref).abs()
+    ok = bool(torch.all(err <= 1e-2 + 1e-2 * ref.abs()).item())
+    ok = ok and bool(torch.isfinite(cf).all().item())
+    if act == "relu":
+        ok = ok and bool(torch.all(cf[ref > 1e-2] > 0).item())
+    return ok, float(err.max().item())
+
+
+_BLOCK = [0]
+
+
+def time_config(run, steps: int, stream, sampler=None):
+    """(ms per launch, median SM MHz during the block or None)."""
+    import torch
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    _BLOCK[0] += 1
+    tag = str(_BLOCK[0])
+    if sampler is not None:
+        sampler.mark("s" + tag)
+    e0.record(stream)
+    for _ in range(steps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mhz = None
+    if sampler is not None and sampler.ok:
+        sampler.mark("e" + tag)
+        mhz = sampler.summary("s" + tag, "e" + tag).get("sm_mhz")
+    return e0.elapsed_time(e1) / steps, mhz
+
+
+def sweep_workload(w: Workload, act: str, use_bias: bool, steps: int, rounds: int,
+                   leaders: int, log=print, sampler=None, seed: int = 0) -> dict:
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    a_h, b_h = make_inputs(w.M, w.N, w.K, w.seed, w.a_scale, w.b_scale)
+    a, b = a_h.to(dev), b_h.to(dev)
+    bias = None
+    if use_bias:
+        g = torch.Generator(device="cpu")
+        g.manual_seed(w.seed + 1000)
+        bias = (torch.randn(w.N, generator=g) * 0.5).to(torch.float16).to(dev)
+    c = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
+    ref = _reference(a, b, bias, act)
+    stream = torch.cuda.current_stream(dev)
+    auto = ops.auto_config(w.M, w.N, w.K, act).as_dict()
+    kept, pruned = candidates(w.M, w.N, w.K, sm_count, ops.config_smem_bytes)
+    if not any(cfg == auto for cfg in kept):
+        kept.append(auto)
+    results = []
+    t_start = time.time()
+    for cfg in kept:
+        def run(cfg=cfg):
+            ops.gemm_config_run(a, b, cfg, bias, act, c)
+        c.fill_(float("nan"))
+        run()
+        torch.cuda.synchronize()
+        ok, err = check(c, ref, act)
+        status = ops.device_status()
+        entry = {"config": cfg, "desc": describe(cfg), "smem": ops.config_smem_bytes(cfg),
+                 "parity": ok and status == 0, "max_abs_err": err}
+        if entry["parity"]:
+            entry["first_ms"], entry["first_mhz"] = time_config(run, steps, stream, sampler)
+        results.append(entry)
+    ranked = sorted((r for r in results if r["parity"]), key=lambda r: r["first_ms"])
+    top = ranked[:leaders]
+    auto_entry = next(r for r in results if r["config"] == auto)
+    if auto_entry not in top and auto_entry["parity"]:
+        top.append(auto_entry)
+    for r in top:
+        r["round_ms"], r["round_mhz"] = [], []
+    rng = random.Random(seed)
+    for _ in range(rounds):
+        order = list(top)
+        rng.shuffle(order)
+        for r in order:
+            def run(cfg=r["config"]):
+                ops.gemm_config_run(a, b, cfg, bias, act, c)
+            ms, mhz = time_config(run, steps, stream, sampler)
+            r["round_ms"].append(ms)
+            r["round_mhz"].append(mhz)
+    for r in top:
+        r["ms"] = statistics.median(r["round_ms"])
+        r["spread_ms"] = [min(r["round_ms"]), max(r["round_ms"])]
+        mhz = [x for x in r["round_mhz"] if x]
+        r["mhz"] = statistics.median(mhz) if mhz else None
+        kc = [m * f for m, f in zip(r["round_ms"], r["round_mhz"]) if f]
+        r["kcycles"] = statistics.median(kc) if kc else None
+    top.sort(key=lambda r: r["ms"])
+    log(f"{w.name} act={act} bias={use_bias}: {len(kept)} candidates, {len(pruned)} pruned, "
+        f"{sum(not r['parity'] for r in results)} failed parity, {time.time() - t_start:.1f} s")
+    return {"workload": w.name, "shape": [w.M, w.N, w.K], "act": act, "bias": use_bias,
+            "sm_count": sm_count, "auto": auto, "results": results, "leaders": top,
+            "pruned": [(cfg, why) for cfg, why in pruned]}
+
+
+# ----------------------------------------------------------------- report ---
+
+def _rate(w_shape, ms, skinny_like: bool):
+    M, N, K = w_shape
+    if skinny_like:
+        return f"{2 * (M * K + K * N + M * N) / (ms * 1e-3) / 1e9:.0f} GB/s"
+    return f"{2 * M * N * K / (ms * 1e-3) / 1e12:.0f} TFLOP/s"
+
+
+def to_markdown(reports: list[dict], command: str, device: str) -> str:
+    out = [f"# Kernel configuration sweep ({device})", "",
+           f"Command: `{command}`", "",
+           "Every candidate was validated against torch's fp32 product with the pages' "
+           "tolerance before it was timed; `first` is one block of back-to-back launches, "
+           "`median` the median of interleaved re-timing rounds of the leaders (and of the "
+           "AUTO configuration).", ""]
+    for rep in reports:
+        M, N, K = rep["shape"]
+        skinny_like = M <= 64
+        fails = [r for r in rep["results"] if not r["parity"]]
+        out += [f"## {rep['workload']} ({M} x {N} x {K}, act={rep['act']}"
+                f"{', bias' if rep['bias'] else ''})", "",
+                f"{len(rep['results'])} candidates timed, {len(rep['pruned'])} pruned "
+                f"(shared memory / k-slices), {len(fails)} failed validation.  "
+                f"AUTO: `{describe(rep['auto'])}`.", "",
+                "| rank | configuration | smem KiB | median ms | rounds min-max | rate | "
+                "SM MHz | ms x MHz | vs AUTO |",
+                "|---|---|---|---|---|---|---|---|---|"]
+        auto_ms = next((r["ms"] for r in rep["leaders"] if r["config"] == rep["auto"]), None)
+        for i, r in enumerate(rep["leaders"]):
+            rel = f"{(auto_ms / r['ms'] - 1) * 100:+.1f} %" if auto_ms else "-"
+            tag = " (AUTO)" if r["config"] == rep["auto"] else ""
+            mhz = f"{r['mhz']:.0f}" if r.get("mhz") else "-"
+            kc = f"{r['kcycles']:.0f}" if r.get("kcycles") else "-"
+            lo, hi = r["spread_ms"]
+            out.append(f"| {i + 1} | `{r['desc']}`{tag} | {r['smem'] / 1024:.0f} | "
+                       f"{r['ms']:.4f} | {lo:.4f}-{hi:.4f} | "
+                       f"{_rate(rep['shape'], r['ms'], skinny_like)} | {mhz} | {kc} | {rel} |")
+        out += ["", "<details><summary>all candidates (first timing)</summary>", "",
+                "| configuration | ms | parity | max abs err |", "|---|---|---|---|"]
+        for r in sorted(rep["results"], key=lambda r: r.get("first_ms", math.inf)):
+            ms = f"{r['first_ms']:.4f}" if "first_ms" in r else "-"
+            out.append(f"| `{r['desc']}` | {ms} | {'ok' if r['parity'] else 'FAIL'} | "
+                       f"{r['max_abs_err']:.3g} |")
+        out += ["", "</details>", ""]
+    return "\n".join(out) + "\n"
+
+
+DEFAULT_SWEEP = [("cube8192", "relu", False), ("mlp_up", "relu", False),
+                 ("mlp_up", "gelu", True), ("decode", "relu", False),
+                 ("decode_n4096", "relu", False), ("decode_m16_n8192_k4096", "relu", False),
+                 ("decode_m64_n2048_k8192", "relu", False),
+                 ("decode_n1024_k16384", "relu", False),
+                 ("decode_n14336_k4096", "relu", False), ("cube1024", "relu", False)]
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--workloads", default=None,
+                    help="comma list of name[:act[:bias]] (default: the standard sweep)")
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--rounds", type=int, default=7)
+    ap.add_argument("--leaders", type=int, default=6)
+    ap.add_argument("--out", default=None, help="write the markdown table here")
+    ap.add_argument("--json", default=None, help="write all results as JSON here")
+    args = ap.parse_args(argv)
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("the sweep needs a CUDA device")
+    plan = DEFAULT_SWEEP
+    if args.workloads:
+        plan = []
+        for item in args.workloads.split(","):
+            parts = item.split(":")
+            plan.append((parts[0], parts[1] if len(parts) > 1 else "relu",
+                         len(parts) > 2 and parts[2] == "bias"))
+    from .clocks import ClockSampler, gpu_id_for
+    sampler = ClockSampler(gpu_id_for(torch.cuda.current_device()))
+    sampler.wait_first()
+    reports = []
+    try:
+        for i, (name, act, use_bias) in enumerate(plan):
+            w = WORKLOADS.get(name) or EXTRA[name]
+            reports.append(sweep_workload(w, act, use_bias, args.steps, args.rounds,
+                                          args.leaders, sampler=sampler, seed=i,
+                                          log=lambda *x: print(*x, file=sys.stderr, flush=True)))
+    finally:
+        sampler.stop()
+    device = torch.cuda.get_device_name()
+    command = "python -m tiled_tensor_core_05_b200.tune " + " ".join(argv or sys.argv[1:])
+    md = to_markdown(reports, command.strip(), device)
+    if args.out:
+        with open(args.out, "w") as f:
+            f.write(md)
+    else:
+        print(md)
+    if args.json:
+        with open(args.json, "w") as f:
+            json.dump(reports, f, indent=1)
+
+
+if __name__ == "__main__":
+    main()
