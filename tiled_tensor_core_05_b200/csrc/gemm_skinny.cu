@@ -368,13 +368,20 @@ constexpr size_t counter_bytes(int n) {
 }
 
 // Number of k-slices per tile: 1 when the tiles already cover the SMs,
-// otherwise as many as fit on the idle SMs, keeping at least 4 k-blocks of 64
-// per slice and at most `max_items` (tile, slice) pairs.
-int choose_slices(int64_t tiles, int64_t KB, int sm_count, int64_t max_items) {
+// otherwise as many as fit on the idle SMs, with at least 16 k-blocks of 64
+// per slice, S * MP <= 256 (the last slice to arrive sums the S partial tiles
+// of 256 x MP fp32 one after another, a cost that grows with S * MP), and at
+// most `max_items` (tile, slice) pairs.  Fitted to a sweep of small-M shapes
+// (M 16-64, N 1024-28672, K 4096-16384): the best or tied-best slice count on
+// each; the former rule (up to SMs / tiles slices of >= 4 k-blocks) was up to
+// 1.85x slower where few column tiles allowed many slices.
+int choose_slices(int64_t tiles, int64_t KB, int MP, int sm_count, int64_t max_items) {
   if (tiles >= sm_count) return 1;
   int64_t s = sm_count / tiles;
-  const int64_t by_k = KB / 4;
+  const int64_t by_k = KB / 16;
+  const int64_t by_fixup = 256 / MP;
   if (s > by_k) s = by_k;
+  if (s > by_fixup) s = by_fixup;
   if (s * tiles > max_items) s = max_items / tiles;
   return s < 1 ? 1 : static_cast<int>(s);
 }
@@ -390,7 +397,7 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_by
   const int64_t tiles = (p.N + kTW - 1) / kTW;
   if (splits < 0 || splits > KB || (splits > 1 && splits * tiles > max_items))
     return GEMM_ERR_CONFIG;
-  const int S = splits > 0 ? splits : choose_slices(tiles, KB, d.sm_count, max_items);
+  const int S = splits > 0 ? splits : choose_slices(tiles, KB, MP, d.sm_count, max_items);
   int* counters = nullptr;
   float* partials = nullptr;
   if (S > 1) {

@@ -180,7 +180,13 @@ def time_config(run, steps: int, stream, sampler=None):
 
 
 def sweep_workload(w: Workload, act: str, use_bias: bool, steps: int, rounds: int,
-                   leaders: int, log=print, sampler=None, seed: int = 0) -> dict:
+                   leaders: int, log=print, sampler=None, seed: int = 0,
+                   round_steps: int | None = None, cool_s: float = 0.0,
+                   only: list[dict] | None = None) -> dict:
+    """Validate and time the candidates of `w` (or only the configurations in
+    `only`, with the AUTO one added), then re-time the leaders in `rounds`
+    shuffled rounds of `round_steps` launches (default `steps`), idling
+    `cool_s` seconds before each block."""
     import torch
     dev = torch.device("cuda", torch.cuda.current_device())
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -196,6 +202,9 @@ def sweep_workload(w: Workload, act: str, use_bias: bool, steps: int, rounds: in
     stream = torch.cuda.current_stream(dev)
     auto = ops.auto_config(w.M, w.N, w.K, act).as_dict()
     kept, pruned = candidates(w.M, w.N, w.K, sm_count, ops.config_smem_bytes)
+    if only is not None:
+        full = {"kernel": 0, "block_n": 0, "stages": 0, "group_rows": 0, "splits": 0}
+        kept, pruned = [{**full, **c} for c in only], []
     if not any(cfg == auto for cfg in kept):
         kept.append(auto)
     results = []
@@ -227,7 +236,9 @@ def sweep_workload(w: Workload, act: str, use_bias: bool, steps: int, rounds: in
         for r in order:
             def run(cfg=r["config"]):
                 ops.gemm_config_run(a, b, cfg, bias, act, c)
-            ms, mhz = time_config(run, steps, stream, sampler)
+            if cool_s > 0:
+                time.sleep(cool_s)
+            ms, mhz = time_config(run, round_steps or steps, stream, sampler)
             r["round_ms"].append(ms)
             r["round_mhz"].append(mhz)
     for r in top:
@@ -307,6 +318,13 @@ def main(argv=None):
                     help="comma list of name[:act[:bias]] (default: the standard sweep)")
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--rounds", type=int, default=7)
+    ap.add_argument("--round-steps", type=int, default=None,
+                    help="launches per block in the re-timing rounds (default: --steps)")
+    ap.add_argument("--cool", type=float, default=0.0,
+                    help="seconds of idle before each re-timing block")
+    ap.add_argument("--only", default=None,
+                    help="';'-separated configurations kernel,block_n,stages,group_rows,splits "
+                         "to time instead of the candidate space (with AUTO added)")
     ap.add_argument("--leaders", type=int, default=6)
     ap.add_argument("--out", default=None, help="write the markdown table here")
     ap.add_argument("--json", default=None, help="write all results as JSON here")
@@ -321,6 +339,11 @@ def main(argv=None):
             parts = item.split(":")
             plan.append((parts[0], parts[1] if len(parts) > 1 else "relu",
                          len(parts) > 2 and parts[2] == "bias"))
+    only = None
+    if args.only:
+        keys = ("kernel", "block_n", "stages", "group_rows", "splits")
+        only = [dict(zip(keys, (int(v) for v in item.split(","))))
+                for item in args.only.split(";") if item.strip()]
     from .clocks import ClockSampler, gpu_id_for
     sampler = ClockSampler(gpu_id_for(torch.cuda.current_device()))
     sampler.wait_first()
@@ -330,6 +353,8 @@ def main(argv=None):
             w = WORKLOADS.get(name) or EXTRA[name]
             reports.append(sweep_workload(w, act, use_bias, args.steps, args.rounds,
                                           args.leaders, sampler=sampler, seed=i,
+                                          round_steps=args.round_steps, cool_s=args.cool,
+                                          only=only,
                                           log=lambda *x: print(*x, file=sys.stderr, flush=True)))
     finally:
         sampler.stop()
