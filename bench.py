@@ -281,6 +281,35 @@ def oracle_seconds_per_row(oracle, a, b) -> float:
     return max(time.perf_counter() - t0, 1e-6) / rows
 
 
+def stream_read_probe(gib: float = 2.0, steps: int = 20):
+    """Achievable HBM streaming-read bandwidth on this GPU: the library's
+    read probe (every byte of a buffer larger than L2 read once) timed with
+    CUDA events.  Context for the small-M kernel, which reads B once."""
+    import torch
+    from tiled_tensor_core_05_b200 import ops
+    n = int(gib * 2 ** 30) // 4
+    buf = torch.ones(n, dtype=torch.int32, device="cuda")
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        ops.read_probe(buf, sink)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        ops.read_probe(buf, sink)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    nbytes = n * 4
+    del buf
+    return {"what": "gemm_read_probe: every byte of a %.0f GiB buffer read once with 16-byte "
+                    "streaming loads (context for the small-M roofline)" % gib,
+            "bytes": nbytes, "ms_per_launch": round(ms, 4),
+            "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+
+
 def cpu_baseline(name, budget_s=10.0):
     """The oracle timed on a bounded sample (leading rows) of the workload."""
     import oracle
@@ -430,6 +459,13 @@ def run_ours(args):
                                                         NOMINAL_FP16_TFLOPS, 2)
             others.append(entry)
         line["other_workloads"] = others
+        probe = stream_read_probe()
+        line["context_stream_read_probe"] = probe
+        for entry in [line] + others:
+            gbs = entry.get("gbs") if entry is not line else (
+                value / world if unit == "GB/s" else None)
+            if gbs:
+                entry["frac_of_read_probe"] = round(gbs / probe["gbs"], 4)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget)
     if dist is not None:

@@ -247,6 +247,20 @@ GEMM_API int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_
 GEMM_API int gemm_activation_f32(const void* x, void* y, int64_t n, int activation,
                                  gemm_stream_t stream);
 
+/* Measurement tool, not part of the GEMM: reads n_bytes of device memory at
+ * `src` once, with 16-byte streaming loads spread over the whole GPU, and
+ * stores the XOR of all its 32-bit words in *sink (a device pointer to 4
+ * bytes, zeroed first on `stream`).  Timed over a buffer larger than L2 it
+ * gives the streaming-read bandwidth that bounds the small-M kernel, which
+ * reads B once.  It is the bandwidth-bound environment check of "TileLang
+ * simplifica la creación de kernels GPU de alto rendimiento"
+ * (posicionamiento-web.ar), section "Del entorno CUDA a la primera medición
+ * reproducible" (a vector sum there), reduced to its reads.
+ *   - src 16-byte aligned, n_bytes a multiple of 16 (0 stores 0); sink
+ *     4-byte aligned; both device memory of the current device.
+ *   - Asynchronous on `stream`.  Returns GEMM_OK or a negative gemm_status. */
+GEMM_API int gemm_read_probe(const void* src, int64_t n_bytes, void* sink, gemm_stream_t stream);
+
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
 GEMM_API int gemm_abi_version(void);
 

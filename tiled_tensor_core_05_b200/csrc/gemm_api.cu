@@ -241,6 +241,31 @@ __global__ void wait_probe_kernel(int* status, uint64_t timeout_ns) {
   }
 }
 
+// Streaming-read probe: the grid reads n16 16-byte words once, each thread
+// four independent streaming (evict-first) loads per step strided by the
+// whole grid, and folds them with XOR so no load is dead; one atomic XOR per
+// warp into *sink.
+__global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict__ src,
+                                                         int64_t n16, unsigned* sink) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  unsigned acc = 0;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    const uint4 v0 = __ldcs(src + i);
+    const uint4 v1 = __ldcs(src + i + stride);
+    const uint4 v2 = __ldcs(src + i + 2 * stride);
+    const uint4 v3 = __ldcs(src + i + 3 * stride);
+    acc ^= v0.x ^ v0.y ^ v0.z ^ v0.w ^ v1.x ^ v1.y ^ v1.z ^ v1.w;
+    acc ^= v2.x ^ v2.y ^ v2.z ^ v2.w ^ v3.x ^ v3.y ^ v3.z ^ v3.w;
+  }
+  for (; i < n16; i += stride) {
+    const uint4 v = __ldcs(src + i);
+    acc ^= v.x ^ v.y ^ v.z ^ v.w;
+  }
+  acc = __reduce_xor_sync(0xffffffffu, acc);
+  if ((threadIdx.x & 31) == 0) atomicXor(sink, acc);
+}
+
 int read_and_clear_status(const DeviceCtx& d, cudaStream_t stream, int* out) {
   int host = 0;
   if (cudaMemcpyAsync(&host, d.status, sizeof(int), cudaMemcpyDeviceToHost, stream) !=
@@ -633,6 +658,26 @@ int gemm_selftest_wait_timeout(int64_t timeout_ns, gemm_stream_t stream, int* de
   wait_probe_kernel<<<1, 32, 0, stream>>>(d.status, static_cast<uint64_t>(timeout_ns));
   if (cudaGetLastError() != cudaSuccess) return GEMM_ERR_LAUNCH;
   return read_and_clear_status(d, stream, device_status);
+}
+
+int gemm_read_probe(const void* src, int64_t n_bytes, void* sink, gemm_stream_t stream) {
+  if (n_bytes < 0 || (n_bytes & 15) != 0 || sink == nullptr) return GEMM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(src) & 15) != 0 || (reinterpret_cast<uintptr_t>(sink) & 3) != 0)
+    return GEMM_ERR_ALIGNMENT;
+  DeviceCtx d;
+  int rc = get_device(&d);
+  if (rc != GEMM_OK) return rc;
+  load_entry_points();
+  // the sink: one 4-byte word; the source: n_bytes as one row
+  if (query_pointer(sink, d.device, 1, 2, 2) != 1) return GEMM_ERR_INVALID_ARG;
+  if (n_bytes > 0 && query_pointer(src, d.device, 1, n_bytes / 2, n_bytes / 2) != 1)
+    return GEMM_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(sink, 0, sizeof(unsigned), stream) != cudaSuccess) return GEMM_ERR_LAUNCH;
+  if (n_bytes == 0) return GEMM_OK;
+  const int grid = 4 * d.sm_count;  // 4 blocks of 512 threads fill an SM's 2048 threads
+  read_probe_kernel<<<grid, 512, 0, stream>>>(static_cast<const uint4*>(src), n_bytes / 16,
+                                               static_cast<unsigned*>(sink));
+  return cudaGetLastError() == cudaSuccess ? GEMM_OK : GEMM_ERR_LAUNCH;
 }
 
 }  // extern "C"

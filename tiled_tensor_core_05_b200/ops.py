@@ -66,6 +66,8 @@ _SIGNATURES = {
                              ctypes.c_void_p], ctypes.c_int),
     "gemm_relu_f16_noalloc": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
                               ctypes.c_int),
+    "gemm_read_probe": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p],
+                        ctypes.c_int),
 }
 
 
@@ -304,3 +306,18 @@ def selftest_wait_timeout(timeout_ns: int, stream=None, device=None) -> int:
                                                 ctypes.byref(st)),
                "gemm_selftest_wait_timeout")
     return int(st.value)
+
+
+def read_probe(buf: torch.Tensor, sink: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Stream-read every byte of the contiguous CUDA tensor ``buf`` once (the
+    library's read-bandwidth probe); returns the 1-element int32 ``sink``
+    holding the XOR of its 32-bit words."""
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise ValueError("buf must be a contiguous CUDA tensor")
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
+    n = buf.numel() * buf.element_size()
+    with torch.cuda.device(buf.device):
+        _check(lib().gemm_read_probe(buf.data_ptr(), n, sink.data_ptr(),
+                                     _stream_handle(stream, buf.device)), "gemm_read_probe")
+    return sink
