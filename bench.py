@@ -24,6 +24,7 @@ import datetime
 import hashlib
 import json
 import os
+import statistics
 import sys
 import time
 
@@ -201,7 +202,7 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
     st = ops.device_status()
     if st != 0:
         raise RuntimeError(f"device reported status {st:#x}")
-    res = {"total_ms": total_ms, "launch_ms": launch_ms, "w": w}
+    res = {"total_ms": total_ms, "launch_ms": launch_ms, "w": w, "step": step}
     if comparator:
         # context only, never on the measured path: cuBLAS through torch on
         # the same inputs, timed the same way right after our kernel
@@ -279,6 +280,50 @@ def oracle_seconds_per_row(oracle, a, b) -> float:
     t0 = time.perf_counter()
     oracle.gemm_relu(a[:rows], b)
     return max(time.perf_counter() - t0, 1e-6) / rows
+
+
+def launch_stats(step, n: int = 50):
+    """Median and best of `n` launches, each between its own pair of CUDA
+    events on the launching stream (outside the timed region; context)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    per = sorted(a.elapsed_time(b) for a, b in zip(starts, ends))
+    return {"launches": n, "median_ms": round(statistics.median(per), 5),
+            "best_ms": round(per[0], 5),
+            "note": "each launch between its own events, after the timed region"}
+
+
+def sustained_run(step, launch_ms: float, seconds: float, gpu_uuid: str):
+    """Back-to-back launches for about `seconds` (after the timed region), with
+    the SM clock and throttle reasons sampled meanwhile: the rate under the
+    power cap rather than in a burst."""
+    import torch
+    n = max(10, int(seconds * 1e3 / max(launch_ms, 1e-3)))
+    sampler = ClockSampler(gpu_uuid)
+    sampler.wait_first()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    sampler.mark("t0")
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("t1")
+    sampler.stop()
+    total = e0.elapsed_time(e1)
+    return {"launches": n, "seconds": round(total / 1e3, 2), "ms_per_launch": round(total / n, 5),
+            "clocks": sampler.summary()}
 
 
 def stream_read_probe(gib: float = 2.0, steps: int = 20):
@@ -466,6 +511,16 @@ def run_ours(args):
                 value / world if unit == "GB/s" else None)
             if gbs:
                 entry["frac_of_read_probe"] = round(gbs / probe["gbs"], 4)
+    if rank == 0 and args.sustained_seconds > 0:
+        line["launch_stats"] = launch_stats(main["step"])
+        sus = sustained_run(main["step"], main["launch_ms"], args.sustained_seconds,
+                            gpu_id_for(local))
+        rate = (w.bytes_min / (sus["ms_per_launch"] * 1e-3) / 1e9 if unit == "GB/s"
+                else w.flops / (sus["ms_per_launch"] * 1e-3) / 1e12)
+        sus["value"] = round(rate, 2)
+        sus["unit"] = unit
+        sus["note"] = "one GPU, back to back after the timed region (context, not the value)"
+        line["sustained"] = sus
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget)
     if dist is not None:
@@ -486,6 +541,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="cube8192")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--sustained-seconds", type=float, default=2.0,
+                    help="length of the back-to-back context run after the timed region "
+                         "(0: skip it and the per-launch statistics)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", type=int, default=0,
                     help="kernel for the main workload: 0 = chosen by shape (gemm_relu_f16), "

@@ -32,18 +32,27 @@ namespace {
 constexpr int kBM = 128;        // tile rows (MMA M)
 constexpr int kBK = 64;         // k-block: 64 fp16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
-constexpr int kThreads = 192;   // 6 warps
-constexpr int kEpiWarps = 4;
+#ifndef TTC_EPI_WARPS
+#define TTC_EPI_WARPS 4
+#endif
+// Epilogue warps: 4 (one per TMEM lane quarter) or 8 (two per quarter, each
+// taking half of the tile's columns).
+constexpr int kEpiWarps = TTC_EPI_WARPS;
+static_assert(kEpiWarps == 4 || kEpiWarps == 8, "epilogue warps");
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
+constexpr int kEpiGroups = kEpiWarps / 4;      // column groups of a tile
+constexpr int kEpiBoxes = 8 / kEpiWarps;       // staging boxes per warp: 32 KiB in all
 constexpr int kEpiRows = 32;    // rows per epilogue warp
 constexpr int kEpiCols = 64;    // columns per epilogue chunk (128 bytes of fp16)
 constexpr int kEpiBuf = kEpiRows * kEpiCols * 2;
 
 // Dynamic shared memory of a tile kernel: 1 KiB of alignment slack, the
-// operand ring, two 32 x 64 fp16 staging boxes per epilogue warp, the
+// operand ring, eight 32 x 64 fp16 staging boxes for the epilogue warps, the
 // mbarriers (full and empty per stage, two accumulator handshakes per
 // buffer, one spare) and the TMEM address slot.
 constexpr int tile_smem_formula(int stage_bytes, int stages) {
-  return 1024 + stages * stage_bytes + kEpiWarps * 2 * kEpiBuf + (2 * stages + 5) * 8 + 16;
+  return 1024 + stages * stage_bytes + kEpiWarps * kEpiBoxes * kEpiBuf + (2 * stages + 5) * 8 +
+         16;
 }
 // One ring stage: A (128 rows x 64 k) and B (64 k x bn columns) ...
 constexpr int single_stage_bytes(int bn) { return kBM * kBK * 2 + kBK * bn * 2; }
@@ -56,7 +65,7 @@ struct TileCfg {
   static constexpr int kBChunk = kBK * 64 * 2;  // one 64-column slab of the B tile
   static constexpr int kBBytes = kBK * BN * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiBuf;
+  static constexpr int kEpiBytes = kEpiWarps * kEpiBoxes * kEpiBuf;
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
   static constexpr uint32_t kTmemCols = 2 * BN;
@@ -83,7 +92,7 @@ struct PairCfg {
   static constexpr int kBChunk = kBK * 64 * 2;
   static constexpr int kBBytes = kBK * 128 * 2;           // this CTA's 128 columns
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiBuf;
+  static constexpr int kEpiBytes = kEpiWarps * kEpiBoxes * kEpiBuf;
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
   static constexpr int kNBuf = SLABS == 1 ? 2 : 1;        // accumulator buffers
@@ -153,21 +162,21 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
   nb = r / rows;
 }
 
-// Epilogue of one accumulator tile, run by one warp for its 32 TMEM lanes:
-// tcgen05.ld 64 columns at a time -> ReLU in fp32 -> RNE to fp16 -> 128-byte
-// swizzled staging row per thread -> TMA store of a 32 x 64 box (double
-// buffered per warp).  Columns at and beyond N rounded down to 8 (the TMA
+// Epilogue of one accumulator tile, run by one warp for its 32 TMEM lanes and
+// COLS of the tile's columns: tcgen05.ld 64 columns at a time -> bias and
+// activation in fp32 -> RNE to fp16 -> 128-byte swizzled staging row per
+// thread -> TMA store of a 32 x 64 box (kEpiBoxes boxes per warp in turn).  Columns at and beyond N rounded down to 8 (the TMA
 // store writes whole 16-byte groups) are written with plain stores.
 // `release()` runs once the last TMEM load of the tile has completed.
 // `bias` (N fp16 values or null) is added per column before the activation.
-template <int BN, int ACT, class Release>
+template <int COLS, int ACT, class Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uint32_t& chunk_no,
                                               const CUtensorMap* tmC, __half* C, int64_t ldc,
                                               const __half* __restrict__ bias, int M, int N,
                                               int n8, int row0, int col_base, int lane,
                                               Release release) {
 #pragma unroll 1
-  for (int c = 0; c < BN / kEpiCols; ++c) {
+  for (int c = 0; c < COLS / kEpiCols; ++c) {
     // the 64 bias values of this chunk as 32 packed pairs (0 past N)
     uint32_t bb[32];
     if (bias != nullptr) {
@@ -185,7 +194,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
     }
     uint32_t v[64];
     tmem_load_32x32b_x64(t_row + c * kEpiCols, v);
-    if (c == BN / kEpiCols - 1) {
+    if (c == COLS / kEpiCols - 1) {
       // the accumulator has been read: hand it back to the MMA issuer
       tc_fence_before_sync();
       __syncwarp();
@@ -207,8 +216,9 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
       h[i] = pack_half2(activate<ACT>(x0), activate<ACT>(x1));
       h[16 + i] = pack_half2(activate<ACT>(y0), activate<ACT>(y1));
     }
-    uint8_t* buf = bufs + (chunk_no & 1u) * kEpiBuf;
-    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+    uint8_t* buf = bufs + (chunk_no % kEpiBoxes) * kEpiBuf;
+    // the store that last used `buf` has read it
+    if (lane == 0) bulk_wait_group_read<kEpiBoxes - 1>();
     __syncwarp();
     // row `lane`, 128 bytes = 8 chunks of 16 bytes, chunk j stored at j ^ (row & 7)
     const uint32_t row_addr = smem_u32(buf) + lane * 128;
@@ -407,7 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue ---
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint8_t* bufs = smEpi + (warp - 2) * 2 * kEpiBuf;
+    const int ew = warp - 2;
+    constexpr int kCols = BN / kEpiGroups;  // columns of the tile this warp drains
+    const int g = ew >> 2;                  // its column group
+    uint8_t* bufs = smEpi + ew * kEpiBoxes * kEpiBuf;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk_no = 0;
@@ -425,10 +438,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after_sync();
       const int row0 = mb * kBM + q * kEpiRows;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
+                             static_cast<uint32_t>(acc * BN + g * kCols);
       uint64_t* release_bar = &acc_empty[acc];
-      epilogue_tile<BN, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
-                             nb * BN, lane, [release_bar] { mbar_arrive(release_bar); });
+      epilogue_tile<kCols, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
+                                nb * BN + g * kCols, lane,
+                                [release_bar] { mbar_arrive(release_bar); });
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -648,7 +662,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------ epilogue (both CTAs) ---
     const int q = warp & 3;
-    uint8_t* bufs = smEpi + (warp - 2) * 2 * kEpiBuf;
+    const int ew = warp - 2;
+    constexpr int kCols = BN / kEpiGroups;
+    const int g = ew >> 2;
+    uint8_t* bufs = smEpi + ew * kEpiBoxes * kEpiBuf;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk_no = 0;
@@ -670,13 +687,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row0 =
             mb * Cfg::kTileM + s * 2 * kBM + static_cast<int>(rank) * kBM + q * kEpiRows;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>((acc * SLABS + s) * BN);
+                               static_cast<uint32_t>((acc * SLABS + s) * BN + g * kCols);
         const bool last = (s == SLABS - 1);
         // the accumulator buffer is handed back after its last slab is read
-        epilogue_tile<BN, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
-                               nb * BN, lane, [release_bar, last] {
-                                 if (last) mbar_arrive_cluster(release_bar);
-                               });
+        epilogue_tile<kCols, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
+                                  nb * BN + g * kCols, lane, [release_bar, last] {
+                                    if (last) mbar_arrive_cluster(release_bar);
+                                  });
       }
       if (++acc == NBUF) {
         acc = 0;
