@@ -298,7 +298,9 @@ def launch_stats(step, n: int = 50):
     per = sorted(a.elapsed_time(b) for a, b in zip(starts, ends))
     return {"launches": n, "median_ms": round(statistics.median(per), 5),
             "best_ms": round(per[0], 5),
-            "note": "each launch between its own events, after the timed region"}
+            "note": "each launch between its own events, after the timed region; for a "
+                    "kernel shorter than the host's time per call the GPU waits for the "
+                    "launch inside the events, so the figure is the host's rate"}
 
 
 def sustained_run(step, launch_ms: float, seconds: float, gpu_uuid: str):
