@@ -202,7 +202,9 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
     st = ops.device_status()
     if st != 0:
         raise RuntimeError(f"device reported status {st:#x}")
-    res = {"total_ms": total_ms, "launch_ms": launch_ms, "w": w, "step": step}
+    # `step` holds raw pointers: keep the tensors alive as long as it is
+    res = {"total_ms": total_ms, "launch_ms": launch_ms, "w": w, "step": step,
+           "tensors": (a, b, c, bias)}
     if comparator:
         # context only, never on the measured path: cuBLAS through torch on
         # the same inputs, timed the same way right after our kernel

@@ -14,10 +14,11 @@
 //     A (128 x 64) and B (64 x BN) tiles, with mbarrier full/empty handshakes;
 //   * warp 1: allocates TMEM and issues tcgen05.mma (128 x BN x 16) from one
 //     thread into a double-buffered fp32 accumulator in TMEM;
-//   * warps 2-5: epilogue.  tcgen05.ld -> ReLU in fp32 -> RNE to fp16 ->
-//     swizzled shared-memory staging -> TMA store, which clips rows/columns
-//     beyond M/N (ragged edges).  The epilogue of tile i overlaps the
-//     main loop of tile i+1 thanks to the second accumulator.
+//   * warps 2-5 (2-9 for the 512-row pair tile): epilogue.  tcgen05.ld ->
+//     bias and activation in fp32 -> RNE to fp16 -> swizzled shared-memory
+//     staging -> TMA store, which clips rows/columns beyond M/N (ragged
+//     edges).  With a second accumulator the epilogue of tile i overlaps the
+//     main loop of tile i+1.
 // Out-of-range A/B elements (M, N or K not a multiple of the tile) are
 // zero-filled by TMA and so contribute nothing to the sum.
 #include <atomic>
@@ -32,16 +33,12 @@ namespace {
 constexpr int kBM = 128;        // tile rows (MMA M)
 constexpr int kBK = 64;         // k-block: 64 fp16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
-#ifndef TTC_EPI_WARPS
-#define TTC_EPI_WARPS 4
-#endif
-// Epilogue warps: 4 (one per TMEM lane quarter) or 8 (two per quarter, each
-// taking half of the tile's columns).
-constexpr int kEpiWarps = TTC_EPI_WARPS;
-static_assert(kEpiWarps == 4 || kEpiWarps == 8, "epilogue warps");
-constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
-constexpr int kEpiGroups = kEpiWarps / 4;      // column groups of a tile
-constexpr int kEpiBoxes = 8 / kEpiWarps;       // staging boxes per warp: 32 KiB in all
+// Epilogue warps: 4 (one per TMEM lane quarter) where the epilogue of a tile
+// overlaps the next tile's main loop (double-buffered accumulators), 8 (two per
+// quarter, each draining half of the tile's columns) where it cannot (the
+// 512-row pair tile fills TMEM with one accumulator).  Either way eight 32 x 64
+// staging boxes (32 KiB): two per warp or one.
+constexpr int epi_threads(int epi_warps) { return 64 + 32 * epi_warps; }
 constexpr int kEpiRows = 32;    // rows per epilogue warp
 constexpr int kEpiCols = 64;    // columns per epilogue chunk (128 bytes of fp16)
 constexpr int kEpiBuf = kEpiRows * kEpiCols * 2;
@@ -50,9 +47,9 @@ constexpr int kEpiBuf = kEpiRows * kEpiCols * 2;
 // operand ring, eight 32 x 64 fp16 staging boxes for the epilogue warps, the
 // mbarriers (full and empty per stage, two accumulator handshakes per
 // buffer, one spare) and the TMEM address slot.
+constexpr int kEpiStaging = 8 * kEpiBuf;  // all staging boxes of a CTA
 constexpr int tile_smem_formula(int stage_bytes, int stages) {
-  return 1024 + stages * stage_bytes + kEpiWarps * kEpiBoxes * kEpiBuf + (2 * stages + 5) * 8 +
-         16;
+  return 1024 + stages * stage_bytes + kEpiStaging + (2 * stages + 5) * 8 + 16;
 }
 // One ring stage: A (128 rows x 64 k) and B (64 k x bn columns) ...
 constexpr int single_stage_bytes(int bn) { return kBM * kBK * 2 + kBK * bn * 2; }
@@ -61,11 +58,14 @@ constexpr int pair_stage_bytes(int slabs) { return slabs * kBM * kBK * 2 + kBK *
 
 template <int BN, int STAGES>
 struct TileCfg {
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kThreads = epi_threads(kEpiWarps);
+  static constexpr int kEpiBoxes = 8 / kEpiWarps;
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBChunk = kBK * 64 * 2;  // one 64-column slab of the B tile
   static constexpr int kBBytes = kBK * BN * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kEpiBytes = kEpiWarps * kEpiBoxes * kEpiBuf;
+  static constexpr int kEpiBytes = kEpiStaging;
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
   static constexpr uint32_t kTmemCols = 2 * BN;
@@ -85,6 +85,9 @@ struct TileCfg {
 // staged per MAC, the epilogue not overlapped).
 template <int STAGES, int SLABS>
 struct PairCfg {
+  static constexpr int kEpiWarps = SLABS == 2 ? 8 : 4;
+  static constexpr int kThreads = epi_threads(kEpiWarps);
+  static constexpr int kEpiBoxes = 8 / kEpiWarps;
   static constexpr int kBN = 256;                         // pair tile columns
   static constexpr int kTileM = 2 * kBM * SLABS;          // pair tile rows
   static constexpr int kSlabBytes = kBM * kBK * 2;        // 128 rows of A, 64 k
@@ -92,7 +95,7 @@ struct PairCfg {
   static constexpr int kBChunk = kBK * 64 * 2;
   static constexpr int kBBytes = kBK * 128 * 2;           // this CTA's 128 columns
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kEpiBytes = kEpiWarps * kEpiBoxes * kEpiBuf;
+  static constexpr int kEpiBytes = kEpiStaging;
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
   static constexpr int kNBuf = SLABS == 1 ? 2 : 1;        // accumulator buffers
@@ -165,11 +168,11 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
 // Epilogue of one accumulator tile, run by one warp for its 32 TMEM lanes and
 // COLS of the tile's columns: tcgen05.ld 64 columns at a time -> bias and
 // activation in fp32 -> RNE to fp16 -> 128-byte swizzled staging row per
-// thread -> TMA store of a 32 x 64 box (kEpiBoxes boxes per warp in turn).  Columns at and beyond N rounded down to 8 (the TMA
+// thread -> TMA store of a 32 x 64 box (BOXES boxes per warp in turn).  Columns at and beyond N rounded down to 8 (the TMA
 // store writes whole 16-byte groups) are written with plain stores.
 // `release()` runs once the last TMEM load of the tile has completed.
 // `bias` (N fp16 values or null) is added per column before the activation.
-template <int COLS, int ACT, class Release>
+template <int COLS, int BOXES, int ACT, class Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uint32_t& chunk_no,
                                               const CUtensorMap* tmC, __half* C, int64_t ldc,
                                               const __half* __restrict__ bias, int M, int N,
@@ -216,9 +219,9 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
       h[i] = pack_half2(activate<ACT>(x0), activate<ACT>(x1));
       h[16 + i] = pack_half2(activate<ACT>(y0), activate<ACT>(y1));
     }
-    uint8_t* buf = bufs + (chunk_no % kEpiBoxes) * kEpiBuf;
+    uint8_t* buf = bufs + (chunk_no % BOXES) * kEpiBuf;
     // the store that last used `buf` has read it
-    if (lane == 0) bulk_wait_group_read<kEpiBoxes - 1>();
+    if (lane == 0) bulk_wait_group_read<BOXES - 1>();
     __syncwarp();
     // row `lane`, 128 bytes = 8 chunks of 16 bytes, chunk j stored at j ^ (row & 7)
     const uint32_t row_addr = smem_u32(buf) + lane * 128;
@@ -251,7 +254,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
 }
 
 template <int BN, int STAGES, int ACT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(TileCfg<BN, STAGES>::kThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
@@ -292,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEpiWarps);
+      mbar_init(&acc_empty[b], Cfg::kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -418,9 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue ---
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int ew = warp - 2;
-    constexpr int kCols = BN / kEpiGroups;  // columns of the tile this warp drains
+    constexpr int kCols = BN * 4 / Cfg::kEpiWarps;  // columns of the tile this warp drains
     const int g = ew >> 2;                  // its column group
-    uint8_t* bufs = smEpi + ew * kEpiBoxes * kEpiBuf;
+    uint8_t* bufs = smEpi + ew * Cfg::kEpiBoxes * kEpiBuf;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk_no = 0;
@@ -440,9 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + g * kCols);
       uint64_t* release_bar = &acc_empty[acc];
-      epilogue_tile<kCols, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
-                                nb * BN + g * kCols, lane,
-                                [release_bar] { mbar_arrive(release_bar); });
+      epilogue_tile<kCols, Cfg::kEpiBoxes, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N,
+                                                n8, row0, nb * BN + g * kCols, lane,
+                                                [release_bar] { mbar_arrive(release_bar); });
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -473,10 +476,11 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 //     both halves);
 //   * the leader's commit frees stage s in both CTAs and tells both epilogues
 //     that an accumulator is ready (multicast arrive);
-//   * each CTA's four epilogue warps drain its own TMEM rows and arrive on the
-//     leader's acc_empty barrier (8 arrivals per accumulator use).
+//   * each CTA's epilogue warps (4, or 8 for the 512-row tile) drain its own
+//     TMEM rows and arrive on the leader's acc_empty barrier (one arrival per
+//     warp of both CTAs per accumulator use).
 template <int STAGES, int SLABS, int ACT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
     tile_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
@@ -520,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 2 * kEpiWarps);
+      mbar_init(&acc_empty[b], 2 * Cfg::kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -663,9 +667,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ epilogue (both CTAs) ---
     const int q = warp & 3;
     const int ew = warp - 2;
-    constexpr int kCols = BN / kEpiGroups;
+    constexpr int kCols = BN * 4 / Cfg::kEpiWarps;
     const int g = ew >> 2;
-    uint8_t* bufs = smEpi + ew * kEpiBoxes * kEpiBuf;
+    uint8_t* bufs = smEpi + ew * Cfg::kEpiBoxes * kEpiBuf;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk_no = 0;
@@ -690,10 +694,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                static_cast<uint32_t>((acc * SLABS + s) * BN + g * kCols);
         const bool last = (s == SLABS - 1);
         // the accumulator buffer is handed back after its last slab is read
-        epilogue_tile<kCols, ACT>(t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0,
-                                  nb * BN + g * kCols, lane, [release_bar, last] {
-                                    if (last) mbar_arrive_cluster(release_bar);
-                                  });
+        epilogue_tile<kCols, Cfg::kEpiBoxes, ACT>(
+            t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0, nb * BN + g * kCols, lane,
+            [release_bar, last] {
+              if (last) mbar_arrive_cluster(release_bar);
+            });
       }
       if (++acc == NBUF) {
         acc = 0;
@@ -767,7 +772,7 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = p.stream;
   cfg.attrs = attr;
@@ -799,7 +804,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = p.stream;
   cfg.attrs = attr;
