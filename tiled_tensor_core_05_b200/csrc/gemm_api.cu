@@ -362,21 +362,21 @@ double wave_efficiency(int64_t tiles, int64_t pairs) {
 }
 
 // The kernel chosen for a shape on a GPU with `sm_count` SMs.  The 512 x 256
-// pair tile stages 25 % fewer bytes per MAC than the 256 x 256 one and, under
-// the 1000 W power cap, runs at a higher clock (measured: 8192^3 1262 against
-// 1173 TFLOP/s sustained, 1390 against 1280 in short runs; the MLP
-// up-projection 1330 against 1290 despite 93 % against 97 % wave efficiency);
-// it is taken unless its last wave wastes more than 6 points more.
-// GELU makes the epilogue expensive enough that hiding it behind the next
-// tile's main loop (the double-buffered 256 x 256 pair tile) wins: the MLP
-// up-projection with bias + GELU took 1.08 ms on the 512-row tile.
-int select_path_for(int64_t M, int64_t N, int sm_count, int activation) {
+// pair tile stages 25 % fewer bytes per MAC than the 256 x 256 one, but its
+// single accumulator leaves each tile's epilogue exposed, which costs more
+// the shorter the main loop.  Measured on an 8192 x 8192 output, ReLU and
+// bias + GELU alike (time of the 512-row tile / time of the 256-row tile):
+// K = 2048 1.03 / 1.01, K = 4096 0.98, K = 6144 0.96, K = 8192 0.94,
+// K = 12288 0.92.  So the 512-row tile is taken for K >= 3072 unless its last
+// wave wastes more than 6 points more of the SM pairs than the 256-row
+// tiling's (the MLP up-projection: 93 % against 97 %, still faster).
+int select_path_for(int64_t M, int64_t N, int64_t K, int sm_count) {
   if (M >= 1 && M <= 64) return GEMM_PATH_SKINNY;
   const int64_t pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
   const int64_t col_tiles = (N + 255) / 256;
   const int64_t tiles256 = ((M + 255) / 256) * col_tiles;
   if (tiles256 < 64) return GEMM_PATH_TILE;
-  if (activation == GEMM_ACT_GELU) return GEMM_PATH_TILE_PAIR;
+  if (K < 3072) return GEMM_PATH_TILE_PAIR;
   const int64_t tiles512 = ((M + 511) / 512) * col_tiles;
   return wave_efficiency(tiles512, pairs) >= wave_efficiency(tiles256, pairs) - 0.06
              ? GEMM_PATH_TILE_PAIR_TALL
@@ -453,7 +453,7 @@ int run_gemm(const void* A, const void* B, const void* bias, void* C, int64_t M,
     rc = resolve_config(kc, M, N, d.sm_count);
     if (rc != GEMM_OK) return rc;
   } else {
-    if (path == GEMM_PATH_AUTO) path = select_path_for(M, N, d.sm_count, activation);
+    if (path == GEMM_PATH_AUTO) path = select_path_for(M, N, K, d.sm_count);
     kc = KernelConfig{path, 0, 0, 0, 0};
     if (resolve_config(kc, M, N, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
   }
@@ -490,8 +490,7 @@ int run_gemm(const void* A, const void* B, const void* bias, void* C, int64_t M,
 }  // namespace ttc
 
 int gemm_select_path(int64_t M, int64_t N, int64_t K) {
-  (void)K;
-  return select_path_for(M, N, 148, GEMM_ACT_RELU);  // a B200 has 148 SMs
+  return select_path_for(M, N, K, 148);  // a B200 has 148 SMs
 }
 
 const char* gemm_status_string(int status) {
@@ -558,7 +557,7 @@ int gemm_auto_config(int64_t M, int64_t N, int64_t K, int activation, gemm_confi
   DeviceCtx d;
   const int rc = get_device(&d);
   if (rc != GEMM_OK) return rc;
-  KernelConfig c{select_path_for(M, N, d.sm_count, activation), 0, 0, 0, 0};
+  KernelConfig c{select_path_for(M, N, K, d.sm_count), 0, 0, 0, 0};
   if (resolve_config(c, M, N, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
   *out = gemm_config{c.kernel, c.block_n, c.stages, c.group_rows, c.splits};
   return GEMM_OK;
