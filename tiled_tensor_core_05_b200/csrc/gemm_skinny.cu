@@ -96,11 +96,10 @@ __device__ __forceinline__ void store_column(const float (&v)[MP], __half* C, in
   if (n >= N) return;
   const float b = bias != nullptr ? __half2float(bias[n]) : 0.0f;
 #pragma unroll
-  for (int m = 0; m < MP; ++m) {
-    if (m < M) {
-      const float x = activate<ACT>(v[m] + b);
-      C[static_cast<int64_t>(m) * ldc + n] = __float2half_rn(x);
-    }
+  for (int m = 0; m < MP; m += 2) {
+    const float2 x = activate2<ACT>(__fadd2_rn(make_float2(v[m], v[m + 1]), splat2(b)));
+    if (m < M) C[static_cast<int64_t>(m) * ldc + n] = __float2half_rn(x.x);
+    if (m + 1 < M) C[static_cast<int64_t>(m + 1) * ldc + n] = __float2half_rn(x.y);
   }
 }
 

@@ -206,18 +206,17 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
     uint32_t h[32];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
-      float y0 = __uint_as_float(v[32 + 2 * i]), y1 = __uint_as_float(v[32 + 2 * i + 1]);
+      // columns 2i, 2i + 1 and 32 + 2i, 32 + 2i + 1 of the chunk, in pairs
+      float2 xv = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+      float2 yv = make_float2(__uint_as_float(v[32 + 2 * i]), __uint_as_float(v[32 + 2 * i + 1]));
       if (bias != nullptr) {
-        const float2 bx = __half22float2(*reinterpret_cast<const __half2*>(&bb[i]));
-        const float2 by = __half22float2(*reinterpret_cast<const __half2*>(&bb[16 + i]));
-        x0 += bx.x;
-        x1 += bx.y;
-        y0 += by.x;
-        y1 += by.y;
+        xv = __fadd2_rn(xv, __half22float2(*reinterpret_cast<const __half2*>(&bb[i])));
+        yv = __fadd2_rn(yv, __half22float2(*reinterpret_cast<const __half2*>(&bb[16 + i])));
       }
-      h[i] = pack_half2(activate<ACT>(x0), activate<ACT>(x1));
-      h[16 + i] = pack_half2(activate<ACT>(y0), activate<ACT>(y1));
+      xv = activate2<ACT>(xv);
+      yv = activate2<ACT>(yv);
+      h[i] = pack_half2(xv.x, xv.y);
+      h[16 + i] = pack_half2(yv.x, yv.y);
     }
     uint8_t* buf = bufs + (chunk_no % BOXES) * kEpiBuf;
     // the store that last used `buf` has read it

@@ -323,32 +323,51 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 // max(x, 0) that maps -0 and NaN to +0.
 __device__ __forceinline__ float relu_f32(float x) { return x > 0.0f ? x : 0.0f; }
 
-// Standard normal CDF Phi(x) = (1 + erf(x / sqrt 2)) / 2, with erf from
-// Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
+// GELU(x) = x Phi(x), Phi(x) = (1 + erf(x / sqrt 2)) / 2 the standard normal
+// CDF, with erf from Abramowitz & Stegun, Handbook of Mathematical Functions,
+// formula 7.1.26:
 //   erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),
 //   t = 1 / (1 + p z), z >= 0, |error| <= 1.5e-7,
 //   p = 0.3275911, a1..a5 = 0.254829592, -0.284496736, 1.421413741,
 //   -1.453152027, 1.061405429.
-// For x < 0, Phi(x) = (1 - erf(|z|)) / 2 is the tail term itself, so no
-// cancellation occurs; |Phi error| <= 0.75e-7 everywhere.
+// With z = |x| / sqrt 2, Phi(-|x|) = (1 - erf(z)) / 2 is the tail term itself
+// (no cancellation) and Phi(|x|) = 1 - Phi(-|x|); |Phi error| <= 0.75e-7.
+// Evaluated two values at a time with the packed fp32 arithmetic of sm_100
+// (fma / mul .f32x2), in the variable u = z sqrt(log2 e), so that
+// exp(-z^2) = 2^(-u^2) is one ex2.approx and 1 + p z = 1 + (p / sqrt(log2 e)) u;
+// the 1/2 of Phi is folded into a1..a5.  Every epilogue, and the scalar form
+// below, evaluates exactly these steps, so all give the same bits.
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
 
-__device__ __forceinline__ float normal_cdf(float x) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  // 1 + p z >= 1: the one-instruction approximate reciprocal (relative error
-  // ~1 ulp) is far inside the formula's 1.5e-7 budget
-  const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  poly *= t;
-  const float tail = 0.5f * poly * __expf(-z * z);  // (1 - erf(z)) / 2
-  return x < 0.0f ? tail : 1.0f - tail;
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+__device__ __forceinline__ float2 gelu2(float2 x) {
+  constexpr float kU = 0.8493218002880191f;  // sqrt(1/2) sqrt(log2 e)
+  constexpr float kP = 0.2727374808792225f;  // p / sqrt(log2 e)
+  const float2 u = __fmul2_rn(make_float2(fabsf(x.x), fabsf(x.y)), splat2(kU));
+  const float2 d = __ffma2_rn(u, splat2(kP), splat2(1.0f));  // 1 + p z >= 1
+  // the approximate reciprocal (about 1 ulp) is far inside the 1.5e-7 budget
+  const float2 t = make_float2(rcp_approx(d.x), rcp_approx(d.y));
+  float2 q = __ffma2_rn(splat2(0.5307027145f), t, splat2(-0.7265760135f));  // a5 / 2, a4 / 2
+  q = __ffma2_rn(q, t, splat2(0.7107068705f));                               // a3 / 2
+  q = __ffma2_rn(q, t, splat2(-0.142248368f));                               // a2 / 2
+  q = __ffma2_rn(q, t, splat2(0.127414796f));                                // a1 / 2
+  q = __fmul2_rn(q, t);
+  const float2 w = __fmul2_rn(u, u);  // z^2 log2 e
+  const float2 tail = __fmul2_rn(q, make_float2(ex2_approx(-w.x), ex2_approx(-w.y)));
+  const float2 upper = __ffma2_rn(tail, splat2(-1.0f), splat2(1.0f));  // Phi(|x|)
+  const float2 phi = make_float2(x.x < 0.0f ? tail.x : upper.x, x.y < 0.0f ? tail.y : upper.y);
+  return __fmul2_rn(x, phi);
 }
 
 // Epilogue activations: kActRelu as above; kActGelu is x * Phi(x) (the exact
@@ -356,14 +375,19 @@ __device__ __forceinline__ float normal_cdf(float x) {
 enum : int { kActNone = 0, kActRelu = 1, kActGelu = 2 };
 
 template <int ACT>
-__device__ __forceinline__ float activate(float x) {
+__device__ __forceinline__ float2 activate2(float2 x) {
   if constexpr (ACT == kActRelu) {
-    return relu_f32(x);
+    return make_float2(relu_f32(x.x), relu_f32(x.y));
   } else if constexpr (ACT == kActGelu) {
-    return x * normal_cdf(x);
+    return gelu2(x);
   } else {
     return x;
   }
+}
+
+template <int ACT>
+__device__ __forceinline__ float activate(float x) {
+  return activate2<ACT>(make_float2(x, x)).x;
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
