@@ -70,9 +70,9 @@ enum gemm_status {
 
 enum gemm_path {
   GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY; fewer than 64 tiles of
-                              256 x 256 -> TILE; K < 3072 -> TILE_PAIR; otherwise
-                              TILE_PAIR_TALL, or TILE_PAIR when the 512-row tiles leave
-                              a much emptier last wave */
+                              256 x 256 -> TILE; K < 3072 (6144 with GELU) -> TILE_PAIR;
+                              otherwise TILE_PAIR_TALL, or TILE_PAIR when the 512-row
+                              tiles leave a much emptier last wave */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile (any shape) */
   GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 256 columns of B per CTA streamed
                               in lock-step, split-K only when tiles < SMs (M <= 64 only) */
@@ -183,9 +183,10 @@ GEMM_API int gemm_config_list(gemm_config* out, int capacity);
  * (invalid sizes or activation, no sm_100 device). */
 GEMM_API int gemm_auto_config(int64_t M, int64_t N, int64_t K, int activation, gemm_config* out);
 
-/* The path GEMM_PATH_AUTO takes for this shape on a 148-SM B200, whatever the
- * activation (pure host function; GEMM_PATH_AUTO itself uses the SM count of
- * the current device). */
+/* The path GEMM_PATH_AUTO takes for this shape with ReLU (or no activation)
+ * on a 148-SM B200 (pure host function; GEMM_PATH_AUTO itself uses the SM
+ * count of the current device, and with GELU keeps the 256-row pair tile up
+ * to K < 6144). */
 GEMM_API int gemm_select_path(int64_t M, int64_t N, int64_t K);
 
 /* Human-readable text for a gemm_status value (static storage). */

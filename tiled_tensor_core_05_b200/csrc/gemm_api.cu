@@ -364,19 +364,21 @@ double wave_efficiency(int64_t tiles, int64_t pairs) {
 // The kernel chosen for a shape on a GPU with `sm_count` SMs.  The 512 x 256
 // pair tile stages 25 % fewer bytes per MAC than the 256 x 256 one, but its
 // single accumulator leaves each tile's epilogue exposed, which costs more
-// the shorter the main loop.  Measured on an 8192 x 8192 output, ReLU and
-// bias + GELU alike (time of the 512-row tile / time of the 256-row tile):
-// K = 2048 1.03 / 1.01, K = 4096 0.98, K = 6144 0.96, K = 8192 0.94,
-// K = 12288 0.92.  So the 512-row tile is taken for K >= 3072 unless its last
+// the shorter the main loop and the heavier the epilogue.  Measured on an
+// 8192 x 8192 output (time of the 512-row tile / time of the 256-row tile):
+//   K            3072   4096   5120   6144   8192
+//   ReLU + bias  1.002  0.995  0.981  0.964  0.943
+//   GELU + bias  1.054  1.024  1.015  0.993  0.966
+// So the 512-row tile is taken from K = 3072 (6144 with GELU) unless its last
 // wave wastes more than 6 points more of the SM pairs than the 256-row
-// tiling's (the MLP up-projection: 93 % against 97 %, still faster).
-int select_path_for(int64_t M, int64_t N, int64_t K, int sm_count) {
+// tiling's (the MLP up-projection with ReLU: 93 % against 97 %, still faster).
+int select_path_for(int64_t M, int64_t N, int64_t K, int sm_count, int activation) {
   if (M >= 1 && M <= 64) return GEMM_PATH_SKINNY;
   const int64_t pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
   const int64_t col_tiles = (N + 255) / 256;
   const int64_t tiles256 = ((M + 255) / 256) * col_tiles;
   if (tiles256 < 64) return GEMM_PATH_TILE;
-  if (K < 3072) return GEMM_PATH_TILE_PAIR;
+  if (K < (activation == GEMM_ACT_GELU ? 6144 : 3072)) return GEMM_PATH_TILE_PAIR;
   const int64_t tiles512 = ((M + 511) / 512) * col_tiles;
   return wave_efficiency(tiles512, pairs) >= wave_efficiency(tiles256, pairs) - 0.06
              ? GEMM_PATH_TILE_PAIR_TALL
@@ -453,7 +455,7 @@ int run_gemm(const void* A, const void* B, const void* bias, void* C, int64_t M,
     rc = resolve_config(kc, M, N, d.sm_count);
     if (rc != GEMM_OK) return rc;
   } else {
-    if (path == GEMM_PATH_AUTO) path = select_path_for(M, N, K, d.sm_count);
+    if (path == GEMM_PATH_AUTO) path = select_path_for(M, N, K, d.sm_count, activation);
     kc = KernelConfig{path, 0, 0, 0, 0};
     if (resolve_config(kc, M, N, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
   }
@@ -490,7 +492,7 @@ int run_gemm(const void* A, const void* B, const void* bias, void* C, int64_t M,
 }  // namespace ttc
 
 int gemm_select_path(int64_t M, int64_t N, int64_t K) {
-  return select_path_for(M, N, K, 148);  // a B200 has 148 SMs
+  return select_path_for(M, N, K, 148, GEMM_ACT_RELU);  // a B200 has 148 SMs
 }
 
 const char* gemm_status_string(int status) {
@@ -557,7 +559,7 @@ int gemm_auto_config(int64_t M, int64_t N, int64_t K, int activation, gemm_confi
   DeviceCtx d;
   const int rc = get_device(&d);
   if (rc != GEMM_OK) return rc;
-  KernelConfig c{select_path_for(M, N, K, d.sm_count), 0, 0, 0, 0};
+  KernelConfig c{select_path_for(M, N, K, d.sm_count, activation), 0, 0, 0, 0};
   if (resolve_config(c, M, N, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
   *out = gemm_config{c.kernel, c.block_n, c.stages, c.group_rows, c.splits};
   return GEMM_OK;
