@@ -182,6 +182,41 @@ def test_workload_fullsize_sampled(oracle_mod, name):
     assert 0.45 < frac < 0.55, frac
 
 
+# --------------------------------------------------------- large extents ---
+
+@pytest.mark.slow
+@pytest.mark.parametrize("m,n,k,path", [
+    (3, 1 << 21, 16, SKINNY),       # 8192 column tiles of the small-M kernel
+    (64, 256, 1 << 20, SKINNY),     # one column tile, 16384 k-blocks in 4 slices
+    (70001, 72, 64, ops.PATH_AUTO),  # 274 pair row tiles, ragged M and N
+    (70001, 72, 64, TILE),          # 547 single-SM row tiles
+    (128, 128, 1 << 20, TILE),      # one tile, 16384 k-blocks
+    (128, 128, 1 << 20, PAIR),      # one pair tile (half of its rows past M)
+], ids=["skinny-wideN", "skinny-deepK", "auto-tallM", "tile-tallM", "tile-deepK",
+        "pair-deepK"])
+def test_large_extents(oracle_mod, m, n, k, path):
+    """Extents far beyond the workloads in one dimension: 64-bit offsets in
+    the epilogues, long k loops, long split-K slices and many tiles; A scaled
+    by 1/sqrt(K) so the sums stay of order 1 (fp32 accumulation keeps them
+    inside the tolerance at any K)."""
+    a_cpu, b_cpu = workloads.make_inputs(m, n, k, seed=k % 1000 + m, a_scale=1.0 / k ** 0.5)
+    a, b = a_cpu.cuda(), b_cpu.cuda()
+    c = torch.empty((m, n), dtype=torch.float16, device="cuda")
+    ops.gemm_f16_ex(a, b, c, relu=True, path=path)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    assert not torch.isnan(c).any() and (c >= 0).all()
+    rng = np.random.default_rng(m + n)
+    rows, cols = sample_points(m, n, rng, n_random=2048, rows=(0, m - 1), cols=(0, n - 1))
+    if len(rows) > 200_000:  # a whole row of the 2M-column case is plenty
+        keep = np.concatenate([np.arange(2048), 2048 + rng.choice(len(rows) - 2048, 100_000,
+                                                                    replace=False)])
+        rows, cols = rows[keep], cols[keep]
+    ref = oracle_mod.gemm_relu_at(a_cpu, b_cpu, rows, cols)
+    got = dev_to_np(c)[rows, cols]
+    check_parity(got, ref, True, f"{m}x{n}x{k} path {path}")
+
+
 # ------------------------------------------------------------ special cases ---
 
 @pytest.mark.parametrize("path", [ops.PATH_AUTO, TILE, PAIR, TALL])
