@@ -103,6 +103,22 @@ __device__ __forceinline__ void store_column(const float (&v)[MP], __half* C, in
   }
 }
 
+// Rows m0 .. m0 + 31 (those < M) of column n of C from 32 fp32 sums, as
+// store_column does for all MP rows.
+template <int ACT>
+__device__ __forceinline__ void store_rows(const float (&v)[32], __half* C, int M, int N,
+                                           int64_t ldc, int n, int m0, const __half* bias) {
+  if (n >= N) return;
+  const float b = bias != nullptr ? __half2float(bias[n]) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float2 x = activate2<ACT>(__fadd2_rn(make_float2(v[i], v[i + 1]), splat2(b)));
+    const int m = m0 + i;
+    if (m < M) C[static_cast<int64_t>(m) * ldc + n] = __float2half_rn(x.x);
+    if (m + 1 < M) C[static_cast<int64_t>(m + 1) * ldc + n] = __float2half_rn(x.y);
+  }
+}
+
 // MP fp32 accumulator columns of this thread's TMEM lane.
 template <int MP>
 __device__ __forceinline__ void load_accumulator(uint32_t taddr, float (&v)[MP]) {
@@ -313,29 +329,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar_sync(1, kEpiWarps * 32);
         if (*last_flag) {
           __threadfence();
+          // Sum the S partial tiles in slice order, 32 rows of C at a time;
+          // the loads of four slices are issued together before they are
+          // added, so the fix-up costs one L2 round trip per four slices
+          // rather than per slice (same sums in the same order: same bits).
+          // This slice's own partial is read back from TMEM at its turn.
+          const int64_t slice_stride = static_cast<int64_t>(kTW) * MP;
 #pragma unroll 1
           for (int h = 0; h < 2; ++h) {
-            float v[MP], acc[MP];
-            load_accumulator<MP>(t_lane + static_cast<uint32_t>(h * MP), v);
-            for (int sl = 0; sl < S; ++sl) {
-              if (sl == slice) {
+            const float* base =
+                partials + ((static_cast<int64_t>(tile) * S) * kTW + h * kSub + row) * MP;
+#pragma unroll 1
+            for (int mc = 0; mc < MP / 32; ++mc) {
+              float acc[32];
+#pragma unroll 1
+              for (int s0 = 0; s0 < S; s0 += 4) {
+                float4 buf[4][8];
 #pragma unroll
-                for (int m = 0; m < MP; ++m) acc[m] = (sl == 0) ? v[m] : acc[m] + v[m];
-              } else {
-                const float* src =
-                    partials + ((static_cast<int64_t>(tile) * S + sl) * kTW + h * kSub + row) * MP;
+                for (int g = 0; g < 4; ++g) {
+                  const int sl = s0 + g;
+                  if (sl < S && sl != slice) {
+                    const float* src = base + sl * slice_stride + mc * 32;
 #pragma unroll
-                for (int m = 0; m < MP; m += 4) {
-                  const float4 p = ld_cg_f4(src + m);
-                  if (sl == 0) {
-                    acc[m] = p.x; acc[m + 1] = p.y; acc[m + 2] = p.z; acc[m + 3] = p.w;
-                  } else {
-                    acc[m] += p.x; acc[m + 1] += p.y; acc[m + 2] += p.z; acc[m + 3] += p.w;
+                    for (int q = 0; q < 8; ++q) buf[g][q] = ld_cg_f4(src + 4 * q);
+                  }
+                }
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                  const int sl = s0 + g;
+                  if (sl < S) {
+                    float val[32];
+                    if (sl == slice) {
+                      uint32_t r[32];
+                      tmem_load_32x32b_x32(t_lane + static_cast<uint32_t>(h * MP + mc * 32), r);
+#pragma unroll
+                      for (int i = 0; i < 32; ++i) val[i] = __uint_as_float(r[i]);
+                    } else {
+#pragma unroll
+                      for (int q = 0; q < 8; ++q) {
+                        val[4 * q] = buf[g][q].x;
+                        val[4 * q + 1] = buf[g][q].y;
+                        val[4 * q + 2] = buf[g][q].z;
+                        val[4 * q + 3] = buf[g][q].w;
+                      }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] = (sl == 0) ? val[i] : acc[i] + val[i];
                   }
                 }
               }
+              store_rows<ACT>(acc, C, M, N, ldc, n0 + h * kSub, mc * 32, bias);
             }
-            store_column<MP, ACT>(acc, C, M, N, ldc, n0 + h * kSub, bias);
           }
         }
       }
