@@ -74,8 +74,9 @@ enum gemm_path {
                               otherwise TILE_PAIR_TALL, or TILE_PAIR when the 512-row
                               tiles leave a much emptier last wave */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile (any shape) */
-  GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 256 columns of B per CTA streamed
-                              in lock-step, split-K only when tiles < SMs (M <= 64 only) */
+  GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 256 (or, with few column tiles, 128)
+                              columns of B per CTA streamed in lock-step, split-K only when
+                              tiles < SMs (M <= 64 only) */
   GEMM_PATH_TILE_PAIR = 3, /* persistent kernel, two SMs (a CTA pair) per 256 x 256 tile
                               (any shape) */
   GEMM_PATH_TILE_PAIR_TALL = 4 /* persistent kernel, a CTA pair per 512 x 256 tile: fewer
@@ -143,14 +144,14 @@ GEMM_API int gemm_f16_general(const void* A, const void* B, const void* bias, vo
  * A field left at 0 takes the value GEMM_PATH_AUTO would use. */
 typedef struct gemm_config {
   int32_t kernel;     /* GEMM_PATH_TILE, _TILE_PAIR, _TILE_PAIR_TALL or _SKINNY (not AUTO) */
-  int32_t block_n;    /* output columns per tile: 128 or 256 for GEMM_PATH_TILE; 256 (the
-                         only width) for the other kernels */
+  int32_t block_n;    /* output columns per tile: 128 or 256 for GEMM_PATH_TILE and
+                         GEMM_PATH_SKINNY; 256 (the only width) for the pair kernels */
   int32_t stages;     /* depth of the shared-memory operand ring (k-blocks of 64 in flight) */
   int32_t group_rows; /* tile kernels: rows of op(A) per raster panel, the L2 grouping of
                          the tile order; 0 = 2048.  Must be 0 for GEMM_PATH_SKINNY */
-  int32_t splits;     /* GEMM_PATH_SKINNY: k-slices per 256-column tile, 1 <= splits <=
-                         ceil(K / 64) and splits * ceil(N / 256) <= the SM count when > 1;
-                         0 = chosen from the shape.  Must be 0 for the tile kernels */
+  int32_t splits;     /* GEMM_PATH_SKINNY: k-slices per column tile, 1 <= splits <=
+                         ceil(K / 64) and splits * ceil(N / block_n) <= the SM count when
+                         > 1; 0 = chosen from the shape.  Must be 0 for the tile kernels */
 } gemm_config;
 
 /* gemm_f16_general with the kernel configuration `cfg` instead of a path.
@@ -168,12 +169,14 @@ GEMM_API int gemm_f16_config(const void* A, const void* B, const void* bias, voi
 /* Dynamic shared memory per CTA (bytes) that the kernel, block_n and stages of
  * `cfg` need, whether or not that configuration is compiled (stages 0 = the
  * default).  A configuration fits a B200 when this is <= 232448.  Returns
- * GEMM_ERR_CONFIG when kernel / block_n name no kernel.  Pure host function. */
+ * GEMM_ERR_CONFIG when kernel / block_n name no kernel (block_n must be given
+ * for GEMM_PATH_TILE and GEMM_PATH_SKINNY).  Pure host function. */
 GEMM_API int gemm_config_smem_bytes(const gemm_config* cfg);
 
 /* The compiled configurations (kernel, block_n, stages; group_rows and
  * splits 0, free at call time): every stage count from 3 up to the shared
- * memory budget of each tile shape.  Writes up to `capacity` of them to `out`
+ * memory budget of each tile shape (up to 6 for the small-M kernel's
+ * streaming ring).  Writes up to `capacity` of them to `out`
  * (may be null when capacity is 0) and returns how many there are.  Pure host
  * function. */
 GEMM_API int gemm_config_list(gemm_config* out, int capacity);

@@ -90,7 +90,10 @@ def test_skinny_configs(oracle_mod, cfg, m):
     bias = rng.standard_normal(n).astype(np.float16)
     ref = oracle_mod.gemm_relu(a.numpy(), b.numpy())
     ref_g = oracle_mod.gemm_general(a, b, bias, "gelu")
-    for splits in (0, 1, 2, 3, 7, 32):
+    tiles = -(-n // cfg.block_n)
+    for splits in (0, 1, 2, 3, 7, 18, 32):
+        if splits > 1 and splits * tiles > torch.cuda.get_device_properties(0).multi_processor_count:
+            continue  # more (tile, slice) items than the split-K workspace holds
         d = dict(cfg.as_dict(), splits=splits)
         c = _run(a, b, d, m=m, n=n)
         check_parity(c, ref, True, f"{d} m={m}")
@@ -103,8 +106,9 @@ def test_skinny_splits_are_deterministic_and_agree():
     a, b = workloads.make_inputs(m, n, k, seed=45)
     outs = {}
     for s in (1, 2, 4, 8, 16, 64):
-        outs[s] = _run(a, b, {"kernel": ops.PATH_SKINNY, "splits": s}, m=m, n=n)
-        again = _run(a, b, {"kernel": ops.PATH_SKINNY, "splits": s}, m=m, n=n)
+        cfg = {"kernel": ops.PATH_SKINNY, "block_n": 256, "splits": s}
+        outs[s] = _run(a, b, cfg, m=m, n=n)
+        again = _run(a, b, cfg, m=m, n=n)
         assert (outs[s].view(np.uint16) == again.view(np.uint16)).all(), s
     # different slice counts sum in different orders: equal within fp32 rounding
     for s, o in outs.items():
@@ -158,7 +162,9 @@ def _raw(cfg, m=256, n=256, k=128, bias=False, act=ops.ACT_RELU):
     ({"kernel": ops.PATH_SKINNY}, 65),                     # M > 64
     ({"kernel": ops.PATH_SKINNY, "group_rows": 512}, 32),
     ({"kernel": ops.PATH_SKINNY, "splits": 3}, 32),        # 3 > 2 k-blocks
-    ({"kernel": ops.PATH_SKINNY, "stages": 6}, 32),
+    ({"kernel": ops.PATH_SKINNY, "block_n": 256, "stages": 6}, 32),  # over the budget
+    ({"kernel": ops.PATH_SKINNY, "block_n": 128, "stages": 7}, 32),  # past the depth cap
+    ({"kernel": ops.PATH_SKINNY, "block_n": 64}, 32),
     ({"kernel": ops.PATH_TILE, "stages": -1}, 256),
 ])
 def test_config_errors_launch_nothing(cfg, m):

@@ -17,15 +17,19 @@ def lib():
 
 def test_built_configs_are_exactly_those_within_the_budget(lib):
     built = {(c.kernel, c.block_n, c.stages) for c in ops.config_list()}
-    kinds = tune.TILE_KINDS + [(ops.PATH_SKINNY, 256)]
+    kinds = tune.TILE_KINDS + [(ops.PATH_SKINNY, w) for w in tune.SKINNY_WIDTHS]
     expect = set()
     for kernel, bn in kinds:
         for st in range(3, 17):
-            if ops.config_smem_bytes({"kernel": kernel, "block_n": bn, "stages": st}) <= BUDGET:
-                expect.add((kernel, bn, st))
+            if ops.config_smem_bytes({"kernel": kernel, "block_n": bn, "stages": st}) > BUDGET:
+                continue
+            if kernel == ops.PATH_SKINNY and st > 6:  # the small-M ring's depth cap
+                continue
+            expect.add((kernel, bn, st))
     assert built == expect
     # the defaults are among them
-    for kernel, bn, st in ((1, 128, 6), (1, 256, 4), (3, 256, 6), (4, 256, 4), (2, 256, 5)):
+    for kernel, bn, st in ((1, 128, 6), (1, 256, 4), (3, 256, 6), (4, 256, 4), (2, 256, 4),
+                           (2, 128, 4)):
         assert (kernel, bn, st) in built
 
 
@@ -37,7 +41,12 @@ def test_smem_formula(lib):
     assert ops.config_smem_bytes({"kernel": 1, "block_n": 256, "stages": 4}) == tile(49152, 4)
     assert ops.config_smem_bytes({"kernel": 3, "stages": 6}) == tile(32768, 6)
     assert ops.config_smem_bytes({"kernel": 4, "stages": 4}) == tile(49152, 4)
-    assert ops.config_smem_bytes({"kernel": 2, "stages": 5}) == 1024 + 5 * 40960 + 13 * 8 + 16
+    assert ops.config_smem_bytes({"kernel": 2, "block_n": 256, "stages": 5}) == \
+        1024 + 5 * 40960 + 13 * 8 + 16
+    assert ops.config_smem_bytes({"kernel": 2, "block_n": 128, "stages": 6}) == \
+        1024 + 6 * 24576 + 15 * 8 + 16
+    assert ops.config_smem_bytes({"kernel": 2, "block_n": 64, "stages": 4}) == -8
+    assert ops.config_smem_bytes({"kernel": 2, "stages": 4}) == -8  # width must be given
     # defaults when stages = 0; AUTO and bad widths name no kernel
     assert ops.config_smem_bytes({"kernel": 3}) == tile(32768, 6)
     assert ops.config_smem_bytes({"kernel": 0}) == -8
@@ -66,11 +75,17 @@ def test_candidates_cube(lib):
 
 
 def test_candidates_small_m(lib):
-    kept, pruned = tune.candidates(32, 4096, 8192, 148, ops.config_smem_bytes)
-    sk = [c for c in kept if c["kernel"] == ops.PATH_SKINNY]
-    # 16 column tiles: up to 9 slices fit 148 items; 128 k-blocks
+    built = {(c.kernel, c.block_n, c.stages) for c in ops.config_list()}
+    kept, pruned = tune.candidates(32, 4096, 8192, 148, ops.config_smem_bytes, built=built)
+    sk = [c for c in kept if c["kernel"] == ops.PATH_SKINNY and c["block_n"] == 256]
+    # 16 column tiles of 256: up to 9 slices fit 148 items; 128 k-blocks
     assert sorted({c["splits"] for c in sk}) == [0, 1, 2, 3, 4, 6, 8]
     assert {c["stages"] for c in sk} == {3, 4, 5}
+    sk128 = [c for c in kept if c["kernel"] == ops.PATH_SKINNY and c["block_n"] == 128]
+    # 32 column tiles of 128: up to 4 slices
+    assert sorted({c["splits"] for c in sk128}) == [0, 1, 2, 3, 4]
+    assert {c["stages"] for c in sk128} == {3, 4, 5, 6}
+    assert any("depth cap" in why for _, why in pruned)
     # tile kernels have a single tile-row: one panel each
     assert all(c["group_rows"] == tune.TILE_ROWS[c["kernel"]] for c in kept
                if c["kernel"] != ops.PATH_SKINNY)
@@ -83,4 +98,4 @@ def test_describe():
     assert tune.describe({"kernel": 4, "block_n": 256, "stages": 4, "group_rows": 2048,
                           "splits": 0}) == "pair-tall 512x256 st4 panel=2048"
     assert tune.describe({"kernel": 2, "block_n": 256, "stages": 5, "group_rows": 0,
-                          "splits": 0}) == "skinny st5 splits=auto"
+                          "splits": 0}) == "skinny 256 st5 splits=auto"

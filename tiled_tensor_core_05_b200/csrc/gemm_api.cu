@@ -412,9 +412,13 @@ int resolve_config(KernelConfig& c, int64_t M, int64_t N, int sm_count) {
       break;
     case GEMM_PATH_TILE_PAIR:
     case GEMM_PATH_TILE_PAIR_TALL:
-    case GEMM_PATH_SKINNY:
       if (c.block_n == 0) c.block_n = 256;
       if (c.block_n != 256) return GEMM_ERR_CONFIG;
+      break;
+    case GEMM_PATH_SKINNY:
+      if (c.block_n == 0)
+        c.block_n = (N + 255) / 256 * kSkinnyNarrowTilesPerSm < sm_count ? 128 : 256;
+      if (c.block_n != 128 && c.block_n != 256) return GEMM_ERR_CONFIG;
       break;
     default:
       return GEMM_ERR_CONFIG;
@@ -530,11 +534,12 @@ int gemm_f16_config(const void* A, const void* B, const void* bias, void* C, int
 int gemm_config_smem_bytes(const gemm_config* cfg) {
   if (cfg == nullptr) return GEMM_ERR_INVALID_ARG;
   int block_n = cfg->block_n;
-  if (block_n == 0 && cfg->kernel != GEMM_PATH_TILE) block_n = 256;
+  if (block_n == 0 && cfg->kernel != GEMM_PATH_TILE && cfg->kernel != GEMM_PATH_SKINNY)
+    block_n = 256;
   const int stages = cfg->stages != 0 ? cfg->stages : default_stages(cfg->kernel, block_n);
   int bytes = -1;
   if (cfg->kernel == GEMM_PATH_SKINNY)
-    bytes = block_n == 256 ? skinny_config_smem_bytes(stages) : -1;
+    bytes = skinny_config_smem_bytes(block_n, stages);
   else
     bytes = tile_config_smem_bytes(cfg->kernel, block_n, stages);
   return bytes > 0 ? bytes : GEMM_ERR_CONFIG;

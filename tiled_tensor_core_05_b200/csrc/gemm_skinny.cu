@@ -36,25 +36,28 @@
 namespace ttc {
 namespace {
 
-constexpr int kTW = 256;       // columns of B (rows of C^T) per CTA tile
+constexpr int kMaxTW = 256;    // widest tile: columns of B (rows of C^T) per CTA
 constexpr int kSub = 128;      // columns per MMA (MMA M)
 constexpr int kBK = 64;        // k-depth of a stage: one 128-byte swizzle row of A
 constexpr int kUmmaK = 16;
 constexpr int kThreads = 192;  // producer, MMA, 4 epilogue warps
 constexpr int kEpiWarps = 4;
 
-// Dynamic shared memory of the small-M kernel: 1 KiB of alignment slack, the
-// ring (256 columns of B and room for A^T per stage), the mbarriers (full
-// and empty per stage, accumulator-full, drain, one spare) and the TMEM
-// address slot.  A^T takes 8 KiB per stage for either MP.
-constexpr int skinny_smem_formula(int stages) {
-  return 1024 + stages * (4 * kBK * 64 * 2 + 8192) + (2 * stages + 3) * 8 + 16;
+// Dynamic shared memory of the small-M kernel with `tw` columns of B per CTA:
+// 1 KiB of alignment slack, the ring (tw columns of B and room for A^T per
+// stage), the mbarriers (full and empty per stage, accumulator-full, drain,
+// one spare) and the TMEM address slot.  A^T takes 8 KiB per stage for
+// either MP.
+constexpr int skinny_smem_formula(int tw, int stages) {
+  return 1024 + stages * (tw / 64 * kBK * 64 * 2 + 8192) + (2 * stages + 3) * 8 + 16;
 }
 
-template <int MP, int STAGES>
+// TW = 256 (two MMAs of M = 128 per 16-deep step) or 128 (one): narrower
+// tiles give twice the CTAs where there are few column tiles.
+template <int MP, int STAGES, int TW>
 struct SkinnyCfg {
   static constexpr int kBChunk = kBK * 64 * 2;    // 64 columns x 64 k-rows = 8 KiB
-  static constexpr int kBBytes = 4 * kBChunk;     // 256 columns
+  static constexpr int kBBytes = TW / 64 * kBChunk;  // TW columns
   // A^T: MP rows x 128 bytes (A stored M x K), or one 64-column slab of 64
   // k-rows (A stored K x M): room for the larger
   static constexpr int kABytesK = MP * kBK * 2;
@@ -62,27 +65,40 @@ struct SkinnyCfg {
   static constexpr int kStageBytes = kBBytes + kABytes;
   static constexpr int kNumBars = 2 * STAGES + 3;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kNumBars * 8 + 16;
-  static constexpr uint32_t kTmemCols = (2 * MP < 32) ? 32 : 2 * MP;
+  static constexpr uint32_t kTmemCols = (TW / kSub * MP < 32) ? 32 : TW / kSub * MP;
   static_assert(MP == 32 || MP == 64, "MP");
+  static_assert(TW == 128 || TW == 256, "tile width");
   static_assert(kABytes % 1024 == 0, "A tile alignment");
-  static_assert(kSmemBytes == skinny_smem_formula(STAGES), "layout");
+  static_assert(kSmemBytes == skinny_smem_formula(TW, STAGES), "layout");
   static_assert(kSmemBytes <= kMaxDynamicSmem, "shared memory budget");
 };
 
-// Ring depths compiled (for MP 32 and 64 and every activation): 3 up to what
-// fits the shared-memory budget.
-constexpr int kSkinnyStages[] = {3, 4, 5};
-constexpr int kNumSkinnyStages = sizeof(kSkinnyStages) / sizeof(kSkinnyStages[0]);
+// Configurations compiled (for MP 32 and 64 and every activation): each tile
+// width with every ring depth from 3 up to what fits the shared-memory budget
+// or 6, whichever is lower (a streaming ring gains nothing deeper: 6 stages of
+// the narrow tile already keep 144 KiB in flight per SM).
+struct SkinnyVariant {
+  int tw;
+  int stages;
+};
+constexpr SkinnyVariant kSkinnyVariants[] = {{256, 3}, {256, 4}, {256, 5}, {128, 3},
+                                             {128, 4}, {128, 5}, {128, 6}};
+constexpr int kNumSkinnyVariants = sizeof(kSkinnyVariants) / sizeof(kSkinnyVariants[0]);
+constexpr int kMaxSkinnyStages = 6;
 
 constexpr bool skinny_variants_complete() {
-  for (int st = 3; st <= 16; ++st) {
-    bool built = false;
-    for (int v : kSkinnyStages) built = built || v == st;
-    if ((skinny_smem_formula(st) <= kMaxDynamicSmem) != built) return false;
+  for (int tw : {128, 256}) {
+    for (int st = 3; st <= 16; ++st) {
+      bool built = false;
+      for (const auto& v : kSkinnyVariants) built = built || (v.tw == tw && v.stages == st);
+      const bool wanted = skinny_smem_formula(tw, st) <= kMaxDynamicSmem && st <= kMaxSkinnyStages;
+      if (wanted != built) return false;
+    }
   }
   return true;
 }
-static_assert(skinny_variants_complete(), "built skinny configurations != those within the budget");
+static_assert(skinny_variants_complete(),
+              "built skinny configurations != those within the budget and depth cap");
 
 __device__ __forceinline__ float4 ld_cg_f4(const float* p) {
   return __ldcg(reinterpret_cast<const float4*>(p));
@@ -134,14 +150,14 @@ __device__ __forceinline__ void load_accumulator(uint32_t taddr, float (&v)[MP])
 // One CTA per (tile, k-slice); blockIdx.x = tile * S + slice.  B (streamed
 // once) is loaded with an L2 evict-first policy and A (re-read by every CTA)
 // with evict-last.
-template <int MP, int STAGES, int ACT>
+template <int MP, int STAGES, int TW, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, __half* __restrict__ C, int M,
                        int N, int K, int64_t ldc, const __half* __restrict__ bias, int S,
                        int layout, float* __restrict__ partials, int* __restrict__ counters,
                        int* status, uint64_t timeout_ns) {
-  using Cfg = SkinnyCfg<MP, STAGES>;
+  using Cfg = SkinnyCfg<MP, STAGES, TW>;
   const bool ta = (layout & kLayoutTransA) != 0;
   const bool tb = (layout & kLayoutTransB) != 0;
   // bytes of one stage: 256 columns of B, and A^T as stored
@@ -210,13 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(&full[stage], stage_bytes);
         uint8_t* bdst = smB + stage * Cfg::kBBytes;
-        if (!tb) {  // row-major B: four 64-column slabs of 64 k-rows
+        if (!tb) {  // row-major B: TW / 64 slabs of 64 columns by 64 k-rows
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tma_load_2d_hint(&tmB, &full[stage], bdst + j * Cfg::kBChunk, tile * kTW + j * 64,
+          for (int j = 0; j < TW / 64; ++j)
+            tma_load_2d_hint(&tmB, &full[stage], bdst + j * Cfg::kBChunk, tile * TW + j * 64,
                              kb * kBK, pol_b);
-        } else {  // B stored N x K: 256 rows of 64 k
-          tma_load_2d_hint(&tmB, &full[stage], bdst, kb * kBK, tile * kTW, pol_b);
+        } else {  // B stored N x K: TW rows of 64 k
+          tma_load_2d_hint(&tmB, &full[stage], bdst, kb * kBK, tile * TW, pol_b);
         }
         if (!ta)  // A stored M x K: MP rows of 64 k
           tma_load_2d_hint(&tmA, &full[stage], smA + stage * Cfg::kABytes, kb * kBK, 0, pol_a);
@@ -257,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // (A^T is K-major when A is stored M x K, MN-major when stored K x M)
           const uint64_t bdesc = operand_desc(a_addr, k, ta, Cfg::kBChunk);
 #pragma unroll
-          for (int h = 0; h < kTW / kSub; ++h) {
+          for (int h = 0; h < TW / kSub; ++h) {
             // MMA A operand = B^T sub-tile h (columns 128h..128h+127 of the
             // tile; 16 KiB into the stage in both layouts): N-major slabs of
             // row-major B, or K-major rows of B stored N x K
@@ -296,24 +312,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         raise_abort(status, abort_flag, kStatusTimeoutBase | (kRoleEpilogue << 4) | 2);
     } else {
       tc_fence_after_sync();
-      const int n0 = tile * kTW + row;
+      const int n0 = tile * TW + row;
       const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       // one 128-column half at a time keeps only MP accumulators per thread live
       if (S == 1) {
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < TW / kSub; ++h) {
           float v[MP];
           load_accumulator<MP>(t_lane + static_cast<uint32_t>(h * MP), v);
           store_column<MP, ACT>(v, C, M, N, ldc, n0 + h * kSub, bias);
         }
       } else {
-        // partial tile of this slice: [item][256 columns][MP]
+        // partial tile of this slice: [item][TW columns][MP]
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < TW / kSub; ++h) {
           float v[MP];
           load_accumulator<MP>(t_lane + static_cast<uint32_t>(h * MP), v);
           float* mine =
-              partials + (static_cast<int64_t>(blockIdx.x) * kTW + h * kSub + row) * MP;
+              partials + (static_cast<int64_t>(blockIdx.x) * TW + h * kSub + row) * MP;
 #pragma unroll
           for (int m = 0; m < MP; m += 4)
             *reinterpret_cast<float4*>(mine + m) = make_float4(v[m], v[m + 1], v[m + 2], v[m + 3]);
@@ -334,11 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // added, so the fix-up costs one L2 round trip per four slices
           // rather than per slice (same sums in the same order: same bits).
           // This slice's own partial is read back from TMEM at its turn.
-          const int64_t slice_stride = static_cast<int64_t>(kTW) * MP;
+          const int64_t slice_stride = static_cast<int64_t>(TW) * MP;
 #pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < TW / kSub; ++h) {
             const float* base =
-                partials + ((static_cast<int64_t>(tile) * S) * kTW + h * kSub + row) * MP;
+                partials + ((static_cast<int64_t>(tile) * S) * TW + h * kSub + row) * MP;
 #pragma unroll 1
             for (int mc = 0; mc < MP / 32; ++mc) {
               float acc[32];
@@ -412,17 +428,17 @@ constexpr size_t counter_bytes(int n) {
 
 // Number of k-slices per tile: 1 when the tiles already cover the SMs,
 // otherwise as many as fit on the idle SMs, with at least 16 k-blocks of 64
-// per slice, S * MP <= 256 (the last slice to arrive sums the S partial tiles
-// of 256 x MP fp32 one after another, a cost that grows with S * MP), and at
-// most `max_items` (tile, slice) pairs.  Fitted to a sweep of small-M shapes
-// (M 16-64, N 1024-28672, K 4096-16384): the best or tied-best slice count on
-// each; the former rule (up to SMs / tiles slices of >= 4 k-blocks) was up to
-// 1.85x slower where few column tiles allowed many slices.
-int choose_slices(int64_t tiles, int64_t KB, int MP, int sm_count, int64_t max_items) {
+// per slice, S * TW * MP <= 65536 (the last slice to arrive sums the S
+// partial tiles of TW x MP fp32 alone, a cost that grows with S * TW * MP),
+// and at most `max_items` (tile, slice) pairs.  Fitted to a sweep of small-M
+// shapes (M 16-64, N 1024-28672, K 4096-16384): the best or tied-best slice
+// count on each; the former rule (up to SMs / tiles slices of >= 4 k-blocks)
+// was up to 1.85x slower where few column tiles allowed many slices.
+int choose_slices(int64_t tiles, int64_t KB, int MP, int TW, int sm_count, int64_t max_items) {
   if (tiles >= sm_count) return 1;
   int64_t s = sm_count / tiles;
   const int64_t by_k = KB / 16;
-  const int64_t by_fixup = 256 / MP;
+  const int64_t by_fixup = 65536 / (static_cast<int64_t>(TW) * MP);
   if (s > by_k) s = by_k;
   if (s > by_fixup) s = by_fixup;
   if (s * tiles > max_items) s = max_items / tiles;
@@ -431,22 +447,22 @@ int choose_slices(int64_t tiles, int64_t KB, int MP, int sm_count, int64_t max_i
 
 // `splits` = 0 chooses the k-slices from the shape; otherwise exactly that
 // many (1 <= splits <= k-blocks, and splits * tiles <= max_items when > 1).
-template <int MP, int STAGES, int ACT>
+template <int MP, int STAGES, int TW, int ACT>
 int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
                 int64_t max_items, int splits) {
-  using Cfg = SkinnyCfg<MP, STAGES>;
+  using Cfg = SkinnyCfg<MP, STAGES, TW>;
   static std::atomic<uint64_t> attr_done{0};
   const int64_t KB = (p.K + kBK - 1) / kBK;
-  const int64_t tiles = (p.N + kTW - 1) / kTW;
+  const int64_t tiles = (p.N + TW - 1) / TW;
   if (splits < 0 || splits > KB || (splits > 1 && splits * tiles > max_items))
     return GEMM_ERR_CONFIG;
-  const int S = splits > 0 ? splits : choose_slices(tiles, KB, MP, d.sm_count, max_items);
+  const int S = splits > 0 ? splits : choose_slices(tiles, KB, MP, TW, d.sm_count, max_items);
   int* counters = nullptr;
   float* partials = nullptr;
   if (S > 1) {
     // counters for the tiles, then one fp32 partial tile per (tile, slice)
     const size_t need = counter_bytes(static_cast<int>(max_items)) +
-                        static_cast<size_t>(tiles) * S * kTW * MP * sizeof(float);
+                        static_cast<size_t>(tiles) * S * TW * MP * sizeof(float);
     if (ws == nullptr || ws_bytes < need) return GEMM_ERR_WORKSPACE;
     counters = static_cast<int*>(ws);
     partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
@@ -459,12 +475,12 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_by
   else  // stored M x K: MP rows of 64 k
     rc = encode_tmap_f16_2d(&tA, p.A, p.K, p.M, p.lda, kBK, MP);
   if (rc != 0) return rc;
-  if (p.layout & kLayoutTransB)  // stored N x K: 256 rows of 64 k
-    rc = encode_tmap_f16_2d(&tB, p.B, p.K, p.N, p.ldb, kBK, kTW);
+  if (p.layout & kLayoutTransB)  // stored N x K: TW rows of 64 k
+    rc = encode_tmap_f16_2d(&tB, p.B, p.K, p.N, p.ldb, kBK, TW);
   else  // row-major: slabs of 64 columns by 64 k-rows
     rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
   if (rc != 0) return rc;
-  auto kern = skinny_gemm_kernel<MP, STAGES, ACT>;
+  auto kern = skinny_gemm_kernel<MP, STAGES, TW, ACT>;
   if (!ensure_smem_attr_skinny(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
                                attr_done))
     return GEMM_ERR_LAUNCH;
@@ -497,29 +513,33 @@ size_t skinny_workspace_bytes(int sm_count, int m_pad) {
   // split-K happens only with fewer tiles than SMs, so at most sm_count
   // (tile, slice) items carry a partial tile
   return counter_bytes(sm_count) +
-         static_cast<size_t>(sm_count) * kTW * static_cast<size_t>(m_pad) * sizeof(float);
+         static_cast<size_t>(sm_count) * kMaxTW * static_cast<size_t>(m_pad) * sizeof(float);
 }
 
 namespace {
 
-template <int MP, int STAGES>
+template <int MP, int STAGES, int TW>
 int launch_act(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes, int splits) {
   switch (p.act) {
-    case kActRelu: return launch_impl<MP, STAGES, kActRelu>(p, d, ws, ws_bytes, d.sm_count, splits);
-    case kActGelu: return launch_impl<MP, STAGES, kActGelu>(p, d, ws, ws_bytes, d.sm_count, splits);
-    default: return launch_impl<MP, STAGES, kActNone>(p, d, ws, ws_bytes, d.sm_count, splits);
+    case kActRelu:
+      return launch_impl<MP, STAGES, TW, kActRelu>(p, d, ws, ws_bytes, d.sm_count, splits);
+    case kActGelu:
+      return launch_impl<MP, STAGES, TW, kActGelu>(p, d, ws, ws_bytes, d.sm_count, splits);
+    default:
+      return launch_impl<MP, STAGES, TW, kActNone>(p, d, ws, ws_bytes, d.sm_count, splits);
   }
 }
 
 template <int MP, int I = 0>
-int dispatch_stages(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
-                    const KernelConfig& c) {
-  if constexpr (I == kNumSkinnyStages) {
+int dispatch_variant(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
+                     const KernelConfig& c) {
+  if constexpr (I == kNumSkinnyVariants) {
     return GEMM_ERR_CONFIG;
   } else {
-    if (c.stages == kSkinnyStages[I])
-      return launch_act<MP, kSkinnyStages[I]>(p, d, ws, ws_bytes, c.splits);
-    return dispatch_stages<MP, I + 1>(p, d, ws, ws_bytes, c);
+    constexpr SkinnyVariant v = kSkinnyVariants[I];
+    if (c.block_n == v.tw && c.stages == v.stages)
+      return launch_act<MP, v.stages, v.tw>(p, d, ws, ws_bytes, c.splits);
+    return dispatch_variant<MP, I + 1>(p, d, ws, ws_bytes, c);
   }
 }
 
@@ -528,20 +548,21 @@ int dispatch_stages(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t w
 int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_bytes,
                        const KernelConfig& c) {
   const int mp = skinny_m_pad(p.M);
-  if (mp == 32) return dispatch_stages<32>(p, d, ws, ws_bytes, c);
-  if (mp == 64) return dispatch_stages<64>(p, d, ws, ws_bytes, c);
+  if (mp == 32) return dispatch_variant<32>(p, d, ws, ws_bytes, c);
+  if (mp == 64) return dispatch_variant<64>(p, d, ws, ws_bytes, c);
   return GEMM_ERR_INVALID_ARG;
 }
 
-int skinny_config_smem_bytes(int stages) {
-  if (stages < 1 || stages > 64) return -1;
-  return skinny_smem_formula(stages);
+int skinny_config_smem_bytes(int block_n, int stages) {
+  if (stages < 1 || stages > 64 || (block_n != 128 && block_n != 256)) return -1;
+  return skinny_smem_formula(block_n, stages);
 }
 
 int skinny_configs_built(KernelConfig* out, int cap) {
-  for (int i = 0; i < kNumSkinnyStages && i < cap; ++i)
-    out[i] = KernelConfig{GEMM_PATH_SKINNY, kTW, kSkinnyStages[i], 0, 0};
-  return kNumSkinnyStages;
+  for (int i = 0; i < kNumSkinnyVariants && i < cap; ++i)
+    out[i] = KernelConfig{GEMM_PATH_SKINNY, kSkinnyVariants[i].tw, kSkinnyVariants[i].stages, 0,
+                          0};
+  return kNumSkinnyVariants;
 }
 
 // ------------------------------------------------ allocation-free variant ---
@@ -555,7 +576,8 @@ constexpr int kNoAllocMP = 32;
 constexpr int kNoAllocMaxItems = 160;
 constexpr size_t kNoAllocCounterBytes = counter_bytes(kNoAllocMaxItems);
 constexpr size_t kNoAllocScratchBytes =
-    kNoAllocCounterBytes + static_cast<size_t>(kNoAllocMaxItems) * kTW * kNoAllocMP * sizeof(float);
+    kNoAllocCounterBytes +
+    static_cast<size_t>(kNoAllocMaxItems) * kMaxTW * kNoAllocMP * sizeof(float);
 static_assert(kNoAllocScratchBytes == 5243648, "documented scratch size");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -592,7 +614,7 @@ int launch_skinny_gemm_noalloc(const GemmProblem& p, const DeviceCtx& d) {
   if (cudaMemsetAsync(scratch, 0, kNoAllocCounterBytes, p.stream) != cudaSuccess)
     return GEMM_ERR_LAUNCH;
   const int64_t items = d.sm_count < kNoAllocMaxItems ? d.sm_count : kNoAllocMaxItems;
-  return launch_impl<kNoAllocMP, kDefaultStagesSkinny, kActRelu>(p, d, scratch,
+  return launch_impl<kNoAllocMP, kDefaultStagesSkinny, kMaxTW, kActRelu>(p, d, scratch,
                                                              kNoAllocScratchBytes, items, 0);
 }
 

@@ -41,6 +41,9 @@ constexpr int kDefaultStagesTall = 4;
 // 4 ties 5 on the decode shape (one k-slice) and is up to 1.95x faster than 5
 // at the same count of several k-slices (offline sweep of small-M shapes)
 constexpr int kDefaultStagesSkinny = 4;
+// The small-M kernel takes 128-column tiles (twice the CTAs) when a problem
+// has fewer 256-column tiles than a quarter of the SMs.
+constexpr int kSkinnyNarrowTilesPerSm = 4;
 
 struct DeviceCtx {
   int device;
@@ -85,7 +88,7 @@ size_t skinny_workspace_bytes(int sm_count, int m_pad);
 int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* workspace,
                        size_t workspace_bytes, const KernelConfig& c);
 int skinny_m_pad(int64_t M);  // MMA N used for M rows (0 if M is too large)
-int skinny_config_smem_bytes(int stages);
+int skinny_config_smem_bytes(int block_n, int stages);  // -1 when block_n is not 128 / 256
 int skinny_configs_built(KernelConfig* out, int cap);
 
 // The small-M kernel with its scratch in a fixed device array of the library

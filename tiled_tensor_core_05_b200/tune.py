@@ -14,13 +14,13 @@ defaults are set from the table this script writes.
 
 For each workload:
   1. the candidate space: every tile shape (128 x 128 and 128 x 256 on one SM,
-     256 x 256 and 512 x 256 on a CTA pair, the 256-column small-M kernel when
-     M <= 64) x ring depths 3..8 x raster panels (1, 2, 4, ... tile-rows, up to
-     all of them) or k-slices;
+     256 x 256 and 512 x 256 on a CTA pair, the 128- and 256-column small-M
+     kernel when M <= 64) x ring depths 3..8 x raster panels (1, 2, 4, ...
+     tile-rows, up to all of them) or k-slices;
   2. pruning: depths whose shared memory (gemm_config_smem_bytes) exceeds the
-     227 KiB a CTA can opt into, duplicate panels (a panel of more tile-rows
-     than the problem has is the whole column), k-slice counts the split-K
-     workspace or K cannot hold;
+     227 KiB a CTA can opt into, small-M ring depths beyond the compiled cap of
+     6, duplicate panels (a panel of more tile-rows than the problem has is
+     the whole column), k-slice counts the split-K workspace or K cannot hold;
   3. validation of each survivor against torch's fp32 product, activated, with
      the pages' check |c - ref| <= 1e-2 + 1e-2 |ref| plus c > 0 wherever
      ref > 1e-2 (ReLU); a candidate that fails is reported and never ranked;
@@ -55,7 +55,7 @@ TILE_KINDS = [(ops.PATH_TILE, 128), (ops.PATH_TILE, 256), (ops.PATH_TILE_PAIR, 2
 TILE_ROWS = {ops.PATH_TILE: 128, ops.PATH_TILE_PAIR: 256, ops.PATH_TILE_PAIR_TALL: 512}
 KERNEL_NAMES = {ops.PATH_TILE: "tile", ops.PATH_SKINNY: "skinny",
                 ops.PATH_TILE_PAIR: "pair", ops.PATH_TILE_PAIR_TALL: "pair-tall"}
-SKINNY_WIDTH = 256
+SKINNY_WIDTHS = (128, 256)
 
 # extra shapes of the sweep beside the named workloads: a small-M product
 # with few column tiles, where split-K has room to act
@@ -77,19 +77,21 @@ def describe(cfg: dict) -> str:
     k = cfg["kernel"]
     if k == ops.PATH_SKINNY:
         s = cfg["splits"]
-        return f"skinny st{cfg['stages']} splits={'auto' if s == 0 else s}"
+        return f"skinny {cfg['block_n']} st{cfg['stages']} splits={'auto' if s == 0 else s}"
     rows = TILE_ROWS[k]
     return (f"{KERNEL_NAMES[k]} {rows}x{cfg['block_n']} st{cfg['stages']} "
             f"panel={cfg['group_rows']}")
 
 
-def candidates(M: int, N: int, K: int, sm_count: int, smem_fn, budget: int = SMEM_BUDGET):
+def candidates(M: int, N: int, K: int, sm_count: int, smem_fn, budget: int = SMEM_BUDGET,
+               built=None):
     """(kept, pruned): kept is a list of config dicts; pruned a list of
-    (config dict, reason).  `smem_fn(cfg) -> bytes` is the library's formula."""
+    (config dict, reason).  `smem_fn(cfg) -> bytes` is the library's formula;
+    `built` (a set of (kernel, block_n, stages)) prunes what is not compiled."""
     kept, pruned = [], []
     kinds = list(TILE_KINDS)
     if M <= 64:
-        kinds.append((ops.PATH_SKINNY, SKINNY_WIDTH))
+        kinds += [(ops.PATH_SKINNY, w) for w in SKINNY_WIDTHS]
     for kernel, bn in kinds:
         for st in STAGE_RANGE:
             base = {"kernel": kernel, "block_n": bn, "stages": st, "group_rows": 0,
@@ -98,8 +100,11 @@ def candidates(M: int, N: int, K: int, sm_count: int, smem_fn, budget: int = SME
             if smem > budget:
                 pruned.append((base, f"shared memory {smem} > {budget}"))
                 continue
+            if built is not None and (kernel, bn, st) not in built:
+                pruned.append((base, "not compiled (depth cap)"))
+                continue
             if kernel == ops.PATH_SKINNY:
-                tiles = -(-N // SKINNY_WIDTH)
+                tiles = -(-N // bn)
                 kb = -(-K // 64)
                 seen = set()
                 for s in (0, 1, 2, 3, 4, 6, 8, 12, 16, 24, 32):
@@ -201,7 +206,8 @@ def sweep_workload(w: Workload, act: str, use_bias: bool, steps: int, rounds: in
     ref = _reference(a, b, bias, act)
     stream = torch.cuda.current_stream(dev)
     auto = ops.auto_config(w.M, w.N, w.K, act).as_dict()
-    kept, pruned = candidates(w.M, w.N, w.K, sm_count, ops.config_smem_bytes)
+    built = {(c.kernel, c.block_n, c.stages) for c in ops.config_list()}
+    kept, pruned = candidates(w.M, w.N, w.K, sm_count, ops.config_smem_bytes, built=built)
     if only is not None:
         full = {"kernel": 0, "block_n": 0, "stages": 0, "group_rows": 0, "splits": 0}
         kept, pruned = [{**full, **c} for c in only], []
