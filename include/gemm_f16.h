@@ -74,9 +74,9 @@ enum gemm_path {
                               otherwise TILE_PAIR_TALL, or TILE_PAIR when the 512-row
                               tiles leave a much emptier last wave */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile (any shape) */
-  GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 256 (or, with few column tiles, 128)
-                              columns of B per CTA streamed in lock-step, split-K only when
-                              tiles < SMs (M <= 64 only) */
+  GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 128 columns of B per CTA when
+                              ceil(N / 128) <= SMs, else 256, streamed in lock-step,
+                              split-K only when tiles < SMs (M <= 64 only) */
   GEMM_PATH_TILE_PAIR = 3, /* persistent kernel, two SMs (a CTA pair) per 256 x 256 tile
                               (any shape) */
   GEMM_PATH_TILE_PAIR_TALL = 4 /* persistent kernel, a CTA pair per 512 x 256 tile: fewer

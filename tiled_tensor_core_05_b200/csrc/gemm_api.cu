@@ -390,7 +390,7 @@ int default_stages(int kernel, int block_n) {
     case GEMM_PATH_TILE: return block_n == 256 ? kDefaultStagesTile256 : kDefaultStagesTile128;
     case GEMM_PATH_TILE_PAIR: return kDefaultStagesPair;
     case GEMM_PATH_TILE_PAIR_TALL: return kDefaultStagesTall;
-    case GEMM_PATH_SKINNY: return kDefaultStagesSkinny;
+    case GEMM_PATH_SKINNY: return block_n == 128 ? kDefaultStagesSkinnyNarrow : kDefaultStagesSkinny;
     default: return 0;
   }
 }
@@ -416,8 +416,7 @@ int resolve_config(KernelConfig& c, int64_t M, int64_t N, int sm_count) {
       if (c.block_n != 256) return GEMM_ERR_CONFIG;
       break;
     case GEMM_PATH_SKINNY:
-      if (c.block_n == 0)
-        c.block_n = (N + 255) / 256 * kSkinnyNarrowTilesPerSm < sm_count ? 128 : 256;
+      if (c.block_n == 0) c.block_n = (N + 127) / 128 <= sm_count ? 128 : 256;
       if (c.block_n != 128 && c.block_n != 256) return GEMM_ERR_CONFIG;
       break;
     default:

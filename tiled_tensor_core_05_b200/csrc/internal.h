@@ -41,9 +41,12 @@ constexpr int kDefaultStagesTall = 4;
 // 4 ties 5 on the decode shape (one k-slice) and is up to 1.95x faster than 5
 // at the same count of several k-slices (offline sweep of small-M shapes)
 constexpr int kDefaultStagesSkinny = 4;
-// The small-M kernel takes 128-column tiles (twice the CTAs) when a problem
-// has fewer 256-column tiles than a quarter of the SMs.
-constexpr int kSkinnyNarrowTilesPerSm = 4;
+// The small-M kernel takes 128-column tiles (twice the CTAs of 256-column
+// ones) when they fit on the SMs in one wave, ceil(N / 128) <= SMs, with a
+// 6-stage ring.  Measured (M 16-64, N 1024-14336, K 4096-16384): 1.1-1.5x
+// faster than 256-column tiles there; on N = 28672 (224 narrow tiles) the
+// wide ones are 1.3x faster.
+constexpr int kDefaultStagesSkinnyNarrow = 6;
 
 struct DeviceCtx {
   int device;
