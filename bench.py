@@ -246,6 +246,12 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
     return res
 
 
+def hbm_bound(w) -> bool:
+    """Small-M products stream B once and are measured in GB/s; the rest are
+    tensor-pipe bound and measured in TFLOP/s."""
+    return w.M <= 64
+
+
 def kernel_for(w) -> str:
     from tiled_tensor_core_05_b200 import ops
     return {ops.PATH_SKINNY: "skinny_gemm_kernel", ops.PATH_TILE: "tile_gemm_kernel",
@@ -257,7 +263,7 @@ def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool):
     from tiled_tensor_core_05_b200 import workloads
     w = workloads.WORKLOADS[name]
     kernel = kernel_for(w)
-    if name == "decode":
+    if hbm_bound(w):
         # HBM bound: algorithmic bytes = A, B read once, C written once
         achieved = w.bytes_min / (launch_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
@@ -370,7 +376,7 @@ def cpu_baseline(name, budget_s=10.0):
     oracle.gemm_relu(a[:rows], b)
     dt = time.perf_counter() - t0
     flops = 2.0 * rows * w.N * w.K
-    if name == "decode":
+    if hbm_bound(w):
         value = (2.0 * (rows * w.K + w.K * w.N + rows * w.N)) / dt / 1e9
         unit = "GB/s"
     else:
@@ -399,7 +405,7 @@ def run_reference(args):
     for _ in range(args.steps):
         oracle.gemm_relu(a[:rows], b)
     dt = (time.perf_counter() - t0) / args.steps
-    if args.workload == "decode":
+    if hbm_bound(w):
         value, unit = 2.0 * (rows * w.K + w.K * w.N + rows * w.N) / dt / 1e9, "GB/s"
     else:
         value, unit = 2.0 * rows * w.N * w.K / dt / 1e12, "TFLOP/s"
@@ -454,7 +460,7 @@ def run_ours(args):
     w = main["w"]
     long_run = main["total_ms"] > 2000.0
     ms = main["total_ms"] / args.steps
-    if args.workload == "decode":
+    if hbm_bound(w):
         value, unit = job_rate(w.bytes_min, world, ms) / 1e9, "GB/s"
     else:
         value, unit = job_rate(w.flops, world, ms) / 1e12, "TFLOP/s"
@@ -463,7 +469,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic (seeded torch.randn on the CPU, cast to fp16)",
             "config": workload_config(w), "gpu_launches": args.steps}
-    if args.workload == "decode":
+    if hbm_bound(w):
         line["pct_of_nominal_hbm"] = round(100 * value / world / NOMINAL_HBM_GBS, 2)
     else:
         line["pct_of_dense_fp16_peak"] = round(100 * value / world / NOMINAL_FP16_TFLOPS, 2)
@@ -500,7 +506,7 @@ def run_ours(args):
                      "roofline": roofline_entry(name, r["launch_ms"], peaks, peak_src, False)}
             if "torch_launch_ms" in r:
                 entry["context_torch_ms_per_call"] = round(r["torch_launch_ms"], 5)
-            if name == "decode":
+            if hbm_bound(ow):
                 entry["gbs"] = round(ow.bytes_min / (r["launch_ms"] * 1e-3) / 1e9, 1)
                 entry["pct_of_nominal_hbm"] = round(100 * entry["gbs"] / NOMINAL_HBM_GBS, 2)
             else:

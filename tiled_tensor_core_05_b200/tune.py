@@ -57,22 +57,6 @@ KERNEL_NAMES = {ops.PATH_TILE: "tile", ops.PATH_SKINNY: "skinny",
                 ops.PATH_TILE_PAIR: "pair", ops.PATH_TILE_PAIR_TALL: "pair-tall"}
 SKINNY_WIDTHS = (128, 256)
 
-# extra shapes of the sweep beside the named workloads: a small-M product
-# with few column tiles, where split-K has room to act
-EXTRA = {w.name: w for w in [
-    Workload("decode_n4096", 32, 4096, 8192, 5, 1.0, 0.02,
-             "M=32, K=8192, N=4096; A ~ N(0,1), B ~ N(0, 0.02^2), seed 5"),
-    Workload("decode_m16_n8192_k4096", 16, 8192, 4096, 6, 1.0, 0.02,
-             "M=16, K=4096, N=8192; A ~ N(0,1), B ~ N(0, 0.02^2), seed 6"),
-    Workload("decode_m64_n2048_k8192", 64, 2048, 8192, 7, 1.0, 0.02,
-             "M=64, K=8192, N=2048; A ~ N(0,1), B ~ N(0, 0.02^2), seed 7"),
-    Workload("decode_n1024_k16384", 32, 1024, 16384, 8, 1.0, 0.02,
-             "M=32, K=16384, N=1024; A ~ N(0,1), B ~ N(0, 0.02^2), seed 8"),
-    Workload("decode_n14336_k4096", 32, 14336, 4096, 9, 1.0, 0.02,
-             "M=32, K=4096, N=14336; A ~ N(0,1), B ~ N(0, 0.02^2), seed 9"),
-]}
-
-
 def describe(cfg: dict) -> str:
     k = cfg["kernel"]
     if k == ops.PATH_SKINNY:
@@ -356,7 +340,7 @@ def main(argv=None):
     reports = []
     try:
         for i, (name, act, use_bias) in enumerate(plan):
-            w = WORKLOADS.get(name) or EXTRA[name]
+            w = WORKLOADS[name]
             reports.append(sweep_workload(w, act, use_bias, args.steps, args.rounds,
                                           args.leaders, sampler=sampler, seed=i,
                                           round_steps=args.round_steps, cool_s=args.cool,

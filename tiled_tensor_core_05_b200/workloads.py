@@ -59,6 +59,17 @@ WORKLOADS = {
         Workload("decode", 32, 28672, 8192, 4, 1.0, 0.02,
                  "decode-shaped M=32, K=8192, N=28672; A ~ N(0,1), B ~ N(0, 0.02^2), "
                  "seed 4 (HBM bound on B)"),
+        # further small-M shapes (the configuration sweep's; few column tiles)
+        Workload("decode_n4096", 32, 4096, 8192, 5, 1.0, 0.02,
+                 "M=32, K=8192, N=4096; A ~ N(0,1), B ~ N(0, 0.02^2), seed 5"),
+        Workload("decode_m16_n8192_k4096", 16, 8192, 4096, 6, 1.0, 0.02,
+                 "M=16, K=4096, N=8192; A ~ N(0,1), B ~ N(0, 0.02^2), seed 6"),
+        Workload("decode_m64_n2048_k8192", 64, 2048, 8192, 7, 1.0, 0.02,
+                 "M=64, K=8192, N=2048; A ~ N(0,1), B ~ N(0, 0.02^2), seed 7"),
+        Workload("decode_n1024_k16384", 32, 1024, 16384, 8, 1.0, 0.02,
+                 "M=32, K=16384, N=1024; A ~ N(0,1), B ~ N(0, 0.02^2), seed 8"),
+        Workload("decode_n14336_k4096", 32, 14336, 4096, 9, 1.0, 0.02,
+                 "M=32, K=4096, N=14336; A ~ N(0,1), B ~ N(0, 0.02^2), seed 9"),
     ]
 }
 
