@@ -491,7 +491,10 @@ def run_ours(args):
             "ms_per_call": round(t_ms, 5),
             "tflops": round(w.flops / (t_ms * 1e-3) / 1e12, 2) if unit == "TFLOP/s" else None,
             "gbs": round(w.bytes_min / (t_ms * 1e-3) / 1e9, 1) if unit == "GB/s" else None}
-    if rank == 0 and not args.no_secondary:
+    # context passes (other workloads, probe, per-launch and sustained runs)
+    # only in single-GPU runs: under torchrun the other ranks would wait for
+    # rank 0 at the closing barrier meanwhile
+    if rank == 0 and world == 1 and not args.no_secondary:
         others = []
         for name, variant in (("mlp_up", "relu"), ("decode", "relu"), ("cube1024", "relu"),
                               ("cube256", "relu"), ("mlp_up", "bias_gelu"), ("decode", "wT")):
@@ -521,7 +524,7 @@ def run_ours(args):
                 value / world if unit == "GB/s" else None)
             if gbs:
                 entry["frac_of_read_probe"] = round(gbs / probe["gbs"], 4)
-    if rank == 0 and args.sustained_seconds > 0:
+    if rank == 0 and world == 1 and args.sustained_seconds > 0:
         line["launch_stats"] = launch_stats(main["step"])
         sus = sustained_run(main["step"], main["launch_ms"], args.sustained_seconds,
                             gpu_id_for(local))

@@ -8,8 +8,8 @@
 //     columns is the MMA M dimension (B^T is MN-major in shared memory, read
 //     straight from row-major B) and the few rows of A are the MMA N
 //     dimension (MP = M rounded up to 32 or 64; A^T is K-major).  One CTA owns
-//     a 256-column tile of C^T: two MMAs per 16-deep k step into two TMEM
-//     accumulators.
+//     a TW-column tile of C^T (TW = 256: two MMAs per 16-deep k step into two
+//     TMEM accumulators; TW = 128, for problems with few column tiles: one).
 //   * lock-step streaming: every CTA walks its k-range upward from the same
 //     start at the same time, so at any moment the whole grid reads the same
 //     band of rows of B across all N.  Row-major B then streams in long
@@ -24,8 +24,9 @@
 //     de una sola línea cada una", applied to the K axis of the GEMM.  Each
 //     slice writes its fp32 partial tile to a workspace and bumps the tile's
 //     arrival counter; whichever slice arrives last sums the S partials in
-//     slice order (deterministic), then applies ReLU -- only after the full K
-//     reduction -- and stores fp16.  No CTA ever waits for another.
+//     slice order (deterministic), then applies the bias and activation --
+//     only after the full K reduction -- and stores fp16.  No CTA ever waits
+//     for another.
 #include <atomic>
 #include <mutex>
 
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Cfg = SkinnyCfg<MP, STAGES, TW>;
   const bool ta = (layout & kLayoutTransA) != 0;
   const bool tb = (layout & kLayoutTransB) != 0;
-  // bytes of one stage: 256 columns of B, and A^T as stored
+  // bytes of one stage: TW columns of B, and A^T as stored
   const uint32_t stage_bytes = Cfg::kBBytes + (ta ? 8192u : static_cast<uint32_t>(Cfg::kABytesK));
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);

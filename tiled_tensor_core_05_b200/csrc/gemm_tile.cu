@@ -180,18 +180,33 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
                                               Release release) {
 #pragma unroll 1
   for (int c = 0; c < COLS / kEpiCols; ++c) {
-    // the 64 bias values of this chunk as 32 packed pairs (0 past N)
+    // the 64 bias values of this chunk as 32 packed pairs (0 past N): eight
+    // 16-byte loads (the same address in every lane) when the chunk lies
+    // inside N, else pair by pair
     uint32_t bb[32];
     if (bias != nullptr) {
       const int col0 = col_base + c * kEpiCols;
+      if (col0 + kEpiCols <= N) {
+        const uint4* src = reinterpret_cast<const uint4*>(bias + col0);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int col = col0 + 2 * i;
-        if (col + 1 < N) {
-          bb[i] = __ldg(reinterpret_cast<const unsigned int*>(bias + col));
-        } else {
-          const unsigned short lo = col < N ? __ldg(reinterpret_cast<const unsigned short*>(bias + col)) : 0;
-          bb[i] = lo;
+        for (int i = 0; i < 8; ++i) {
+          const uint4 q = __ldg(src + i);
+          bb[4 * i] = q.x;
+          bb[4 * i + 1] = q.y;
+          bb[4 * i + 2] = q.z;
+          bb[4 * i + 3] = q.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = col0 + 2 * i;
+          if (col + 1 < N) {
+            bb[i] = __ldg(reinterpret_cast<const unsigned int*>(bias + col));
+          } else {
+            const unsigned short lo =
+                col < N ? __ldg(reinterpret_cast<const unsigned short*>(bias + col)) : 0;
+            bb[i] = lo;
+          }
         }
       }
     }
