@@ -630,45 +630,108 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       bool ok = true;
       int site = 0;
       const uint32_t idesc = idesc_f16_f32(2 * kBM, BN, ta, !tb);
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
-          ok = false;
-          site = 5;
-          break;
+      // The MMAs of k-block `kb` (held in ring stage `st`) for slabs
+      // [s_begin, s_end) into the accumulator at `d_tmem`.
+      auto issue = [&](uint32_t d_tmem, int st, int kb, int s_begin, int s_end) {
+        const uint32_t a_addr = smem_u32(smA + st * Cfg::kABytes);
+        const uint32_t b_addr = smem_u32(smB + st * Cfg::kBBytes);
+#pragma unroll
+        for (int k = 0; k < kBK / kUmmaK; ++k) {
+          const uint64_t bdesc = operand_desc(b_addr, k, !tb, Cfg::kBChunk);
+#pragma unroll
+          for (int s = 0; s < SLABS; ++s) {
+            if (s < s_begin || s >= s_end) continue;
+            const uint64_t adesc = operand_desc(a_addr + s * Cfg::kSlabBytes, k, ta, Cfg::kBChunk);
+            umma_f16_pair(d_tmem + static_cast<uint32_t>(s * BN), adesc, bdesc, idesc,
+                          (kb | k) != 0 ? 1u : 0u);
+          }
         }
-        tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * SLABS * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
+      };
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        if constexpr (SLABS == 2) {
+          // One accumulator of two slabs; the epilogue hands each slab back on
+          // its own barrier (acc_empty[s]) as soon as it has read it.  The
+          // next tile's slab-0 MMAs start on the k-blocks already in the ring
+          // while slab 1 is still being drained; those stages are freed once
+          // their slab-1 MMAs have been issued too.
+          if (!mbar_wait(&acc_empty[0], acc_phase ^ 1u, abort_flag, timeout_ns)) {
             ok = false;
-            site = 6;
+            site = 5;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = smem_u32(smA + stage * Cfg::kABytes);
-          const uint32_t b_addr = smem_u32(smB + stage * Cfg::kBBytes);
-#pragma unroll
-          for (int k = 0; k < kBK / kUmmaK; ++k) {
-            const uint64_t bdesc = operand_desc(b_addr, k, !tb, Cfg::kBChunk);
-#pragma unroll
-            for (int s = 0; s < SLABS; ++s) {
-              const uint64_t adesc =
-                  operand_desc(a_addr + s * Cfg::kSlabBytes, k, ta, Cfg::kBChunk);
-              umma_f16_pair(d_tmem + static_cast<uint32_t>(s * BN), adesc, bdesc, idesc,
-                            (kb | k) != 0 ? 1u : 0u);
+          const int early = num_kb < STAGES ? num_kb : STAGES;
+          const int stage0 = stage;
+          for (int kb = 0; kb < early; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
+              ok = false;
+              site = 6;
+              break;
+            }
+            tc_fence_after_sync();
+            issue(tmem_base, stage, kb, 0, 1);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
             }
           }
-          umma_commit_pair(&empty[stage], 0x3);  // stage s free in both CTAs
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+          if (!ok) break;
+          if (!mbar_wait(&acc_empty[1], acc_phase ^ 1u, abort_flag, timeout_ns)) {
+            ok = false;
+            site = 7;
+            break;
           }
-        }
-        if (!ok) break;
-        umma_commit_pair(&acc_full[acc], 0x3);  // both epilogues may read
-        if (++acc == NBUF) {
-          acc = 0;
+          tc_fence_after_sync();
+          for (int kb = 0, st = stage0; kb < early; ++kb) {
+            issue(tmem_base, st, kb, 1, 2);
+            umma_commit_pair(&empty[st], 0x3);  // stage free in both CTAs
+            if (++st == STAGES) st = 0;
+          }
+          for (int kb = early; kb < num_kb; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
+              ok = false;
+              site = 6;
+              break;
+            }
+            tc_fence_after_sync();
+            issue(tmem_base, stage, kb, 0, 2);
+            umma_commit_pair(&empty[stage], 0x3);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit_pair(&acc_full[0], 0x3);  // both epilogues may read
           acc_phase ^= 1u;
+        } else {
+          if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, timeout_ns)) {
+            ok = false;
+            site = 5;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * SLABS * BN);
+          for (int kb = 0; kb < num_kb; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
+              ok = false;
+              site = 6;
+              break;
+            }
+            tc_fence_after_sync();
+            issue(d_tmem, stage, kb, 0, SLABS);
+            umma_commit_pair(&empty[stage], 0x3);  // stage s free in both CTAs
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit_pair(&acc_full[acc], 0x3);  // both epilogues may read
+          if (++acc == NBUF) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
         }
       }
       if (!ok) {
@@ -699,20 +762,19 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const uint32_t release_bar = acc_empty_leader + acc * 8;
 #pragma unroll 1
       for (int s = 0; s < SLABS; ++s) {
+        // two slabs (single accumulator): each slab has its own barrier and is
+        // handed back as soon as it has been read; one slab (two accumulator
+        // buffers): the buffer's barrier
+        const uint32_t release_bar = acc_empty_leader + (SLABS == 2 ? s : acc) * 8;
         const int row0 =
             mb * Cfg::kTileM + s * 2 * kBM + static_cast<int>(rank) * kBM + q * kEpiRows;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                static_cast<uint32_t>((acc * SLABS + s) * BN + g * kCols);
-        const bool last = (s == SLABS - 1);
-        // the accumulator buffer is handed back after its last slab is read
         epilogue_tile<kCols, Cfg::kEpiBoxes, ACT>(
             t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0, nb * BN + g * kCols, lane,
-            [release_bar, last] {
-              if (last) mbar_arrive_cluster(release_bar);
-            });
+            [release_bar] { mbar_arrive_cluster(release_bar); });
       }
       if (++acc == NBUF) {
         acc = 0;
