@@ -864,7 +864,9 @@ template <int STAGES, int SLABS, int ACT>
 int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
   using Cfg = PairCfg<STAGES, SLABS>;
   static std::atomic<uint64_t> attr_done{0};
-  static int max_pairs[64] = {};
+  // pairs that can be resident at once, per device (0 = not asked yet; racing
+  // first calls store the same value)
+  static std::atomic<int> max_pairs[64] = {};
   CUtensorMap tA, tB, tC;
   int rc = encode_operand_maps(p, kBM, 128, &tA, &tB);  // this CTA's half: 128 columns
   const uint64_t n8 = static_cast<uint64_t>(p.N) & ~7ull;
@@ -886,7 +888,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // pairs that can be resident at once (GPC layout may leave an SM unpaired)
-  int& resident = max_pairs[d.device & 63];
+  int resident = max_pairs[d.device & 63].load(std::memory_order_relaxed);
   if (resident == 0) {
     cfg.gridDim = dim3(2 * (d.sm_count / 2), 1, 1);
     int n = 0;
@@ -895,6 +897,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
       n = d.sm_count / 2;
     }
     resident = n;
+    max_pairs[d.device & 63].store(n, std::memory_order_relaxed);
   }
   const int64_t num_tiles = ((p.M + Cfg::kTileM - 1) / Cfg::kTileM) * ((p.N + 255) / 256);
   const int pairs = static_cast<int>(num_tiles < resident ? num_tiles : resident);
