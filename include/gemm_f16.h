@@ -73,7 +73,8 @@ enum gemm_path {
                               256 x 256 -> TILE; K < 3072 (6144 with GELU) -> TILE_PAIR;
                               otherwise TILE_PAIR_TALL, or TILE_PAIR when the 512-row
                               tiles leave a much emptier last wave */
-  GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile (any shape) */
+  GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile, BN = 64, 128 or
+                              256 by the tile count (any shape) */
   GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 128 columns of B per CTA when
                               ceil(N / 128) <= SMs, else 256, streamed in lock-step,
                               split-K only when tiles < SMs (M <= 64 only) */
@@ -144,8 +145,9 @@ GEMM_API int gemm_f16_general(const void* A, const void* B, const void* bias, vo
  * A field left at 0 takes the value GEMM_PATH_AUTO would use. */
 typedef struct gemm_config {
   int32_t kernel;     /* GEMM_PATH_TILE, _TILE_PAIR, _TILE_PAIR_TALL or _SKINNY (not AUTO) */
-  int32_t block_n;    /* output columns per tile: 128 or 256 for GEMM_PATH_TILE and
-                         GEMM_PATH_SKINNY; 256 (the only width) for the pair kernels */
+  int32_t block_n;    /* output columns per tile: 64, 128 or 256 for GEMM_PATH_TILE; 128
+                         or 256 for GEMM_PATH_SKINNY; 256 (the only width) for the pair
+                         kernels */
   int32_t stages;     /* depth of the shared-memory operand ring (k-blocks of 64 in flight) */
   int32_t group_rows; /* tile kernels: rows of op(A) per raster panel, the L2 grouping of
                          the tile order; 0 = 2048.  Must be 0 for GEMM_PATH_SKINNY */

@@ -153,7 +153,7 @@ def _raw(cfg, m=256, n=256, k=128, bias=False, act=ops.ACT_RELU):
 @pytest.mark.parametrize("cfg,m", [
     ({"kernel": 0}, 256),                                  # AUTO is not a kernel
     ({"kernel": 9}, 256),
-    ({"kernel": ops.PATH_TILE, "block_n": 64}, 256),
+    ({"kernel": ops.PATH_TILE, "block_n": 32}, 256),
     ({"kernel": ops.PATH_TILE, "stages": 2}, 256),         # not built
     ({"kernel": ops.PATH_TILE, "block_n": 256, "stages": 5}, 256),  # over the budget
     ({"kernel": ops.PATH_TILE_PAIR, "stages": 7}, 256),

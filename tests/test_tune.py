@@ -28,8 +28,8 @@ def test_built_configs_are_exactly_those_within_the_budget(lib):
             expect.add((kernel, bn, st))
     assert built == expect
     # the defaults are among them
-    for kernel, bn, st in ((1, 128, 6), (1, 256, 4), (3, 256, 6), (4, 256, 4), (2, 256, 4),
-                           (2, 128, 6)):
+    for kernel, bn, st in ((1, 64, 6), (1, 128, 6), (1, 256, 4), (3, 256, 6), (4, 256, 4),
+                           (2, 256, 4), (2, 128, 6)):
         assert (kernel, bn, st) in built
 
 
@@ -51,7 +51,8 @@ def test_smem_formula(lib):
     assert ops.config_smem_bytes({"kernel": 3}) == tile(32768, 6)
     assert ops.config_smem_bytes({"kernel": 0}) == -8
     assert ops.config_smem_bytes({"kernel": 1, "block_n": 0}) == -8
-    assert ops.config_smem_bytes({"kernel": 1, "block_n": 64}) == -8
+    assert ops.config_smem_bytes({"kernel": 1, "block_n": 32}) == -8
+    assert ops.config_smem_bytes({"kernel": 1, "block_n": 64, "stages": 8}) == tile(24576, 8)
     assert ops.config_smem_bytes({"kernel": 4, "block_n": 128}) == -8
 
 
@@ -67,7 +68,8 @@ def test_candidates_cube(lib):
     assert all("shared memory" in why for _, why in pruned)
     assert len({tuple(sorted(c.items())) for c in kept}) == len(kept)
     # panels: 1, 2, 4, ... tile-rows up to the whole column (64 rows of 128)
-    panels = sorted({c["group_rows"] for c in kept if c["kernel"] == ops.PATH_TILE})
+    panels = sorted({c["group_rows"] for c in kept
+                     if c["kernel"] == ops.PATH_TILE and c["block_n"] == 128})
     assert panels == [128 * g for g in (1, 2, 4, 8, 16, 32, 64)]
     tall = sorted({c["group_rows"] for c in kept if c["kernel"] == ops.PATH_TILE_PAIR_TALL})
     assert tall == [512 * g for g in (1, 2, 4, 8, 16)]

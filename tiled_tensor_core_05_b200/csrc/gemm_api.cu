@@ -387,7 +387,9 @@ int select_path_for(int64_t M, int64_t N, int64_t K, int sm_count, int activatio
 
 int default_stages(int kernel, int block_n) {
   switch (kernel) {
-    case GEMM_PATH_TILE: return block_n == 256 ? kDefaultStagesTile256 : kDefaultStagesTile128;
+    case GEMM_PATH_TILE:
+      return block_n == 256 ? kDefaultStagesTile256
+                            : (block_n == 64 ? kDefaultStagesTile64 : kDefaultStagesTile128);
     case GEMM_PATH_TILE_PAIR: return kDefaultStagesPair;
     case GEMM_PATH_TILE_PAIR_TALL: return kDefaultStagesTall;
     case GEMM_PATH_SKINNY: return block_n == 128 ? kDefaultStagesSkinnyNarrow : kDefaultStagesSkinny;
@@ -404,11 +406,13 @@ int resolve_config(KernelConfig& c, int64_t M, int64_t N, int sm_count) {
     case GEMM_PATH_TILE:
       if (c.block_n == 0) {
         // 128 x 256 tiles when there are enough of them to fill the GPU,
-        // otherwise 128 x 128 tiles (twice as many CTAs for small problems)
+        // otherwise 128 x 128 tiles (twice as many CTAs for small problems),
+        // or 128 x 64 tiles when even those would fill at most half the SMs
         const int64_t tiles256 = ((M + 127) / 128) * ((N + 255) / 256);
-        c.block_n = tiles256 >= sm_count ? 256 : 128;
+        const int64_t tiles128 = ((M + 127) / 128) * ((N + 127) / 128);
+        c.block_n = tiles256 >= sm_count ? 256 : (2 * tiles128 <= sm_count ? 64 : 128);
       }
-      if (c.block_n != 128 && c.block_n != 256) return GEMM_ERR_CONFIG;
+      if (c.block_n != 64 && c.block_n != 128 && c.block_n != 256) return GEMM_ERR_CONFIG;
       break;
     case GEMM_PATH_TILE_PAIR:
     case GEMM_PATH_TILE_PAIR_TALL:

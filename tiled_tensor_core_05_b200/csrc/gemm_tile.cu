@@ -116,6 +116,8 @@ struct TileVariant {
   int stages;
 };
 constexpr TileVariant kTileVariants[] = {
+    {GEMM_PATH_TILE, 64, 3},       {GEMM_PATH_TILE, 64, 4},       {GEMM_PATH_TILE, 64, 5},
+    {GEMM_PATH_TILE, 64, 6},       {GEMM_PATH_TILE, 64, 7},       {GEMM_PATH_TILE, 64, 8},
     {GEMM_PATH_TILE, 128, 3},      {GEMM_PATH_TILE, 128, 4},      {GEMM_PATH_TILE, 128, 5},
     {GEMM_PATH_TILE, 128, 6},      {GEMM_PATH_TILE, 256, 3},      {GEMM_PATH_TILE, 256, 4},
     {GEMM_PATH_TILE_PAIR, 256, 3}, {GEMM_PATH_TILE_PAIR, 256, 4}, {GEMM_PATH_TILE_PAIR, 256, 5},
@@ -125,7 +127,7 @@ constexpr int kNumTileVariants = sizeof(kTileVariants) / sizeof(kTileVariants[0]
 
 constexpr int variant_smem_bytes(int kernel, int block_n, int stages) {
   return kernel == GEMM_PATH_TILE
-             ? (block_n == 128 || block_n == 256
+             ? (block_n == 64 || block_n == 128 || block_n == 256
                     ? tile_smem_formula(single_stage_bytes(block_n), stages)
                     : -1)
          : block_n != 256                       ? -1
@@ -136,7 +138,7 @@ constexpr int variant_smem_bytes(int kernel, int block_n, int stages) {
 
 // The table holds exactly the depths from 3 to the budget's limit.
 constexpr bool variants_complete() {
-  const int kinds[4][2] = {{GEMM_PATH_TILE, 128}, {GEMM_PATH_TILE, 256},
+  const int kinds[5][2] = {{GEMM_PATH_TILE, 64}, {GEMM_PATH_TILE, 128}, {GEMM_PATH_TILE, 256},
                            {GEMM_PATH_TILE_PAIR, 256}, {GEMM_PATH_TILE_PAIR_TALL, 256}};
   for (const auto& k : kinds) {
     for (int st = 3; st <= 16; ++st) {

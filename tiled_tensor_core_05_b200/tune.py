@@ -13,7 +13,7 @@ times or picks among configurations at run time.  Its GEMM_PATH_AUTO rules and
 defaults are set from the table this script writes.
 
 For each workload:
-  1. the candidate space: every tile shape (128 x 128 and 128 x 256 on one SM,
+  1. the candidate space: every tile shape (128 x 64, 128 x 128 and 128 x 256 on one SM,
      256 x 256 and 512 x 256 on a CTA pair, the 128- and 256-column small-M
      kernel when M <= 64) x ring depths 3..8 x raster panels (1, 2, 4, ...
      tile-rows, up to all of them) or k-slices;
@@ -50,8 +50,8 @@ from .workloads import WORKLOADS, Workload, make_inputs
 
 SMEM_BUDGET = 232448  # bytes of dynamic shared memory a CTA may opt into (sm_100)
 STAGE_RANGE = range(3, 9)
-TILE_KINDS = [(ops.PATH_TILE, 128), (ops.PATH_TILE, 256), (ops.PATH_TILE_PAIR, 256),
-              (ops.PATH_TILE_PAIR_TALL, 256)]
+TILE_KINDS = [(ops.PATH_TILE, 64), (ops.PATH_TILE, 128), (ops.PATH_TILE, 256),
+              (ops.PATH_TILE_PAIR, 256), (ops.PATH_TILE_PAIR_TALL, 256)]
 TILE_ROWS = {ops.PATH_TILE: 128, ops.PATH_TILE_PAIR: 256, ops.PATH_TILE_PAIR_TALL: 512}
 KERNEL_NAMES = {ops.PATH_TILE: "tile", ops.PATH_SKINNY: "skinny",
                 ops.PATH_TILE_PAIR: "pair", ops.PATH_TILE_PAIR_TALL: "pair-tall"}
