@@ -28,7 +28,7 @@ def test_built_configs_are_exactly_those_within_the_budget(lib):
             expect.add((kernel, bn, st))
     assert built == expect
     # the defaults are among them
-    for kernel, bn, st in ((1, 64, 6), (1, 128, 6), (1, 256, 4), (3, 256, 6), (4, 256, 4),
+    for kernel, bn, st in ((1, 64, 4), (1, 128, 6), (1, 256, 4), (3, 256, 6), (4, 256, 4),
                            (2, 256, 4), (2, 128, 6)):
         assert (kernel, bn, st) in built
 

@@ -34,7 +34,7 @@ constexpr int kMaxDynamicSmem = 232448;
 
 // Defaults used by GEMM_PATH_AUTO and by a gemm_config field left at 0.
 constexpr int kDefaultGroupRows = 2048;
-constexpr int kDefaultStagesTile64 = 6;
+constexpr int kDefaultStagesTile64 = 4;
 constexpr int kDefaultStagesTile128 = 6;
 constexpr int kDefaultStagesTile256 = 4;
 constexpr int kDefaultStagesPair = 6;
