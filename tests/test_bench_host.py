@@ -1,0 +1,109 @@
+"""Host-side logic of bench.py that needs no GPU: the unit of each workload,
+the roofline arithmetic and the traffic lookup, the clock summary, and the
+JSON line of the reference arm (the CPU oracle) on a small workload."""
+import io
+import json
+import os
+import sys
+import time
+from contextlib import redirect_stdout
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from tiled_tensor_core_05_b200 import workloads  # noqa: E402
+from tiled_tensor_core_05_b200.clocks import ClockSampler  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_tensor_core_05_b200 import build, ops
+    build.build()
+    return ops.lib()
+
+
+def test_units_follow_the_shape():
+    for name, w in workloads.WORKLOADS.items():
+        assert bench.hbm_bound(w) == (w.M <= 64), name
+
+
+def test_roofline_arithmetic(lib):
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    w = workloads.WORKLOADS["cube8192"]
+    r = bench.roofline_entry("cube8192", 1.0, peaks, "measured", long_run=False)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(w.flops / 1e-3 / 1e12, rel=1e-4)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1600.0, rel=1e-3)
+    assert r["kernel"] == "tile_pair_gemm_kernel"
+    r = bench.roofline_entry("cube8192", 1.0, peaks, "measured", long_run=True)
+    assert r["peak"] == 1400.0
+    d = workloads.WORKLOADS["decode"]
+    r = bench.roofline_entry("decode", 0.1, peaks, "measured", long_run=False)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(d.bytes_min / 1e-4 / 1e9, rel=1e-4)
+    assert d.bytes_min == 472121344
+    assert r["kernel"] == "skinny_gemm_kernel"
+
+
+def test_traffic_is_reported_only_for_the_captured_source(lib, tmp_path, monkeypatch):
+    entry = bench.traffic_for("cube8192", "tile_pair_gemm_kernel")
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        table = json.load(f)
+    rec = table["tile_pair_gemm_kernel/cube8192"]
+    if rec["kernel_src_sha"] == bench.kernel_source_hash("tile_pair_gemm_kernel"):
+        assert entry == rec["dram_bytes_per_launch"]
+    else:
+        assert entry is None
+    # a changed source (another hash) hides the figure
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda k: "0" * 16)
+    assert bench.traffic_for("cube8192", "tile_pair_gemm_kernel") is None
+    assert bench.traffic_for("cube256", "tile_gemm_kernel") is None  # never captured
+
+
+def _sampler(samples, marks):
+    s = ClockSampler.__new__(ClockSampler)
+    s.samples, s.marks, s.ok, s.max_mhz = samples, marks, True, 1965
+    s.bits = [(name, 1 << i) for i, (name, _) in enumerate(ClockSampler.REASONS)]
+    return s
+
+
+def test_clock_summary_window_and_reasons():
+    t = 100.0
+    # (time, MHz, reason bits, W): power cap (bit 3) inside the window only
+    samples = [(t + 0.001 * i, 1965 if i < 10 else 1300, (1 << 3) if i >= 10 else 0, 500.0)
+               for i in range(30)]
+    s = _sampler(samples, {"warm0": t, "t0": t + 0.0095, "t1": t + 0.0295})
+    out = s.summary()
+    assert out["sm_mhz"] == 1300 and out["samples"] == 20
+    assert out["reasons"] == ["sw_power_cap"]
+    # a timed region too short for three samples falls back to warm-up + timed
+    s = _sampler(samples, {"warm0": t, "t0": t + 0.0155, "t1": t + 0.0165})
+    out = s.summary()
+    assert out["samples"] == 17 and "warm-up" in out["note"]
+
+
+def test_clock_summary_without_nvml():
+    s = ClockSampler.__new__(ClockSampler)
+    s.ok, s.err = False, "no NVML here"
+    out = s.summary()
+    assert out["sm_mhz"] is None and "NVML unavailable" in out["note"]
+
+
+def test_reference_arm_line(monkeypatch):
+    class Args:
+        workload, steps, warmup, gpus = "cube256", 2, 1, 1
+    monkeypatch.setenv("RANK", "0")
+    buf = io.StringIO()
+    t0 = time.time()
+    with redirect_stdout(buf):
+        assert bench.run_reference(Args) == 0
+    assert time.time() - t0 < 60
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["config"]["workload"] == "cube256" and line["gpu_launches"] == 0
+    assert line["higher_is_better"] is True and line["dtype"] == "f64"
