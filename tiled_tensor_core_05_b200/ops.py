@@ -8,7 +8,11 @@ the library is missing or the call fails, a ``RuntimeError`` is raised.
 The operation is C = ReLU(A @ B) (``gemm_relu_f16``) or C = A @ B
 (``gemm_f16``) on row-major fp16 matrices with fp32 accumulation, as in
 "Writing high-performance kernels in TileLang" (atlascloud.ai blog), section
-"Escribamos un GEMM".
+"Escribamos un GEMM"; ``gemm_bias_act_f16`` adds a per-column bias and GELU
+("TileLang simplifica la creación de kernels GPU de alto rendimiento",
+posicionamiento-web.ar, section "Fusionar operaciones para reducir viajes a
+memoria"), ``gemm_general`` the transposed operand layouts, and
+``gemm_config_run`` an explicit kernel configuration for offline tuning.
 """
 from __future__ import annotations
 
