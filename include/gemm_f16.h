@@ -81,7 +81,8 @@ enum gemm_path {
   GEMM_PATH_TILE_PAIR = 3, /* persistent kernel, two SMs (a CTA pair) per 256 x 256 tile
                               (any shape) */
   GEMM_PATH_TILE_PAIR_TALL = 4 /* persistent kernel, a CTA pair per 512 x 256 tile: fewer
-                                  bytes staged per MAC, epilogue not overlapped */
+                                  bytes staged per MAC; a single accumulator, so a tile's
+                                  epilogue overlaps only the start of the next tile */
 };
 
 enum gemm_activation {
