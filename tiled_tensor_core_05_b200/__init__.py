@@ -11,7 +11,8 @@ computes anything itself and raises if the library is missing.
     z = gemm_general(x, w_nk, bias, "relu", trans_b=True)  # w stored N x K
 
 ``tune`` is the offline configuration sweep (``python -m
-tiled_tensor_core_05_b200.tune``), ``build`` compiles the library in-tree.
+tiled_tensor_core_05_b200.tune``), ``shard`` the column-sharded product across
+ranks, ``build`` compiles the library in-tree.
 
 Importing this package does not load the library (so that ``workloads`` can be
 used on machines without a GPU); the first call does.
