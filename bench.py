@@ -13,6 +13,10 @@ stream; the job time is the max over ranks.  With N > 1 (torchrun, one rank
 per GPU) every rank runs its own independent replica of the problem (weak
 scaling, no collective on the data path).
 
+``e2e`` is the same metric through the host-buffer entry point
+``gemm_relu_f16_host``: page-locked host A and B in, C back in host memory,
+every step, with the library's copies pipelined against its kernels.
+
 ``--impl reference`` times the CPU oracle (the plain fp64 definition of the
 operation) on a bounded sample of the same workload on the host cores; under
 torchrun only rank 0 runs it.
@@ -221,26 +225,43 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
                                    per_launch=False)
         t_ms = t_total / steps
         res["torch_launch_ms"] = t_ms
-    if e2e:
-        # end to end through the C ABI: pinned host inputs -> device, the
-        # kernel, result -> pinned host, every step
+    if e2e and variant in ("relu", "bias_gelu"):
+        # end to end through the C ABI's host-buffer entry point: page-locked
+        # host A and B in, the kernels, C back in host memory, every step (the
+        # library pipelines the copies with the kernels panel by panel)
         a_h = a_cpu.pin_memory()
         b_h = b_cpu.pin_memory()
         c_h = torch.empty((w.M, w.N), dtype=torch.float16).pin_memory()
+        bias_h = None if bias is None else bias.cpu().pin_memory()
+        if bias_h is None:
+            hfn, hargs = lib.gemm_relu_f16_host, (a_h.data_ptr(), b_h.data_ptr(), c_h.data_ptr(),
+                                                  w.M, w.N, w.K, w.K, w.N, w.N, h)
+        else:
+            hfn, hargs = lib.gemm_f16_host, (a_h.data_ptr(), b_h.data_ptr(), bias_h.data_ptr(),
+                                             c_h.data_ptr(), w.M, w.N, w.K, w.K, w.N, w.N,
+                                             ops.ACT_GELU, h)
 
         def e2e_step():
-            a.copy_(a_h, non_blocking=True)
-            b.copy_(b_h, non_blocking=True)
-            step()
-            c_h.copy_(c, non_blocking=True)
+            rc = hfn(*hargs)
+            if rc != 0:
+                raise RuntimeError(f"host-buffer call failed: {ops.status_string(rc)}")
 
         e_steps = max(3, min(steps, 10))
         e_total, _ = time_launches(e2e_step, e_steps, 1, stream, dist, None, per_launch=False)
         res["e2e_ms"] = e_total / e_steps
-        res["h2d"] = a.numel() * 2 + b.numel() * 2
+        res["h2d"] = (a.numel() + b.numel() + (0 if bias is None else bias.numel())) * 2
         res["d2h"] = c.numel() * 2
-        if not torch.equal(c_h.view(torch.int16), c.cpu().view(torch.int16)):
-            raise RuntimeError("end-to-end result differs from the device result")
+        # the host result against the device result of the measured call:
+        # the panels may run other kernels, so the same tolerance as parity
+        step()
+        torch.cuda.synchronize()
+        dev = c.cpu()
+        res["e2e_bits_equal"] = bool(torch.equal(c_h.view(torch.int16), dev.view(torch.int16)))
+        if not res["e2e_bits_equal"]:
+            d, r = c_h.float(), dev.float()
+            if not bool(((d - r).abs() <= 1e-2 + 1e-2 * r.abs()).all()):
+                raise RuntimeError("end-to-end result differs from the device result")
+        res["e2e_plan"] = ops.host_plan(w.M, w.N, w.K)
     del a, b, c
     torch.cuda.empty_cache()
     return res
@@ -481,7 +502,9 @@ def run_ours(args):
             (w.bytes_min / (e_ms * 1e-3) / 1e9)
         line["e2e"] = {"value": round(world * ev, 2), "unit": unit,
                        "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"],
-                       "ms_per_step": round(e_ms, 4)}
+                       "ms_per_step": round(e_ms, 4),
+                       "call": "gemm_relu_f16_host" if args.variant == "relu" else "gemm_f16_host",
+                       "plan": main["e2e_plan"], "bits_equal_device": main["e2e_bits_equal"]}
     line["clocks"] = clocks
     if "torch_launch_ms" in main:
         t_ms = main["torch_launch_ms"]

@@ -247,6 +247,86 @@ GEMM_API int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_
                                    int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
                                    gemm_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Host-buffer entry points.  C = act(A @ B + bias), the operation of
+ * gemm_bias_act_f16 ("Writing high-performance kernels in TileLang",
+ * atlascloud.ai blog, section "Escribamos un GEMM"; the bias + activation
+ * epilogue of "TileLang simplifica la creación de kernels GPU de alto
+ * rendimiento", posicionamiento-web.ar, section "Fusionar operaciones para
+ * reducir viajes a memoria"), with A, B, bias and C in HOST memory.  The pages
+ * run the kernel on device tensors only; moving the data is an interface
+ * addition.
+ *
+ *   - A (M x K, lda >= K), B (K x N, ldb >= N) and C (M x N, ldc >= N) are
+ *     row-major fp16 host arrays, ld in elements; bias is N fp16 values or
+ *     NULL.  Host pointers have no alignment or ld rule (the library copies
+ *     them into 16-byte-aligned device rows).  Device or managed pointers are
+ *     refused with GEMM_ERR_INVALID_ARG.
+ *   - Page-locked host memory (cudaHostAlloc, cudaHostRegister, torch's
+ *     pin_memory) lets the copies run asynchronously and overlap one another
+ *     and the kernels.  Pageable memory gives the same result, but the driver
+ *     stages it and the call blocks for its copies.
+ *   - The library copies one operand whole and streams the other, and C, in
+ *     panels (the plan of gemm_host_plan_for): panel i's kernel runs on
+ *     `stream` as soon as its rows (or columns) are on the device, and its
+ *     part of C is copied back while later panels are still coming in.  The
+ *     kernel of each panel is the one GEMM_PATH_AUTO takes for the panel's
+ *     shape, so the bits may differ in the last place from one
+ *     gemm_bias_act_f16 over the whole problem (the same accuracy).
+ *   - Stream-ordered and asynchronous: the work starts after earlier work on
+ *     `stream`, later work on `stream` starts after C is in host memory, and
+ *     the call returns once everything is enqueued.  Read C, and reuse A, B
+ *     and bias, only after synchronising `stream`.
+ *   - Device memory: per (device, stream) the library keeps device copies of
+ *     A, B, C and bias (16-byte rows), two copy streams and their events,
+ *     allocated on first use and grown when a larger problem comes
+ *     (cudaMalloc; growing synchronises `stream` first), until
+ *     gemm_host_release() or process exit.  Not for use inside CUDA-graph
+ *     capture.  Calls on one stream from several host threads at once are
+ *     not supported.
+ *   - M == 0 or N == 0 is a no-op; K == 0 writes C = act(bias) (+0 without a
+ *     bias), and A and B are not read.
+ * Returns GEMM_OK or a negative gemm_status (GEMM_ERR_WORKSPACE when the
+ * device copies cannot be allocated). */
+GEMM_API int gemm_f16_host(const void* A, const void* B, const void* bias, void* C, int64_t M,
+                           int64_t N, int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                           int activation, gemm_stream_t stream);
+
+/* C = ReLU(A @ B) with host buffers: gemm_f16_host with no bias and
+ * GEMM_ACT_RELU, the signature of gemm_relu_f16. */
+GEMM_API int gemm_relu_f16_host(const void* A, const void* B, void* C, int64_t M, int64_t N,
+                                int64_t K, int64_t lda, int64_t ldb, int64_t ldc,
+                                gemm_stream_t stream);
+
+enum gemm_host_split {
+  GEMM_HOST_SPLIT_ROWS = 0, /* B copied whole; A and C in panels of rows */
+  GEMM_HOST_SPLIT_COLS = 1  /* A copied whole; B and C in panels of columns */
+};
+
+/* How gemm_f16_host splits an M x N x K problem. */
+typedef struct gemm_host_plan {
+  int32_t split;         /* a gemm_host_split value */
+  int32_t panels;        /* number of panels, 1..16 */
+  int64_t panel_extent;  /* rows (multiple of 512) or columns (multiple of 256) per panel,
+                            the last panel possibly fewer */
+  double estimate_bytes; /* the plan's copy-time estimate, as bytes over one direction of
+                            the host link: max(first + streamed + C / panels,
+                            first + streamed / panels + C) */
+} gemm_host_plan;
+
+/* The plan gemm_f16_host takes: of the two splits, the one with the smaller
+ * estimate (rows on a tie); panels of about 16 MiB of streamed bytes (operand
+ * + C), at most 16, whole 512-row or 256-column tiles each.  Pure host
+ * function.  Returns GEMM_OK, or GEMM_ERR_INVALID_ARG for a null `out`,
+ * M < 1, N < 1 or K < 0. */
+GEMM_API int gemm_host_plan_for(int64_t M, int64_t N, int64_t K, gemm_host_plan* out);
+
+/* Frees the device copies, copy streams and events of every (device, stream)
+ * gemm_f16_host has used, after synchronising each of those streams.  Not to
+ * be called while another thread is inside gemm_f16_host.  Returns GEMM_OK
+ * or GEMM_ERR_LAUNCH. */
+GEMM_API int gemm_host_release(void);
+
 /* y[i] = act(x[i]) for n fp32 values in device memory, with the exact code
  * the GEMM epilogues use (GELU: x * Phi(x), Phi from Abramowitz & Stegun
  * 7.1.26, |Phi error| <= 1e-6).  For checking the activations on their own.

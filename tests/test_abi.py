@@ -73,7 +73,7 @@ def test_path_selection(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gemm_abi_version() >= 10000
+    assert lib.gemm_abi_version() >= 10200
 
 
 def test_argument_errors_are_reported_before_any_device_work(lib):
@@ -86,3 +86,61 @@ def test_argument_errors_are_reported_before_any_device_work(lib):
     # empty output: a no-op, whatever the pointers
     assert lib.gemm_relu_f16(null, null, null, 0, 5, 5, 8, 8, 8, None) == 0
     assert lib.gemm_f16(null, null, null, 5, 0, 5, 8, 8, 8, None) == 0
+
+
+def test_host_entry_argument_errors_before_any_device_work(lib):
+    null = ctypes.c_void_p(0)
+    buf = (ctypes.c_uint16 * 64)()
+    assert lib.gemm_f16_host(null, null, null, null, -1, 4, 4, 4, 4, 4, 1, None) == -1
+    assert lib.gemm_f16_host(buf, buf, null, buf, 2, 2, 2, 2, 2, 2, 9, None) == -1  # activation
+    assert lib.gemm_relu_f16_host(null, null, null, 0, 5, 5, 5, 5, 5, None) == 0    # empty
+    assert lib.gemm_relu_f16_host(null, null, null, 5, 0, 5, 5, 5, 5, None) == 0
+    assert lib.gemm_relu_f16_host(null, buf, buf, 2, 2, 2, 2, 2, 2, None) == -1      # null A
+    assert lib.gemm_relu_f16_host(buf, buf, buf, 2, 4, 4, 3, 4, 4, None) == -1       # lda < K
+    assert lib.gemm_relu_f16_host(buf, buf, buf, 2, 4, 4, 4, 4, 3, None) == -1       # ldc < N
+    assert lib.gemm_relu_f16_host(buf, buf, buf, 1 << 31, 4, 4, 4, 4, 4, None) == -1
+
+
+PLAN_SHAPES = [(M, N, K) for M in (1, 32, 300, 1000, 4096, 8192, 20000)
+               for N in (1, 256, 1000, 14336, 28672) for K in (0, 64, 1000, 8192)]
+
+
+def test_host_plan_invariants(lib):
+    """The host-buffer plan: whole 512-row / 256-column panels, 1 to 16 of
+    them covering the split dimension exactly, an estimate that follows its
+    formula, never above the serial copy and never below either direction's
+    bytes."""
+    from tiled_tensor_core_05_b200 import ops
+    for M, N, K in PLAN_SHAPES:
+        p = ops.host_plan(M, N, K)
+        by_rows = p["split"] == ops.HOST_SPLIT_ROWS
+        dim, unit = (M, 512) if by_rows else (N, 256)
+        P, ext = p["panels"], p["panel_extent"]
+        assert 1 <= P <= 16, (M, N, K, p)
+        assert ext % unit == 0 or ext == dim, (M, N, K, p)
+        assert (P - 1) * ext < dim <= P * ext, (M, N, K, p)
+        a, b, c = 2.0 * M * K, 2.0 * K * N, 2.0 * M * N
+        first, streamed = (b, a) if by_rows else (a, b)
+        est = max(first + streamed + c / P, first + streamed / P + c)
+        assert p["estimate_bytes"] == pytest.approx(est, rel=1e-12), (M, N, K, p)
+        assert max(a + b, c) <= est * (1 + 1e-12) and est <= (a + b + c) * (1 + 1e-12)
+
+
+def test_host_plan_on_the_workloads(lib):
+    from tiled_tensor_core_05_b200 import ops
+    # the cube: B whole, A and C in 16 panels of 512 rows (the split is a tie)
+    p = ops.host_plan(8192, 8192, 8192)
+    assert (p["split"], p["panels"], p["panel_extent"]) == (ops.HOST_SPLIT_ROWS, 16, 512)
+    assert p["estimate_bytes"] == 2 * 8192 * 8192 * 2 + 8192 * 8192 * 2 / 16
+    # the MLP up-projection: C (224 MiB) dominates; A (64 MiB) whole first
+    p = ops.host_plan(8192, 14336, 4096)
+    assert (p["split"], p["panels"], p["panel_extent"]) == (ops.HOST_SPLIT_COLS, 14, 1024)
+    # decode: B is nearly everything; streamed in column panels behind A
+    p = ops.host_plan(32, 28672, 8192)
+    assert p["split"] == ops.HOST_SPLIT_COLS and p["panels"] == 16
+    # small problems: one panel
+    assert ops.host_plan(1000, 1000, 1000)["panels"] == 1
+    assert ops.host_plan(1, 1, 0)["panels"] == 1
+    for bad in ((0, 4, 4), (4, 0, 4), (4, 4, -1)):
+        with pytest.raises(RuntimeError):
+            ops.host_plan(*bad)

@@ -9,6 +9,7 @@ computes anything itself and raises if the library is missing.
     c = gemm_relu_f16(a, b)                        # ReLU(a @ b), a (M, K), b (K, N) fp16
     y = gemm_bias_act_f16(x, w, bias, "gelu")      # GELU(x @ w + bias)
     z = gemm_general(x, w_nk, bias, "relu", trans_b=True)  # w stored N x K
+    c_host = gemm_host(a_cpu, b_cpu)               # CPU tensors in and out, copies pipelined
 
 ``tune`` is the offline configuration sweep (``python -m
 tiled_tensor_core_05_b200.tune``), ``shard`` the column-sharded product across
@@ -22,7 +23,7 @@ from __future__ import annotations
 __all__ = ["gemm_relu_f16", "gemm_f16", "gemm_f16_ex", "gemm_bias_act_f16", "gemm_general",
            "gemm_config_run", "GemmConfig", "auto_config", "config_list", "config_smem_bytes",
            "activation_f32", "read_probe", "select_path", "device_status", "status_string",
-           "lib"]
+           "gemm_host", "host_plan", "host_release", "lib"]
 
 
 def __getattr__(name):

@@ -23,7 +23,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libttc05.so")
-SOURCES = ["gemm_api.cu", "gemm_tile.cu", "gemm_skinny.cu"]
+SOURCES = ["gemm_api.cu", "gemm_tile.cu", "gemm_skinny.cu", "gemm_host.cu"]
 HEADERS = ["sm100.cuh", "internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

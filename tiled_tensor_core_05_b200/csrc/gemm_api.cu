@@ -349,7 +349,7 @@ using namespace ttc;
 
 extern "C" {
 
-int gemm_abi_version(void) { return 10100; }
+int gemm_abi_version(void) { return 10200; }
 
 namespace ttc {
 namespace {

@@ -11,8 +11,9 @@ The operation is C = ReLU(A @ B) (``gemm_relu_f16``) or C = A @ B
 "Escribamos un GEMM"; ``gemm_bias_act_f16`` adds a per-column bias and GELU
 ("TileLang simplifica la creación de kernels GPU de alto rendimiento",
 posicionamiento-web.ar, section "Fusionar operaciones para reducir viajes a
-memoria"), ``gemm_general`` the transposed operand layouts, and
-``gemm_config_run`` an explicit kernel configuration for offline tuning.
+memoria"), ``gemm_general`` the transposed operand layouts, ``gemm_config_run`` an
+explicit kernel configuration for offline tuning, and ``gemm_host`` the same
+product on CPU (host) tensors, copied in and out by the library.
 """
 from __future__ import annotations
 
@@ -43,6 +44,17 @@ class GemmConfig(ctypes.Structure):
         return "GemmConfig(" + ", ".join(f"{k}={v}" for k, v in self.as_dict().items()) + ")"
 
 
+class HostPlan(ctypes.Structure):
+    """``gemm_host_plan`` of the C ABI: how ``gemm_f16_host`` splits a problem."""
+    _fields_ = [("split", ctypes.c_int32), ("panels", ctypes.c_int32),
+                ("panel_extent", ctypes.c_int64), ("estimate_bytes", ctypes.c_double)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+HOST_SPLIT_ROWS, HOST_SPLIT_COLS = 0, 1
+
 _SIGNATURES = {
     "gemm_relu_f16": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
                       ctypes.c_int),
@@ -72,6 +84,12 @@ _SIGNATURES = {
                               ctypes.c_int),
     "gemm_read_probe": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p],
                         ctypes.c_int),
+    "gemm_f16_host": ([ctypes.c_void_p] * 4 + [ctypes.c_int64] * 6 +
+                      [ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
+    "gemm_relu_f16_host": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
+                           ctypes.c_int),
+    "gemm_host_plan_for": ([ctypes.c_int64] * 3 + [ctypes.POINTER(HostPlan)], ctypes.c_int),
+    "gemm_host_release": ([], ctypes.c_int),
 }
 
 
@@ -325,3 +343,63 @@ def read_probe(buf: torch.Tensor, sink: torch.Tensor | None = None, stream=None)
         _check(lib().gemm_read_probe(buf.data_ptr(), n, sink.data_ptr(),
                                      _stream_handle(stream, buf.device)), "gemm_read_probe")
     return sink
+
+
+def _host_ld(t: torch.Tensor) -> int:
+    """Row stride in elements of a 2-D CPU fp16 tensor with contiguous columns
+    (any stride >= cols; a single row passes its column count)."""
+    if t.dim() != 2 or t.dtype != torch.float16 or t.is_cuda:
+        raise ValueError("expected a 2-D CPU float16 tensor")
+    if t.size(1) > 1 and t.stride(1) != 1:
+        raise ValueError("columns must be contiguous (stride(1) == 1)")
+    return int(t.stride(0)) if t.size(0) > 1 else int(t.size(1))
+
+
+def gemm_host(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None,
+              act: str | int = "relu", out: torch.Tensor | None = None, *, stream=None,
+              sync: bool = True) -> torch.Tensor:
+    """C = act(A @ B + bias) on CPU fp16 tensors (``gemm_f16_host``): the
+    library copies A, B and bias to the current CUDA device, runs its kernels
+    panel by panel while the copies stream, and copies C back into ``out``.
+    Page-locked tensors (``pin_memory()``) let the copies overlap; ``out``
+    defaults to a new page-locked tensor.  With ``sync=False`` the call only
+    enqueues the work on ``stream``: synchronise it before reading ``out``."""
+    M, K = a.shape
+    K2, N = b.shape
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    code = _ACTS[act] if isinstance(act, str) else int(act)
+    if bias is not None and (bias.dtype != torch.float16 or bias.is_cuda or
+                             bias.numel() != N or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous CPU fp16 tensor of N elements")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, pin_memory=True)
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be M x N")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    h = _stream_handle(stream, dev)
+    with torch.cuda.device(dev):
+        rc = lib().gemm_f16_host(a.data_ptr(), b.data_ptr(),
+                                 None if bias is None else bias.data_ptr(), out.data_ptr(),
+                                 M, N, K, _host_ld(a), _host_ld(b), _host_ld(out), code, h)
+        _check(rc, "gemm_f16_host")
+    if sync:
+        if stream is None:
+            torch.cuda.current_stream(dev).synchronize()
+        elif hasattr(stream, "synchronize"):
+            stream.synchronize()
+        else:  # a raw handle
+            torch.cuda.synchronize(dev)
+    return out
+
+
+def host_plan(M: int, N: int, K: int) -> dict:
+    """The split ``gemm_f16_host`` takes for an M x N x K problem (pure host)."""
+    p = HostPlan()
+    _check(lib().gemm_host_plan_for(M, N, K, ctypes.byref(p)), "gemm_host_plan_for")
+    return p.as_dict()
+
+
+def host_release() -> None:
+    """Free the device copies and copy streams ``gemm_host`` keeps."""
+    _check(lib().gemm_host_release(), "gemm_host_release")
