@@ -13,7 +13,9 @@
  * Conventions shared by every entry point
  *   - A, B, C are DEVICE pointers (cudaMalloc / torch CUDA memory) to IEEE
  *     binary16 storage on the current CUDA device.  Host pointers are rejected
- *     with GEMM_ERR_INVALID_ARG.
+ *     with GEMM_ERR_INVALID_ARG.  (The host-buffer entry points, gemm_f16_host
+ *     and its companions, take host pointers instead and state their own
+ *     rules.)
  *   - lda, ldb, ldc are row strides in ELEMENTS (lda >= K, ldb >= N, ldc >= N).
  *     Columns are contiguous.
  *   - Pointers must be 16-byte aligned and every ld a multiple of 8 elements
@@ -307,8 +309,9 @@ enum gemm_host_split {
 typedef struct gemm_host_plan {
   int32_t split;         /* a gemm_host_split value */
   int32_t panels;        /* number of panels, 1..16 */
-  int64_t panel_extent;  /* rows (multiple of 512) or columns (multiple of 256) per panel,
-                            the last panel possibly fewer */
+  int64_t panel_extent;  /* rows (multiple of 512) or columns (multiple of 256, at least
+                            2048) per panel, or all of M or N; the last panel possibly
+                            fewer */
   double estimate_bytes; /* the plan's copy-time estimate, as bytes over one direction of
                             the host link: max(first + streamed + C / panels,
                             first + streamed / panels + C) */
@@ -316,10 +319,24 @@ typedef struct gemm_host_plan {
 
 /* The plan gemm_f16_host takes: of the two splits, the one with the smaller
  * estimate (rows on a tie); panels of about 16 MiB of streamed bytes (operand
- * + C), at most 16, whole 512-row or 256-column tiles each.  Pure host
+ * + C), at most 16, whole 512-row or 256-column tiles each, and column panels
+ * at least 2048 columns wide (narrower strided copies are slow).  Pure host
  * function.  Returns GEMM_OK, or GEMM_ERR_INVALID_ARG for a null `out`,
  * M < 1, N < 1 or K < 0. */
 GEMM_API int gemm_host_plan_for(int64_t M, int64_t N, int64_t K, gemm_host_plan* out);
+
+/* gemm_f16_host with the caller's plan instead of gemm_host_plan_for's, for
+ * choosing plans offline (as gemm_f16_config does for kernels).  Only
+ * plan->split and plan->panel_extent are read: the split, and the rows or
+ * columns per panel (clamped to M or N).  GEMM_ERR_CONFIG when the split is
+ * not a gemm_host_split value, panel_extent < 1, a column panel is not a
+ * multiple of 8 columns (unless it covers all N), or there would be more
+ * than 16 panels; GEMM_ERR_INVALID_ARG for a null plan; otherwise as
+ * gemm_f16_host. */
+GEMM_API int gemm_f16_host_planned(const void* A, const void* B, const void* bias, void* C,
+                                   int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb,
+                                   int64_t ldc, int activation, const gemm_host_plan* plan,
+                                   gemm_stream_t stream);
 
 /* Frees the device copies, copy streams and events of every (device, stream)
  * gemm_f16_host has used, after synchronising each of those streams.  Not to

@@ -106,7 +106,8 @@ PLAN_SHAPES = [(M, N, K) for M in (1, 32, 300, 1000, 4096, 8192, 20000)
 
 
 def test_host_plan_invariants(lib):
-    """The host-buffer plan: whole 512-row / 256-column panels, 1 to 16 of
+    """The host-buffer plan: whole 512-row / 256-column panels (column panels
+    at least 2048 wide), 1 to 16 of
     them covering the split dimension exactly, an estimate that follows its
     formula, never above the serial copy and never below either direction's
     bytes."""
@@ -118,6 +119,7 @@ def test_host_plan_invariants(lib):
         P, ext = p["panels"], p["panel_extent"]
         assert 1 <= P <= 16, (M, N, K, p)
         assert ext % unit == 0 or ext == dim, (M, N, K, p)
+        assert by_rows or ext >= 2048 or ext == dim, (M, N, K, p)
         assert (P - 1) * ext < dim <= P * ext, (M, N, K, p)
         a, b, c = 2.0 * M * K, 2.0 * K * N, 2.0 * M * N
         first, streamed = (b, a) if by_rows else (a, b)
@@ -132,15 +134,32 @@ def test_host_plan_on_the_workloads(lib):
     p = ops.host_plan(8192, 8192, 8192)
     assert (p["split"], p["panels"], p["panel_extent"]) == (ops.HOST_SPLIT_ROWS, 16, 512)
     assert p["estimate_bytes"] == 2 * 8192 * 8192 * 2 + 8192 * 8192 * 2 / 16
-    # the MLP up-projection: C (224 MiB) dominates; A (64 MiB) whole first
+    # the MLP up-projection: C (224 MiB) dominates; A (64 MiB) whole first,
+    # then 2048-column panels (the narrowest column panel)
     p = ops.host_plan(8192, 14336, 4096)
-    assert (p["split"], p["panels"], p["panel_extent"]) == (ops.HOST_SPLIT_COLS, 14, 1024)
+    assert (p["split"], p["panels"], p["panel_extent"]) == (ops.HOST_SPLIT_COLS, 7, 2048)
     # decode: B is nearly everything; streamed in column panels behind A
     p = ops.host_plan(32, 28672, 8192)
-    assert p["split"] == ops.HOST_SPLIT_COLS and p["panels"] == 16
+    assert (p["split"], p["panels"], p["panel_extent"]) == (ops.HOST_SPLIT_COLS, 14, 2048)
     # small problems: one panel
     assert ops.host_plan(1000, 1000, 1000)["panels"] == 1
     assert ops.host_plan(1, 1, 0)["panels"] == 1
     for bad in ((0, 4, 4), (4, 0, 4), (4, 4, -1)):
         with pytest.raises(RuntimeError):
             ops.host_plan(*bad)
+
+
+def test_host_planned_rejects_bad_plans_before_device_work(lib):
+    from tiled_tensor_core_05_b200 import ops
+    buf = (ctypes.c_uint16 * 64)()
+    null = ctypes.c_void_p(0)
+
+    def call(split, extent, M=4, N=100):
+        p = ops.HostPlan(split=split, panels=0, panel_extent=extent, estimate_bytes=0.0)
+        return lib.gemm_f16_host_planned(buf, buf, null, buf, M, N, 4, 4, N, N, 1,
+                                         ctypes.byref(p), None)
+    assert call(2, 8) == -8                 # no such split
+    assert call(0, 0) == -8                 # empty panels
+    assert call(1, 12) == -8                # column panels must keep 16-byte device rows
+    assert call(0, 1, M=17) == -8           # 17 panels
+    assert lib.gemm_f16_host_planned(buf, buf, null, buf, 4, 4, 4, 4, 4, 4, 1, None, None) == -1

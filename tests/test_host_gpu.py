@@ -158,3 +158,18 @@ def test_host_rejects_device_memory():
     null = ctypes.c_void_p(0)
     assert ops.lib().gemm_relu_f16_host(null, c.data_ptr(), c.data_ptr(), 64, 64, 64, 64, 64,
                                         64, h) == -1
+
+
+@pytest.mark.parametrize("plan", [{"split": 0, "panel_extent": 1}, {"split": 0, "panel_extent": 700},
+                                  {"split": 1, "panel_extent": 8}, {"split": 1, "panel_extent": 1000},
+                                  {"split": 1, "panel_extent": 4096}],
+                         ids=["rows1", "rows700", "cols8", "cols1000", "cols-whole"])
+def test_host_planned(oracle_mod, plan):
+    """The caller's plan instead of the library's: one-row panels, panels of
+    8 columns (the narrowest the device rows allow), ragged last panels."""
+    M, N, K = (12, 96, 200) if plan["panel_extent"] in (1, 8) else (1500, 3000, 300)
+    a, b = inputs(M, N, K, seed=61)
+    bias = (torch.randn(N, generator=torch.Generator().manual_seed(62)) * 0.5).half()
+    out = ops.gemm_host(a.pin_memory(), b.pin_memory(), bias.pin_memory(), "gelu", plan=plan)
+    check_parity(out.numpy(), oracle_mod.gemm_bias_act(a, b, bias, "gelu"), False,
+                 f"host planned {plan}")

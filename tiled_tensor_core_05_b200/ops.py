@@ -89,6 +89,9 @@ _SIGNATURES = {
     "gemm_relu_f16_host": ([ctypes.c_void_p] * 3 + [ctypes.c_int64] * 6 + [ctypes.c_void_p],
                            ctypes.c_int),
     "gemm_host_plan_for": ([ctypes.c_int64] * 3 + [ctypes.POINTER(HostPlan)], ctypes.c_int),
+    "gemm_f16_host_planned": ([ctypes.c_void_p] * 4 + [ctypes.c_int64] * 6 +
+                              [ctypes.c_int, ctypes.POINTER(HostPlan), ctypes.c_void_p],
+                              ctypes.c_int),
     "gemm_host_release": ([], ctypes.c_int),
 }
 
@@ -357,13 +360,15 @@ def _host_ld(t: torch.Tensor) -> int:
 
 def gemm_host(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None,
               act: str | int = "relu", out: torch.Tensor | None = None, *, stream=None,
-              sync: bool = True) -> torch.Tensor:
+              sync: bool = True, plan: dict | None = None) -> torch.Tensor:
     """C = act(A @ B + bias) on CPU fp16 tensors (``gemm_f16_host``): the
     library copies A, B and bias to the current CUDA device, runs its kernels
     panel by panel while the copies stream, and copies C back into ``out``.
     Page-locked tensors (``pin_memory()``) let the copies overlap; ``out``
     defaults to a new page-locked tensor.  With ``sync=False`` the call only
-    enqueues the work on ``stream``: synchronise it before reading ``out``."""
+    enqueues the work on ``stream``: synchronise it before reading ``out``.
+    ``plan`` ({"split": 0 or 1, "panel_extent": n}) replaces the library's
+    own split (``gemm_f16_host_planned``)."""
     M, K = a.shape
     K2, N = b.shape
     if K != K2:
@@ -379,10 +384,15 @@ def gemm_host(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None
     dev = torch.device("cuda", torch.cuda.current_device())
     h = _stream_handle(stream, dev)
     with torch.cuda.device(dev):
-        rc = lib().gemm_f16_host(a.data_ptr(), b.data_ptr(),
-                                 None if bias is None else bias.data_ptr(), out.data_ptr(),
-                                 M, N, K, _host_ld(a), _host_ld(b), _host_ld(out), code, h)
-        _check(rc, "gemm_f16_host")
+        args = (a.data_ptr(), b.data_ptr(), None if bias is None else bias.data_ptr(),
+                out.data_ptr(), M, N, K, _host_ld(a), _host_ld(b), _host_ld(out), code)
+        if plan is None:
+            _check(lib().gemm_f16_host(*args, h), "gemm_f16_host")
+        else:
+            p = HostPlan(split=int(plan["split"]), panels=0,
+                         panel_extent=int(plan["panel_extent"]), estimate_bytes=0.0)
+            _check(lib().gemm_f16_host_planned(*args, ctypes.byref(p), h),
+                   "gemm_f16_host_planned")
     if sync:
         if stream is None:
             torch.cuda.current_stream(dev).synchronize()
