@@ -99,6 +99,19 @@ def test_pair_kernel_multi_tile(oracle_mod, m, n, k):
             check_parity(run(a, b, relu=relu, path=path), ref, relu, f"{path} {m}x{n}x{k}")
 
 
+@pytest.mark.parametrize("m,n,k", [(4600, 2300, 520), (8192, 14336, 256), (300, 1000, 130),
+                                   (100, 500, 64)])
+def test_tall_tile_last_wave_halves(oracle_mod, m, n, k):
+    """The 512-row pair tile splits the tiles of a sparse last wave into two
+    256-row halves: whole tiles followed by halves (81 and 896 tiles on 74
+    pairs), halves only (one wave of 2 or 1 tiles), a ragged last row of
+    tiles, and a half entirely below M (100 rows).  Compared in full."""
+    a, b = workloads.make_inputs(m, n, k, seed=5000 + m + n + k)
+    for relu in (True, False):
+        ref = oracle_mod.gemm_relu(a, b) if relu else oracle_mod.gemm(a, b)
+        check_parity(run(a, b, relu=relu, path=TALL), ref, relu, f"tall {m}x{n}x{k}")
+
+
 @pytest.mark.parametrize("m,n,k", [(m, n, k) for (m, n, k) in GRID if m <= 64] +
                          [(32, 129, 257), (64, 1000, 1000), (7, 4096, 65), (64, 2048, 4099),
                           (32, 256, 8192), (5, 600, 3000), (33, 520, 12000), (1, 64, 70000)])

@@ -501,7 +501,8 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
                           int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
-                          int layout, int group_m, int* status, uint64_t timeout_ns) {
+                          int layout, int group_m, int split_from, int* status,
+                          uint64_t timeout_ns) {
   using Cfg = PairCfg<STAGES, SLABS>;
   const bool ta = (layout & kLayoutTransA) != 0;
   const bool tb = (layout & kLayoutTransB) != 0;
@@ -532,6 +533,18 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + kBK - 1) / kBK;
   const int n8 = N & ~7;
+  // Work units: tiles [0, split_from) whole, then each tile from split_from
+  // on as two units of one 256-row slab (the host splits the tiles of a last
+  // wave that holds at most half as many tiles as there are pairs, so that
+  // wave takes about half a tile's time; split_from == num_tiles otherwise).
+  const int num_units = 2 * num_tiles - split_from;
+  // unit -> tile coordinates, first row of the unit and its slab count
+  auto unit_coords = [&](int u, int& mb, int& nb, int& row_base, int& slabs) {
+    const bool half = u >= split_from;
+    tile_coords(half ? split_from + (u - split_from) / 2 : u, num_m, num_n, group_m, mb, nb);
+    row_base = mb * Cfg::kTileM + (half ? ((u - split_from) & 1) * 2 * kBM : 0);
+    slabs = half ? 1 : SLABS;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -571,20 +584,22 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-        int mb, nb;
-        tile_coords(tile, num_m, num_n, group_m, mb, nb);
-        const int a_row = mb * Cfg::kTileM + static_cast<int>(rank) * kBM;  // slab 0
+      for (int unit = pair; unit < num_units && ok; unit += npairs) {
+        int mb, nb, row_base, slabs;
+        unit_coords(unit, mb, nb, row_base, slabs);
+        const int a_row = row_base + static_cast<int>(rank) * kBM;  // slab 0
         const int b_col = nb * BN + static_cast<int>(rank) * 128;
+        const uint32_t tx = 2u * static_cast<uint32_t>(slabs * Cfg::kSlabBytes + Cfg::kBBytes);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
+          if (leader) mbar_arrive_expect_tx(&full[stage], tx);
           const uint32_t bar = full_leader + stage * 8;
 #pragma unroll
           for (int s = 0; s < SLABS; ++s) {
+            if (s >= slabs) break;
             uint8_t* adst = smA + stage * Cfg::kABytes + s * Cfg::kSlabBytes;
             const int row = a_row + s * 2 * kBM;
             if (!ta) {
@@ -628,7 +643,8 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
-      uint32_t acc_phase = 0;
+      uint32_t acc_phase = 0;  // also the phase of acc_empty[0] with two slabs
+      uint32_t slab1_phase = 0;
       bool ok = true;
       int site = 0;
       const uint32_t idesc = idesc_f16_f32(2 * kBM, BN, ta, !tb);
@@ -649,7 +665,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
           }
         }
       };
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+      for (int unit = pair; unit < num_units && ok; unit += npairs) {
         if constexpr (SLABS == 2) {
           // One accumulator of two slabs; the epilogue hands each slab back on
           // its own barrier (acc_empty[s]) as soon as it has read it.  The
@@ -662,7 +678,10 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
             break;
           }
           tc_fence_after_sync();
-          const int early = num_kb < STAGES ? num_kb : STAGES;
+          // a half tile (a unit from split_from on) has slab 0 only: no early
+          // start, every k-block in the loop below
+          const bool whole = unit < split_from;
+          const int early = !whole ? 0 : (num_kb < STAGES ? num_kb : STAGES);
           const int stage0 = stage;
           for (int kb = 0; kb < early; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
@@ -678,17 +697,21 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
             }
           }
           if (!ok) break;
-          if (!mbar_wait(&acc_empty[1], acc_phase ^ 1u, abort_flag, timeout_ns)) {
-            ok = false;
-            site = 7;
-            break;
+          if (whole) {
+            if (!mbar_wait(&acc_empty[1], slab1_phase ^ 1u, abort_flag, timeout_ns)) {
+              ok = false;
+              site = 7;
+              break;
+            }
+            slab1_phase ^= 1u;
+            tc_fence_after_sync();
           }
-          tc_fence_after_sync();
           for (int kb = 0, st = stage0; kb < early; ++kb) {
             issue(tmem_base, st, kb, 1, 2);
             umma_commit_pair(&empty[st], 0x3);  // stage free in both CTAs
             if (++st == STAGES) st = 0;
           }
+          const int slab_end = whole ? 2 : 1;
           for (int kb = early; kb < num_kb; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
               ok = false;
@@ -696,7 +719,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
               break;
             }
             tc_fence_after_sync();
-            issue(tmem_base, stage, kb, 0, 2);
+            issue(tmem_base, stage, kb, 0, slab_end);
             umma_commit_pair(&empty[stage], 0x3);
             if (++stage == STAGES) {
               stage = 0;
@@ -752,9 +775,9 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk_no = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs) {
-      int mb, nb;
-      tile_coords(tile, num_m, num_n, group_m, mb, nb);
+    for (int unit = pair; unit < num_units; unit += npairs) {
+      int mb, nb, row_base, slabs;
+      unit_coords(unit, mb, nb, row_base, slabs);
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, timeout_ns) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -765,13 +788,12 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       }
       tc_fence_after_sync();
 #pragma unroll 1
-      for (int s = 0; s < SLABS; ++s) {
+      for (int s = 0; s < slabs; ++s) {
         // two slabs (single accumulator): each slab has its own barrier and is
         // handed back as soon as it has been read; one slab (two accumulator
         // buffers): the buffer's barrier
         const uint32_t release_bar = acc_empty_leader + (SLABS == 2 ? s : acc) * 8;
-        const int row0 =
-            mb * Cfg::kTileM + s * 2 * kBM + static_cast<int>(rank) * kBM + q * kEpiRows;
+        const int row0 = row_base + s * 2 * kBM + static_cast<int>(rank) * kBM + q * kEpiRows;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                static_cast<uint32_t>((acc * SLABS + s) * BN + g * kCols);
         epilogue_tile<kCols, Cfg::kEpiBoxes, ACT>(
@@ -902,14 +924,22 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
     max_pairs[d.device & 63].store(n, std::memory_order_relaxed);
   }
   const int64_t num_tiles = ((p.M + Cfg::kTileM - 1) / Cfg::kTileM) * ((p.N + 255) / 256);
-  const int pairs = static_cast<int>(num_tiles < resident ? num_tiles : resident);
+  // with the 512-row tile, a last wave of at most resident / 2 tiles runs as
+  // twice as many 256-row halves
+  int64_t split_from = num_tiles;
+  if constexpr (SLABS == 2) {
+    const int64_t rem = num_tiles % resident;
+    if (rem != 0 && 2 * rem <= resident) split_from = num_tiles - rem;
+  }
+  const int64_t units = 2 * num_tiles - split_from;
+  const int pairs = static_cast<int>(units < resident ? units : resident);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.numAttrs = 1 + pdl_attribute(&attr[1]);
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
-      static_cast<int>(p.K), p.layout, group_tiles(group_rows, Cfg::kTileM), d.status,
-      d.timeout_ns);
+      static_cast<int>(p.K), p.layout, group_tiles(group_rows, Cfg::kTileM),
+      static_cast<int>(split_from), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
