@@ -282,8 +282,9 @@ GEMM_API int gemm_relu_f16_noalloc(const void* A, const void* B, void* C, int64_
  *   - Device memory: per (device, stream) the library keeps device copies of
  *     A, B, C and bias (16-byte rows), two copy streams and their events,
  *     allocated on first use and grown when a larger problem comes
- *     (cudaMalloc; growing synchronises `stream` first), until
- *     gemm_host_release() or process exit.  Not for use inside CUDA-graph
+ *     (cudaMalloc; growing waits for the earlier calls' work first), until
+ *     gemm_host_release() or process exit.  A call's copies into them start
+ *     after the previous call on the same staging has finished with them.  Not for use inside CUDA-graph
  *     capture.  Calls on one stream from several host threads at once are
  *     not supported.
  *   - M == 0 or N == 0 is a no-op; K == 0 writes C = act(bias) (+0 without a
@@ -339,9 +340,10 @@ GEMM_API int gemm_f16_host_planned(const void* A, const void* B, const void* bia
                                    gemm_stream_t stream);
 
 /* Frees the device copies, copy streams and events of every (device, stream)
- * gemm_f16_host has used, after synchronising each of those streams.  Not to
- * be called while another thread is inside gemm_f16_host.  Returns GEMM_OK
- * or GEMM_ERR_LAUNCH. */
+ * gemm_f16_host has used, after waiting for the work of each one's last call
+ * (on the library's own copy stream and event: the callers' streams need not
+ * exist any more).  Not to be called while another thread is inside
+ * gemm_f16_host.  Returns GEMM_OK or GEMM_ERR_LAUNCH. */
 GEMM_API int gemm_host_release(void);
 
 /* y[i] = act(x[i]) for n fp32 values in device memory, with the exact code

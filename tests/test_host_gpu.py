@@ -173,3 +173,22 @@ def test_host_planned(oracle_mod, plan):
     out = ops.gemm_host(a.pin_memory(), b.pin_memory(), bias.pin_memory(), "gelu", plan=plan)
     check_parity(out.numpy(), oracle_mod.gemm_bias_act(a, b, bias, "gelu"), False,
                  f"host planned {plan}")
+
+
+def test_host_release_after_the_callers_stream_is_destroyed(oracle_mod):
+    """The staging of a stream the caller has since destroyed is freed (and a
+    later call on a new stream works) without the library touching the dead
+    handle."""
+    from cuda.bindings import runtime as rt
+    err, s = rt.cudaStreamCreateWithFlags(1)  # cudaStreamNonBlocking
+    assert err == rt.cudaError_t.cudaSuccess
+    handle = int(s)
+    a, b = inputs(200, 300, 100, seed=71)
+    out = torch.empty((200, 300), dtype=torch.float16).pin_memory()
+    ops.gemm_host(a.pin_memory(), b.pin_memory(), out=out, stream=handle, sync=False)
+    assert rt.cudaStreamSynchronize(s)[0] == rt.cudaError_t.cudaSuccess
+    assert rt.cudaStreamDestroy(s)[0] == rt.cudaError_t.cudaSuccess
+    check_parity(out.numpy(), oracle_mod.gemm_relu(a, b), True, "host on a raw stream")
+    ops.host_release()
+    out2 = ops.gemm_host(a.pin_memory(), b.pin_memory())
+    check_parity(out2.numpy(), oracle_mod.gemm_relu(a, b), True, "host after the stream died")

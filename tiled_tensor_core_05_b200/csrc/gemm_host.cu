@@ -95,12 +95,17 @@ bool is_host_memory(const void* p) {
 }
 
 // Staging of one (device, caller stream): device copies of A, B, C and the
-// bias (grow-only), two copy streams and the events that order them.
+// bias (grow-only), two copy streams and the events that order them.  Every
+// call ends with its device-to-host stream waiting for its last kernel, so
+// `join` (recorded there last) completes only once nothing of the call uses
+// the buffers any more; the next call's copies wait for it, and growing or
+// freeing the buffers waits for it, without touching the caller's stream
+// (whose handle may be gone by then).
 struct Staging {
   int device = -1;
   cudaStream_t user = nullptr;
   cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, tail = nullptr, join = nullptr;
   cudaEvent_t in[kMaxPanels] = {}, out[kMaxPanels] = {};
   void* buf[4] = {};  // A, B, C, bias
   size_t cap[4] = {};
@@ -110,6 +115,7 @@ struct Staging {
     if (cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&tail, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess)
       return false;
     for (int i = 0; i < kMaxPanels; ++i)
@@ -119,10 +125,11 @@ struct Staging {
     return true;
   }
 
-  // Frees everything; the caller's stream is synchronised first so that no
-  // enqueued copy or kernel still uses the buffers.
+  // Frees everything, once the last call's work is done.
   void release() {
-    if (device >= 0) cudaStreamSynchronize(user);
+    if (join != nullptr) cudaEventSynchronize(join);
+    if (h2d != nullptr) cudaStreamSynchronize(h2d);
+    if (d2h != nullptr) cudaStreamSynchronize(d2h);
     for (int i = 0; i < 4; ++i) {
       if (buf[i] != nullptr) cudaFree(buf[i]);
       buf[i] = nullptr;
@@ -134,19 +141,20 @@ struct Staging {
       in[i] = out[i] = nullptr;
     }
     if (fork != nullptr) cudaEventDestroy(fork);
+    if (tail != nullptr) cudaEventDestroy(tail);
     if (join != nullptr) cudaEventDestroy(join);
     if (h2d != nullptr) cudaStreamDestroy(h2d);
     if (d2h != nullptr) cudaStreamDestroy(d2h);
-    fork = join = nullptr;
+    fork = tail = join = nullptr;
     h2d = d2h = nullptr;
   }
 
-  // Buffer `i` of at least `bytes`.  Growing waits for the caller's stream,
-  // which every earlier call joined back into, before freeing the old one.
+  // Buffer `i` of at least `bytes`.  Growing waits for the earlier calls'
+  // work (their `join`) before freeing the old one.
   int reserve(int i, size_t bytes) {
     if (bytes == 0 || cap[i] >= bytes) return GEMM_OK;
     if (buf[i] != nullptr) {
-      if (cudaStreamSynchronize(user) != cudaSuccess) return GEMM_ERR_LAUNCH;
+      if (cudaEventSynchronize(join) != cudaSuccess) return GEMM_ERR_LAUNCH;
       cudaFree(buf[i]);
       buf[i] = nullptr;
       cap[i] = 0;
@@ -255,9 +263,11 @@ int run_host(const void* A, const void* B, const void* bias, void* C, int64_t M,
   const bool by_rows = plan.split == GEMM_HOST_SPLIT_ROWS;
   const int64_t dim = by_rows ? M : N;
 
-  // fork: both copy streams start after the caller's earlier work
+  // fork: both copy streams start after the caller's earlier work, and the
+  // copies into the buffers after the previous call's last use of them
   bool ok = cudaEventRecord(st->fork, user) == cudaSuccess &&
             cudaStreamWaitEvent(st->h2d, st->fork, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(st->h2d, st->join, 0) == cudaSuccess &&
             cudaStreamWaitEvent(st->d2h, st->fork, 0) == cudaSuccess;
   int gemm_rc = GEMM_OK;
   if (ok && bias != nullptr)
@@ -297,9 +307,12 @@ int run_host(const void* A, const void* B, const void* bias, void* C, int64_t M,
                  : copy2d(hC + lo * 2, ldc * 2, dC + lo, ldc_d * 2, ext * 2, M,
                           cudaMemcpyDeviceToHost, st->d2h) == cudaSuccess;
   }
-  // join, also after a failure, so that later work on the caller's stream
-  // stays ordered after whatever was enqueued
-  const bool joined = cudaEventRecord(st->join, st->d2h) == cudaSuccess &&
+  // join, also after a failure: the device-to-host stream waits for the
+  // last kernel enqueued on the caller's stream, `join` marks the end of
+  // everything, and later work on the caller's stream waits for it
+  const bool joined = cudaEventRecord(st->tail, user) == cudaSuccess &&
+                      cudaStreamWaitEvent(st->d2h, st->tail, 0) == cudaSuccess &&
+                      cudaEventRecord(st->join, st->d2h) == cudaSuccess &&
                       cudaStreamWaitEvent(user, st->join, 0) == cudaSuccess;
   if (gemm_rc != GEMM_OK) return gemm_rc;
   if (!ok || !joined) {
