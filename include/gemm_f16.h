@@ -37,6 +37,10 @@
  *     (device, stream) on first use (cudaMalloc; about 10 MB on a 148-SM GPU)
  *     and keeps until process exit.  Make that first call outside CUDA-graph
  *     capture.  Two calls on different streams never share a workspace.
+ *   - The device-pointer entry points can be captured in CUDA graphs once a
+ *     first call on the same device and stream has run outside the capture
+ *     (it creates the workspace and caches kernel attributes); replays read
+ *     the buffers' current contents.
  *   - No entry point throws; errors are negative return codes.
  */
 #ifndef TTC05_GEMM_F16_H
