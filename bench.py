@@ -78,16 +78,18 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_for(workload: str, kernel: str):
+def traffic_for(workload: str, kernel: str, variant: str = "relu"):
     """DRAM bytes (read + write) per launch from a committed ncu capture of
-    `kernel` on `workload`, if it was taken on the current sources (else None)."""
+    `kernel` on `workload` (and `variant`, other than the plain ReLU one), if
+    it was taken on the current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             table = json.load(f)
     except (OSError, ValueError):
         return None
-    e = table.get(f"{kernel}/{workload}")
+    key = f"{kernel}/{workload}" + ("" if variant == "relu" else f"/{variant}")
+    e = table.get(key)
     if not e or e.get("kernel_src_sha") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
@@ -280,7 +282,7 @@ def kernel_for(w) -> str:
             ops.PATH_TILE_PAIR_TALL: "tile_pair_gemm_kernel"}[ops.select_path(w.M, w.N, w.K)]
 
 
-def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool):
+def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool, variant: str = "relu"):
     from tiled_tensor_core_05_b200 import workloads
     w = workloads.WORKLOADS[name]
     kernel = kernel_for(w)
@@ -289,14 +291,14 @@ def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool):
         achieved = w.bytes_min / (launch_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_for(name, kernel),
+                "frac": round(achieved / peak, 4), "traffic": traffic_for(name, kernel, variant),
                 "kernel": kernel, "algorithmic_bytes_per_launch": w.bytes_min,
                 "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"}
     achieved = w.flops / (launch_ms * 1e-3) / 1e12
     key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
     peak = peaks.get(key, peaks["bf16_tflops"])
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4), "traffic": traffic_for(name, kernel),
+            "frac": round(achieved / peak, 4), "traffic": traffic_for(name, kernel, variant),
             "kernel": kernel, "algorithmic_flops_per_launch": w.flops,
             "peak_source": f"{peak_src} {key} (cuBLAS bf16; fp16 has the same nominal rate)"}
 
@@ -495,7 +497,7 @@ def run_ours(args):
     else:
         line["pct_of_dense_fp16_peak"] = round(100 * value / world / NOMINAL_FP16_TFLOPS, 2)
     line["roofline"] = roofline_entry(args.workload, main["launch_ms"], peaks, peak_src,
-                                      long_run)
+                                      long_run, args.variant)
     if "e2e_ms" in main:
         e_ms = main["e2e_ms"]
         ev = (w.flops / (e_ms * 1e-3) / 1e12) if unit == "TFLOP/s" else \
@@ -529,7 +531,8 @@ def run_ours(args):
             entry = {"workload": name, "variant": variant, "M": ow.M, "N": ow.N, "K": ow.K,
                      "ms_per_launch": round(r["launch_ms"], 5),
                      "tflops": round(ow.flops / (r["launch_ms"] * 1e-3) / 1e12, 2),
-                     "roofline": roofline_entry(name, r["launch_ms"], peaks, peak_src, False)}
+                     "roofline": roofline_entry(name, r["launch_ms"], peaks, peak_src, False,
+                                                variant)}
             if "torch_launch_ms" in r:
                 entry["context_torch_ms_per_call"] = round(r["torch_launch_ms"], 5)
             if hbm_bound(ow):

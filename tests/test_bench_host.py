@@ -63,6 +63,21 @@ def test_traffic_is_reported_only_for_the_captured_source(lib, tmp_path, monkeyp
     assert bench.traffic_for("cube256", "tile_gemm_kernel") is None  # never captured
 
 
+def test_traffic_is_keyed_by_variant(tmp_path, monkeypatch):
+    """A variant's line reads its own capture, never the plain ReLU one."""
+    table = {"k/w": {"kernel_src_sha": "s", "dram_bytes_per_launch": 1},
+             "k/w/bias_gelu": {"kernel_src_sha": "s", "dram_bytes_per_launch": 2}}
+    os.makedirs(tmp_path / "profiles")
+    with open(tmp_path / "profiles" / "traffic.json", "w") as f:
+        json.dump(table, f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda k: "s")
+    assert bench.traffic_for("w", "k") == 1
+    assert bench.traffic_for("w", "k", "relu") == 1
+    assert bench.traffic_for("w", "k", "bias_gelu") == 2
+    assert bench.traffic_for("w", "k", "wT") is None
+
+
 def _sampler(samples, marks):
     s = ClockSampler.__new__(ClockSampler)
     s.samples, s.marks, s.ok, s.max_mhz = samples, marks, True, 1965
