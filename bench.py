@@ -388,15 +388,35 @@ def stream_read_probe(gib: float = 2.0, steps: int = 20):
             "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
 
 
-def cpu_baseline(name, budget_s=10.0):
-    """The oracle timed on a bounded sample (leading rows) of the workload."""
+def parity_summary(got, ref) -> dict:
+    """Element-by-element comparison of fp16 results with the acceptance rule
+    of the tests: |got - ref| <= 1e-2 + 1e-2 |ref|, and got > 0 wherever
+    ref > 1e-2 (ReLU output)."""
+    import numpy as np
+    g = np.asarray(got, dtype=np.float16).astype(np.float64)
+    r = np.asarray(ref, dtype=np.float16).astype(np.float64)
+    err = np.abs(g - r)
+    bad = ~(err <= 1e-2 + 1e-2 * np.abs(r))  # NaN counts as out of tolerance
+    big = r > 1e-2
+    sign_bad = int(np.count_nonzero(big & ~(g > 0)))
+    rel = err[big] / r[big]
+    return {"elements": int(r.size), "max_abs_err": float(np.nanmax(err)) if r.size else 0.0,
+            "max_rel_err": float(rel.max()) if rel.size else 0.0,
+            "out_of_tolerance": int(np.count_nonzero(bad)), "sign_mismatches": sign_bad,
+            "pass": bool(not bad.any() and sign_bad == 0)}
+
+
+def cpu_baseline(name, budget_s=10.0, gpu_c=None):
+    """The oracle timed on a bounded sample (leading rows) of the workload.
+    With `gpu_c` (the measured call's result, on the device) the sample's
+    rows are also compared with the oracle's (`parity`)."""
     import oracle
     from tiled_tensor_core_05_b200 import workloads
     w = workloads.WORKLOADS[name]
     a, b = workloads.workload_inputs(name)
     rows = int(max(1, min(w.M, budget_s / oracle_seconds_per_row(oracle, a, b))))
     t0 = time.perf_counter()
-    oracle.gemm_relu(a[:rows], b)
+    ref = oracle.gemm_relu(a[:rows], b)
     dt = time.perf_counter() - t0
     flops = 2.0 * rows * w.N * w.K
     if hbm_bound(w):
@@ -405,9 +425,13 @@ def cpu_baseline(name, budget_s=10.0):
     else:
         value = flops / dt / 1e12
         unit = "TFLOP/s"
-    return {"value": value, "unit": unit, "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"first {rows} of {w.M} rows of C ({rows}x{w.N}x{w.K}), {dt:.1f} s",
-            "seconds": round(dt, 2)}
+    out = {"value": value, "unit": unit, "cores": oracle.max_threads(), "kind": "oracle",
+           "sample": f"first {rows} of {w.M} rows of C ({rows}x{w.N}x{w.K}), {dt:.1f} s",
+           "seconds": round(dt, 2)}
+    if gpu_c is not None:
+        out["parity"] = dict(parity_summary(gpu_c[:rows].cpu().numpy(), ref),
+                             rows=f"0-{rows - 1} of {w.M}")
+    return out
 
 
 # ------------------------------------------------------------------ arms ---
@@ -561,7 +585,9 @@ def run_ours(args):
         sus["note"] = "one GPU, back to back after the timed region (context, not the value)"
         line["sustained"] = sus
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget)
+        # the measured call's result (ReLU variants) against the oracle's rows
+        gpu_c = main["tensors"][2] if args.variant in ("relu", "wT") else None
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget, gpu_c)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()

@@ -122,3 +122,25 @@ def test_reference_arm_line(monkeypatch):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["config"]["workload"] == "cube256" and line["gpu_launches"] == 0
     assert line["higher_is_better"] is True and line["dtype"] == "f64"
+
+
+def test_parity_summary():
+    import numpy as np
+    ref = np.array([[0.0, 1.0, 2.0], [0.5, 0.0, 100.0]], dtype=np.float16)
+    s = bench.parity_summary(ref.copy(), ref)
+    assert s["pass"] and s["out_of_tolerance"] == 0 and s["max_abs_err"] == 0.0
+    assert s["elements"] == 6
+    got = ref.copy()
+    got[1, 2] = 100.5             # 0.5 off at |ref| = 100: within 1e-2 + 1e-2 * 100
+    s = bench.parity_summary(got, ref)
+    assert s["pass"] and s["max_abs_err"] == 0.5 and abs(s["max_rel_err"] - 0.005) < 1e-12
+    got[0, 1] = 1.5               # 0.5 off at 1.0: out of tolerance
+    s = bench.parity_summary(got, ref)
+    assert not s["pass"] and s["out_of_tolerance"] == 1
+    got = ref.copy()
+    got[1, 0] = 0.0               # a positive reference value clamped away
+    s = bench.parity_summary(got, ref)
+    assert not s["pass"] and s["sign_mismatches"] == 1
+    got = ref.copy()
+    got[0, 0] = np.nan
+    assert not bench.parity_summary(got, ref)["pass"]
