@@ -101,3 +101,23 @@ def test_describe():
                           "splits": 0}) == "pair-tall 512x256 st4 panel=2048"
     assert tune.describe({"kernel": 2, "block_n": 256, "stages": 5, "group_rows": 0,
                           "splits": 0}) == "skinny 256 st5 splits=auto"
+
+
+def test_host_plan_candidates():
+    from tiled_tensor_core_05_b200 import ops, tune
+    c = tune.host_plan_candidates(8192, 8192)
+    assert {"split": ops.HOST_SPLIT_ROWS, "panel_extent": 512} in c
+    assert {"split": ops.HOST_SPLIT_COLS, "panel_extent": 8192} in c
+    assert len(c) == len({(p["split"], p["panel_extent"]) for p in c})
+    for M, N in ((8192, 14336), (32, 28672), (1000, 1003), (7, 9)):
+        for p in tune.host_plan_candidates(M, N):
+            dim = M if p["split"] == ops.HOST_SPLIT_ROWS else N
+            assert 1 <= p["panel_extent"] <= dim
+            assert -(-dim // p["panel_extent"]) <= 16
+            if p["split"] == ops.HOST_SPLIT_COLS and p["panel_extent"] < dim:
+                assert p["panel_extent"] % 8 == 0
+    # decode: 1024-column panels would be 28 of them; rows collapse to one panel
+    d = tune.host_plan_candidates(32, 28672)
+    assert {"split": ops.HOST_SPLIT_COLS, "panel_extent": 1024} not in d
+    assert [p for p in d if p["split"] == ops.HOST_SPLIT_ROWS] == [
+        {"split": ops.HOST_SPLIT_ROWS, "panel_extent": 32}]

@@ -3,6 +3,12 @@ raster panel, split-K) for the fused fp16 GEMM + activation.
 
     python -m tiled_tensor_core_05_b200.tune [--workloads cube8192,mlp_up,...]
                                              [--steps 30] [--out table.md] [--json out.json]
+    python -m tiled_tensor_core_05_b200.tune --host [--workloads cube8192,mlp_up,decode]
+
+With --host the sweep is over the host-buffer entry point's panel plans
+(gemm_f16_host_planned: row or column panels of several widths, and the plan
+gemm_host_plan_for picks), with the host link's copy rates measured beside
+them (host-to-device alone, device-to-host alone, both at once).
 
 The tuning workflow of "TileLang simplifica la creación de kernels GPU de alto
 rendimiento" (posicionamiento-web.ar) and "TileLang explicado: kernels de IA
@@ -248,6 +254,153 @@ def sweep_workload(w: Workload, act: str, use_bias: bool, steps: int, rounds: in
 
 # ----------------------------------------------------------------- report ---
 
+# ------------------------------------------------------- host-buffer plans ---
+
+HOST_ROW_EXTENTS = (512, 1024, 2048, 4096)
+HOST_COL_EXTENTS = (1024, 2048, 4096, 8192)
+
+
+def host_plan_candidates(M: int, N: int, max_panels: int = 16) -> list[dict]:
+    """Row and column panel plans gemm_f16_host_planned accepts for an M x N
+    output: at most `max_panels` panels, column panels whole multiples of 8
+    columns; the single-panel plan of each split included."""
+    out, seen = [], set()
+    for split, dim, extents in ((ops.HOST_SPLIT_ROWS, M, HOST_ROW_EXTENTS + (M,)),
+                                (ops.HOST_SPLIT_COLS, N, HOST_COL_EXTENTS + (N,))):
+        for ext in extents:
+            ext = min(ext, dim)
+            if ext < 1 or -(-dim // ext) > max_panels or (split, ext) in seen:
+                continue
+            if split == ops.HOST_SPLIT_COLS and ext < dim and ext % 8:
+                continue
+            seen.add((split, ext))
+            out.append({"split": split, "panel_extent": ext})
+    return out
+
+
+def _events_ms(fn, reps: int, streams=()) -> float:
+    """Median over `reps` of one call of `fn` between CUDA events on the
+    current stream (side `streams` joined back in before the end event)."""
+    import torch
+    cur = torch.cuda.current_stream()
+    times = []
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(cur)
+        for st in streams:
+            st.wait_event(e0)
+        fn()
+        for st in streams:
+            ev = torch.cuda.Event()
+            ev.record(st)
+            cur.wait_event(ev)
+        e1.record(cur)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def sweep_host(w: Workload, steps: int, rounds: int, seed: int = 0, log=print) -> dict:
+    """Time every host-buffer plan for workload `w` (ReLU), after checking its
+    result against the device path's, and the host link's copy rates."""
+    import torch
+    a, b = make_inputs(w.M, w.N, w.K, w.seed, w.a_scale, w.b_scale)
+    a_h, b_h = a.pin_memory(), b.pin_memory()
+    c_h = torch.empty((w.M, w.N), dtype=torch.float16).pin_memory()
+    dev = ops.gemm_relu_f16(a.cuda(), b.cuda())
+    in_bytes = (a.numel() + b.numel()) * 2
+    out_bytes = c_h.numel() * 2
+    # the link: the same bytes as one call, in one direction or both at once
+    h_in = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(in_bytes, dtype=torch.uint8, device="cuda")
+    d_out = torch.empty(out_bytes, dtype=torch.uint8, device="cuda")
+    h_out = torch.empty(out_bytes, dtype=torch.uint8).pin_memory()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def h2d():
+        with torch.cuda.stream(s1):
+            d_in.copy_(h_in, non_blocking=True)
+
+    def d2h():
+        with torch.cuda.stream(s2):
+            h_out.copy_(d_out, non_blocking=True)
+
+    def both():
+        h2d()
+        d2h()
+    link = {"h2d_ms": _events_ms(h2d, 5, (s1,)), "d2h_ms": _events_ms(d2h, 5, (s2,)),
+            "both_ms": _events_ms(both, 5, (s1, s2))}
+    link["h2d_gbs"] = in_bytes / link["h2d_ms"] / 1e6
+    link["d2h_gbs"] = out_bytes / link["d2h_ms"] / 1e6
+    del h_in, d_in, d_out, h_out
+    plans = [None] + host_plan_candidates(w.M, w.N)
+    auto = ops.host_plan(w.M, w.N, w.K)
+    results = []
+    for plan in plans:
+        c_h.fill_(float("nan"))
+        ops.gemm_host(a_h, b_h, None, "relu", c_h, plan=plan)
+        ok, err = check(c_h.cuda(), dev.float(), "relu")
+        results.append({"plan": plan or {"split": auto["split"],
+                                         "panel_extent": auto["panel_extent"]},
+                        "auto": plan is None, "valid": ok, "max_abs_err": err, "ms": []})
+    rng = random.Random(seed)
+    order = [i for i, r in enumerate(results) if r["valid"]]
+    for _ in range(rounds):
+        rng.shuffle(order)
+        for i in order:
+            plan = plans[i]
+            results[i]["ms"].append(_events_ms(
+                lambda: ops.gemm_host(a_h, b_h, None, "relu", c_h, sync=False, plan=plan),
+                steps))
+    for r in results:
+        r["median_ms"] = statistics.median(r["ms"]) if r["ms"] else None
+    serial = {}
+    da, db = a.cuda(), b.cuda()
+    dc = torch.empty_like(dev)
+
+    def serial_call():
+        da.copy_(a_h, non_blocking=True)
+        db.copy_(b_h, non_blocking=True)
+        ops.gemm_relu_f16(da, db, dc)
+        c_h.copy_(dc, non_blocking=True)
+    serial["ms"] = _events_ms(serial_call, steps)
+    log(f"{w.name}: link {link}, serial {serial['ms']:.3f} ms")
+    return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "in_bytes": in_bytes,
+            "out_bytes": out_bytes, "link": link, "serial_ms": serial["ms"], "auto": auto,
+            "plans": results}
+
+
+def host_markdown(reports: list[dict], command: str, device: str) -> str:
+    lines = [f"# Host-buffer plan sweep ({device})", "", f"Command: `{command}`", ""]
+    for r in reports:
+        k = r["link"]
+        lines += [f"## {r['workload']} ({r['M']} x {r['N']} x {r['K']}, ReLU)", "",
+                  f"Link: {r['in_bytes'] / 2**20:.0f} MiB host-to-device alone "
+                  f"{k['h2d_ms']:.3f} ms ({k['h2d_gbs']:.1f} GB/s); "
+                  f"{r['out_bytes'] / 2**20:.0f} MiB device-to-host alone {k['d2h_ms']:.3f} ms "
+                  f"({k['d2h_gbs']:.1f} GB/s); both at once {k['both_ms']:.3f} ms.  "
+                  f"Serial copies and kernel on one stream: {r['serial_ms']:.3f} ms.", "",
+                  "| plan | panels | valid | median ms | rounds min-max | TFLOP/s |",
+                  "|---|---|---|---|---|---|"]
+        flops = 2.0 * r["M"] * r["N"] * r["K"]
+        rows = sorted(r["plans"], key=lambda p: p["median_ms"] or float("inf"))
+        for p in rows:
+            pl = p["plan"]
+            dim = r["M"] if pl["split"] == ops.HOST_SPLIT_ROWS else r["N"]
+            name = ("rows" if pl["split"] == ops.HOST_SPLIT_ROWS else "cols") + \
+                f" {pl['panel_extent']}" + (" (AUTO)" if p["auto"] else "")
+            if p["median_ms"] is None:
+                lines.append(f"| {name} | {-(-dim // pl['panel_extent'])} | no | - | - | - |")
+                continue
+            lines.append(f"| {name} | {-(-dim // pl['panel_extent'])} | yes | "
+                         f"{p['median_ms']:.3f} | {min(p['ms']):.3f}-{max(p['ms']):.3f} | "
+                         f"{flops / (p['median_ms'] * 1e-3) / 1e12:.1f} |")
+        lines.append("")
+    return "\n".join(lines)
+
+
 def _rate(w_shape, ms, skinny_like: bool):
     M, N, K = w_shape
     if skinny_like:
@@ -318,10 +471,28 @@ def main(argv=None):
     ap.add_argument("--leaders", type=int, default=6)
     ap.add_argument("--out", default=None, help="write the markdown table here")
     ap.add_argument("--json", default=None, help="write all results as JSON here")
+    ap.add_argument("--host", action="store_true",
+                    help="sweep the host-buffer entry point's panel plans instead")
     args = ap.parse_args(argv)
     import torch
     if not torch.cuda.is_available():
         raise SystemExit("the sweep needs a CUDA device")
+    if args.host:
+        names = (args.workloads or "cube8192,mlp_up,decode").split(",")
+        reports = [sweep_host(WORKLOADS[n], args.steps, args.rounds, seed=i,
+                              log=lambda *x: print(*x, file=sys.stderr, flush=True))
+                   for i, n in enumerate(names)]
+        command = "python -m tiled_tensor_core_05_b200.tune " + " ".join(argv or sys.argv[1:])
+        md = host_markdown(reports, command.strip(), torch.cuda.get_device_name())
+        if args.out:
+            with open(args.out, "w") as f:
+                f.write(md)
+        else:
+            print(md)
+        if args.json:
+            with open(args.json, "w") as f:
+                json.dump(reports, f, indent=1)
+        return
     plan = DEFAULT_SWEEP
     if args.workloads:
         plan = []
