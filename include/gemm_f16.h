@@ -323,7 +323,7 @@ typedef struct gemm_host_plan {
 } gemm_host_plan;
 
 /* The plan gemm_f16_host takes: of the two splits, the one with the smaller
- * estimate (rows on a tie); panels of about 16 MiB of streamed bytes (operand
+ * estimate (rows on a tie); panels of about 32 MiB of streamed bytes (operand
  * + C), at most 16, whole 512-row or 256-column tiles each, and column panels
  * at least 2048 columns wide (narrower strided copies are slow).  Pure host
  * function.  Returns GEMM_OK, or GEMM_ERR_INVALID_ARG for a null `out`,

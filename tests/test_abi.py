@@ -130,10 +130,10 @@ def test_host_plan_invariants(lib):
 
 def test_host_plan_on_the_workloads(lib):
     from tiled_tensor_core_05_b200 import ops
-    # the cube: B whole, A and C in 16 panels of 512 rows (the split is a tie)
+    # the cube: B whole, A and C in 8 panels of 1024 rows (the split is a tie)
     p = ops.host_plan(8192, 8192, 8192)
-    assert (p["split"], p["panels"], p["panel_extent"]) == (ops.HOST_SPLIT_ROWS, 16, 512)
-    assert p["estimate_bytes"] == 2 * 8192 * 8192 * 2 + 8192 * 8192 * 2 / 16
+    assert (p["split"], p["panels"], p["panel_extent"]) == (ops.HOST_SPLIT_ROWS, 8, 1024)
+    assert p["estimate_bytes"] == 2 * 8192 * 8192 * 2 + 8192 * 8192 * 2 / 8
     # the MLP up-projection: C (224 MiB) dominates; A (64 MiB) whole first,
     # then 2048-column panels (the narrowest column panel)
     p = ops.host_plan(8192, 14336, 4096)

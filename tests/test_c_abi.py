@@ -42,7 +42,7 @@ def test_c_program_links_and_runs(program):
     assert lines["entry_points"] == f"{len(declared)} missing 0"
     assert int(lines["abi"]) >= 10200
     assert lines["path_cube"] == f"{ops.PATH_TILE_PAIR_TALL} path_decode {ops.PATH_SKINNY}"
-    assert lines["plan"] == "rc 0 split 0 panels 16 extent 512"
+    assert lines["plan"] == "rc 0 split 0 panels 8 extent 1024"
     smem, configs = lines["smem"].split(" configs ")
     assert 0 < int(smem) <= 232448 and int(configs) == len(ops.config_list())
     assert lines["bad_size"] == "-1 empty 0"

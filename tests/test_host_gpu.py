@@ -61,7 +61,7 @@ def test_host_small_full(oracle_mod, shape, pinned, relu):
     check_parity(out.numpy(), ref, relu, f"host {shape}")
 
 
-@pytest.mark.parametrize("shape", [(9000, 2048, 1000), (2048, 10000, 520), (40, 70000, 1000)],
+@pytest.mark.parametrize("shape", [(20000, 2048, 1000), (2048, 24000, 520), (40, 70000, 1000)],
                          ids=["row-panels", "col-panels", "col-panels-small-M"])
 def test_host_panels_full(oracle_mod, shape):
     """Several panels with a ragged last one, compared in full."""
@@ -74,7 +74,7 @@ def test_host_panels_full(oracle_mod, shape):
     check_parity(out.numpy(), oracle_mod.gemm_relu(a, b), True, f"host panels {shape}")
 
 
-@pytest.mark.parametrize("shape", [(1000, 1000, 1000), (9000, 2048, 1000), (2048, 10000, 520)],
+@pytest.mark.parametrize("shape", [(1000, 1000, 1000), (20000, 2048, 1000), (2048, 24000, 520)],
                          ids=["one-panel", "row-panels", "col-panels"])
 def test_host_bias_gelu(oracle_mod, shape):
     M, N, K = shape

@@ -40,7 +40,7 @@ constexpr int64_t kColUnit = 256;  // columns of the widest tile
 // up-projection 8192 x 14336 x 4096 end to end in 6.9 ms with 1024-column
 // panels, 6.2 ms with 2048).
 constexpr int64_t kMinColPanel = 2048;
-constexpr double kPanelTargetBytes = 16.0 * 1024 * 1024;  // streamed bytes per panel
+constexpr double kPanelTargetBytes = 32.0 * 1024 * 1024;  // streamed bytes per panel
 
 int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
 
