@@ -4,7 +4,7 @@ Some callers must not allocate device memory while they run: plugins whose
 enqueue step may not allocate, processes whose GPU memory belongs to a pool
 allocator, and latency-critical loops where cudaMalloc's implicit device
 synchronisation would stall other work.  For them gemm_relu_f16_noalloc runs
-the small-M small-M kernel with its scratch (fp32 partial tiles and arrival
+the small-M kernel with its scratch (fp32 partial tiles and arrival
 counters) in a fixed array inside the library, limited to M <= 32.
 
 These tests call it through the C ABI, twice in a row on the same inputs
