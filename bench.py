@@ -161,11 +161,24 @@ def time_launches(fn, steps: int, warmup: int, stream, dist=None, sampler=None,
     return total, per_ms
 
 
+def parity_rows(M: int, max_rows: int) -> list:
+    """Rows of an M-row result to compare with the oracle: all of them when
+    there are at most `max_rows`, else `max_rows` rows spread evenly over M
+    (first and last included), so that every tile row of every kernel's
+    tiling is sampled."""
+    if M <= max_rows:
+        return list(range(M))
+    step = (M - 1) / (max_rows - 1)
+    return sorted({int(round(i * step)) for i in range(max_rows)})
+
+
 def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
-                     comparator=False, variant="relu", path=0):
+                     comparator=False, variant="relu", path=0, check_rows=0):
     """Time one workload.  variant: "relu" (gemm_relu_f16, the measured path),
     "bias_gelu" (gemm_bias_act_f16 with a per-column bias and GELU) or "wT"
-    (gemm_f16_general with B stored N x K, ReLU)."""
+    (gemm_f16_general with B stored N x K, ReLU).  With `check_rows` > 0 the
+    result's rows (all, or that many spread over M) are kept for the oracle
+    check."""
     import torch
 
     from tiled_tensor_core_05_b200 import ops, workloads
@@ -210,7 +223,13 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
         raise RuntimeError(f"device reported status {st:#x}")
     # `step` holds raw pointers: keep the tensors alive as long as it is
     res = {"total_ms": total_ms, "launch_ms": launch_ms, "w": w, "step": step,
-           "tensors": (a, b, c, bias)}
+           "tensors": (a, b, c, bias), "variant": variant, "name": name}
+    if check_rows:
+        # rows of the measured call's result, kept on the host for the oracle
+        # check of the cpu_baseline leg
+        rows = parity_rows(w.M, check_rows)
+        res["check"] = {"rows": rows, "c_rows": c[torch.as_tensor(rows, device=c.device)].cpu(),
+                        "bias": None if bias is None else bias.cpu()}
     if comparator:
         # context only, never on the measured path: cuBLAS through torch on
         # the same inputs, timed the same way right after our kernel
@@ -388,18 +407,21 @@ def stream_read_probe(gib: float = 2.0, steps: int = 20):
             "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
 
 
-def parity_summary(got, ref) -> dict:
+def parity_summary(got, ref, relu: bool = True) -> dict:
     """Element-by-element comparison of fp16 results with the acceptance rule
-    of the tests: |got - ref| <= 1e-2 + 1e-2 |ref|, and got > 0 wherever
-    ref > 1e-2 (ReLU output)."""
+    of the tests: |got - ref| <= 1e-2 + 1e-2 |ref|, and wherever |ref| > 1e-2
+    the sign of got equals the sign of ref (for ReLU output: got > 0)."""
     import numpy as np
     g = np.asarray(got, dtype=np.float16).astype(np.float64)
     r = np.asarray(ref, dtype=np.float16).astype(np.float64)
-    err = np.abs(g - r)
+    with np.errstate(invalid="ignore"):
+        err = np.where(g == r, 0.0, np.abs(g - r))  # equal infinities count as equal
     bad = ~(err <= 1e-2 + 1e-2 * np.abs(r))  # NaN counts as out of tolerance
-    big = r > 1e-2
-    sign_bad = int(np.count_nonzero(big & ~(g > 0)))
-    rel = err[big] / r[big]
+    big = np.abs(r) > 1e-2
+    sign_bad = int(np.count_nonzero(big & (np.sign(g) != np.sign(r))))
+    if relu:
+        sign_bad += int(np.count_nonzero(g < 0))
+    rel = err[big] / np.abs(r[big])
     return {"elements": int(r.size), "max_abs_err": float(np.nanmax(err)) if r.size else 0.0,
             "max_rel_err": float(rel.max()) if rel.size else 0.0,
             "out_of_tolerance": int(np.count_nonzero(bad)), "sign_mismatches": sign_bad,
@@ -432,6 +454,55 @@ def cpu_baseline(name, budget_s=10.0, gpu_c=None):
         out["parity"] = dict(parity_summary(gpu_c[:rows].cpu().numpy(), ref),
                              rows=f"0-{rows - 1} of {w.M}")
     return out
+
+
+def oracle_check(res) -> dict:
+    """Part of the cpu_baseline leg: the oracle's rows of one measured
+    workload (all rows, or a spread sample; see parity_rows) against the rows
+    of the measured call's result kept by measure_workload."""
+    import numpy as np
+
+    import oracle
+    from tiled_tensor_core_05_b200 import workloads
+    chk = res["check"]
+    w = res["w"]
+    a, b = workloads.workload_inputs(w.name)
+    a_rows = a[torch_index(chk["rows"])]
+    if res["variant"] == "bias_gelu":
+        ref = oracle.gemm_bias_act(a_rows, b, chk["bias"], "gelu")
+        relu = False
+    else:  # "relu" and "wT" (B stored N x K: the same product)
+        ref = oracle.gemm_relu(a_rows, b)
+        relu = True
+    s = parity_summary(np.asarray(chk["c_rows"].numpy()), ref, relu)
+    s["rows"] = len(chk["rows"])
+    return s
+
+
+def torch_index(rows):
+    import torch
+    return torch.as_tensor(rows, dtype=torch.long)
+
+
+def compact_record(res, peaks, peak_src) -> dict:
+    """One short line of the per-workload table that ends the bench line."""
+    w = res["w"]
+    ms = res["launch_ms"]
+    roof = roofline_entry(w.name, ms, peaks, peak_src, False, res["variant"])
+    # keys: op = the variant; frac = of the measured peak; pct_nom = % of the
+    # nominal 2.25 PFLOP/s or 8 TB/s; traffic = ncu DRAM bytes per launch
+    rec = {"workload": w.name, "op": res["variant"], "ms": round(ms, 4),
+           "value": roof["achieved"], "unit": roof["unit"], "frac": roof["frac"],
+           "pct_nom": round(100 * roof["achieved"] / (
+               NOMINAL_HBM_GBS if roof["unit"] == "GB/s" else NOMINAL_FP16_TFLOPS), 1),
+           "traffic": roof["traffic"]}
+    return rec
+
+
+def parity_text(s: dict, M: int) -> str:
+    """'pass 256/8192 rows' (or 'FAIL ...' with the counts)."""
+    head = "pass" if s["pass"] else f"FAIL {s['out_of_tolerance']} out, {s['sign_mismatches']} sign"
+    return f"{head} {s['rows']}/{M} rows"
 
 
 # ------------------------------------------------------------------ arms ---
@@ -482,6 +553,38 @@ def workload_config(w):
             "l2": l2, "parallelism": "replicas (one independent problem per GPU)"}
 
 
+def sharded_decode(dist, world, rank, steps, warmup, gather=True):
+    """The column-sharded small-M product across the ranks (one process per
+    GPU): every rank holds A and its own block of whole 256-column tiles of
+    B, computes its block of C = ReLU(A @ B) and, with `gather`, all-gathers
+    the blocks so that every rank holds the whole C.  Total work is fixed
+    (strong scaling): the job rate is the whole problem's algorithmic bytes
+    over the max-over-ranks time per step.  Returns (record, C on the device,
+    or None without `gather`)."""
+    import torch
+
+    from tiled_tensor_core_05_b200 import shard, workloads
+    w = workloads.WORKLOADS["decode"]
+    a_cpu, b_cpu = workloads.workload_inputs("decode")
+    n0, n1 = shard.column_range(w.N, world, rank)
+    a = a_cpu.cuda()
+    b_blk = b_cpu[:, n0:n1].contiguous().cuda()
+    del b_cpu
+    out = torch.empty((w.M, w.N), dtype=torch.float16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        shard.gemm_sharded(a, b_blk, n_total=w.N, out=out, rank=rank, world=world,
+                           gather=gather)
+
+    total_ms, _ = time_launches(step, steps, warmup, stream, dist)
+    ms = total_ms / steps
+    rec = {"workload": "decode", "n_gpus": world, "scaling": "strong", "gather": gather,
+           "ms": round(ms, 5), "value": round(w.bytes_min / (ms * 1e-3) / 1e9, 1),
+           "unit": "GB/s", "columns_per_rank": n1 - n0}
+    return rec, (out if gather else None)
+
+
 def run_ours(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -494,14 +597,17 @@ def run_ours(args):
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local))
         dist = tdist
-    from tiled_tensor_core_05_b200 import ops, workloads
+    from tiled_tensor_core_05_b200 import ops
     ops.lib()
     peaks, peak_src = load_peaks()
+    single = rank == 0 and world == 1
+    check = single and not args.no_cpu_baseline
     sampler = ClockSampler(gpu_id_for(local))
     sampler.wait_first()
     main = measure_workload(args.workload, args.steps, args.warmup, dist, sampler,
                             e2e=not args.no_e2e, comparator=not args.no_comparator,
-                            path=args.path, variant=args.variant)
+                            path=args.path, variant=args.variant,
+                            check_rows=256 if check else 0)
     sampler.stop()
     clocks = sampler.summary()
     w = main["w"]
@@ -532,67 +638,81 @@ def run_ours(args):
                        "call": "gemm_relu_f16_host" if args.variant == "relu" else "gemm_f16_host",
                        "plan": main["e2e_plan"], "bits_equal_device": main["e2e_bits_equal"]}
     line["clocks"] = clocks
+    context = {}
     if "torch_launch_ms" in main:
-        t_ms = main["torch_launch_ms"]
-        line["context_torch_matmul_relu"] = {
-            "what": "torch.relu(torch.matmul(a, b)) (cuBLAS fp16 + a separate ReLU kernel), "
-                    "same inputs and timing; context only, not on the measured path",
-            "ms_per_call": round(t_ms, 5),
-            "tflops": round(w.flops / (t_ms * 1e-3) / 1e12, 2) if unit == "TFLOP/s" else None,
-            "gbs": round(w.bytes_min / (t_ms * 1e-3) / 1e9, 1) if unit == "GB/s" else None}
+        context["torch_matmul_act_ms"] = round(main["torch_launch_ms"], 5)
+    # the sharded small-M product (row f4) at every rank count: each rank
+    # streams its 1/N of B; every rank takes the same steps and collectives
+    if not args.no_shard:
+        srec, s_out = sharded_decode(dist, world, rank, max(args.steps, 20),
+                                     max(args.warmup, 3))
+        if s_out is not None and check:
+            srec["check"] = {"rows": list(range(s_out.shape[0])), "c_rows": s_out.cpu(),
+                             "bias": None}
+        del s_out
+        torch.cuda.empty_cache()
+    else:
+        srec = None
     # context passes (other workloads, probe, per-launch and sustained runs)
     # only in single-GPU runs: under torchrun the other ranks would wait for
     # rank 0 at the closing barrier meanwhile
-    if rank == 0 and world == 1 and not args.no_secondary:
-        others = []
+    others = []
+    if single and not args.no_secondary:
         for name, variant in (("mlp_up", "relu"), ("decode", "relu"), ("cube1024", "relu"),
-                              ("cube256", "relu"), ("mlp_up", "bias_gelu"), ("decode", "wT")):
-            if name == args.workload and variant == "relu":
+                              ("ragged1000", "relu"), ("cube256", "relu"),
+                              ("mlp_up", "bias_gelu"), ("decode", "wT")):
+            if name == args.workload and variant == args.variant:
                 continue
             r = measure_workload(name, max(args.steps, 20), max(args.warmup, 3), None, None,
-                                 e2e=False, comparator=not args.no_comparator, variant=variant)
-            ow = r["w"]
-            entry = {"workload": name, "variant": variant, "M": ow.M, "N": ow.N, "K": ow.K,
-                     "ms_per_launch": round(r["launch_ms"], 5),
-                     "tflops": round(ow.flops / (r["launch_ms"] * 1e-3) / 1e12, 2),
-                     "roofline": roofline_entry(name, r["launch_ms"], peaks, peak_src, False,
-                                                variant)}
-            if "torch_launch_ms" in r:
-                entry["context_torch_ms_per_call"] = round(r["torch_launch_ms"], 5)
-            if hbm_bound(ow):
-                entry["gbs"] = round(ow.bytes_min / (r["launch_ms"] * 1e-3) / 1e9, 1)
-                entry["pct_of_nominal_hbm"] = round(100 * entry["gbs"] / NOMINAL_HBM_GBS, 2)
-            else:
-                entry["pct_of_dense_fp16_peak"] = round(100 * entry["tflops"] /
-                                                        NOMINAL_FP16_TFLOPS, 2)
-            others.append(entry)
-        line["other_workloads"] = others
+                                 e2e=False, comparator=not args.no_comparator, variant=variant,
+                                 check_rows=512 if check else 0)
+            r.pop("step")
+            r.pop("tensors")
+            others.append(r)
+            torch.cuda.empty_cache()
         probe = stream_read_probe()
-        line["context_stream_read_probe"] = probe
-        for entry in [line] + others:
-            gbs = entry.get("gbs") if entry is not line else (
-                value / world if unit == "GB/s" else None)
-            if gbs:
-                entry["frac_of_read_probe"] = round(gbs / probe["gbs"], 4)
-    if rank == 0 and world == 1 and args.sustained_seconds > 0:
-        line["launch_stats"] = launch_stats(main["step"])
+        context["read_probe_gbs"] = probe["gbs"]
+    if single and args.sustained_seconds > 0:
+        ls = launch_stats(main["step"])
+        context["launch_median_ms"] = ls["median_ms"]
+        context["launch_best_ms"] = ls["best_ms"]
         sus = sustained_run(main["step"], main["launch_ms"], args.sustained_seconds,
                             gpu_id_for(local))
         rate = (w.bytes_min / (sus["ms_per_launch"] * 1e-3) / 1e9 if unit == "GB/s"
                 else w.flops / (sus["ms_per_launch"] * 1e-3) / 1e12)
-        sus["value"] = round(rate, 2)
-        sus["unit"] = unit
-        sus["note"] = "one GPU, back to back after the timed region (context, not the value)"
-        line["sustained"] = sus
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # the measured call's result (ReLU variants) against the oracle's rows
-        gpu_c = main["tensors"][2] if args.variant in ("relu", "wT") else None
-        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget, gpu_c)
+        sc = sus["clocks"]
+        context["sustained"] = {"seconds": sus["seconds"], "ms": sus["ms_per_launch"],
+                                "value": round(rate, 2), "unit": unit,
+                                "sm_mhz": sc.get("sm_mhz"), "reasons": sc.get("reasons")}
+    # the first record is the main workload's
+    records = [compact_record(r, peaks, peak_src) for r in [main] + others]
+    if "read_probe_gbs" in context:
+        for rec in records:
+            if rec["unit"] == "GB/s":
+                rec["frac_probe"] = round(rec["value"] / context["read_probe_gbs"], 4)
+    if check:
+        # the cpu_baseline leg: the oracle timed on a sample of the main
+        # workload, and every measured result compared with the oracle
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget,
+                                            main["tensors"][2]
+                                            if args.variant in ("relu", "wT") else None)
+        for rec, r in zip(records, [main] + others):
+            rec["parity"] = parity_text(oracle_check(r), r["w"].M)
+        if srec is not None and "check" in srec:
+            from tiled_tensor_core_05_b200 import workloads
+            srec["parity"] = parity_text(oracle_check(dict(srec, variant="relu",
+                                                           w=workloads.WORKLOADS["decode"])),
+                                         32)
+    if srec is not None:
+        srec.pop("check", None)
+        context["sharded_decode"] = srec
+    line["context"] = context
+    line["configs"] = records  # last: the short per-workload table
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps(line, separators=(",", ":")), flush=True)
     return 0
 
 
@@ -606,6 +726,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="cube8192")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-shard", action="store_true",
+                    help="skip the column-sharded decode leg (each rank 1/N of B)")
     ap.add_argument("--sustained-seconds", type=float, default=2.0,
                     help="length of the back-to-back context run after the timed region "
                          "(0: skip it and the per-launch statistics)")

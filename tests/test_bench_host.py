@@ -144,3 +144,78 @@ def test_parity_summary():
     got = ref.copy()
     got[0, 0] = np.nan
     assert not bench.parity_summary(got, ref)["pass"]
+
+
+def test_parity_summary_gelu_signs():
+    """GELU output may be negative: only the sign pattern where |ref| > 1e-2
+    and the tolerance count, not got >= 0."""
+    import numpy as np
+    ref = np.array([-0.17, -0.005, 0.0, 0.8], dtype=np.float16)
+    s = bench.parity_summary(ref.copy(), ref, relu=False)
+    assert s["pass"]
+    assert not bench.parity_summary(ref.copy(), ref, relu=True)["pass"]  # negatives
+    got = ref.copy()
+    got[0] = 0.0                  # -0.17 lost its sign (and is 0.17 off)
+    s = bench.parity_summary(got, ref, relu=False)
+    assert not s["pass"] and s["sign_mismatches"] == 1
+
+
+@pytest.mark.parametrize("M,n", [(32, 512), (1000, 512), (8192, 256), (8192, 512), (2, 2)])
+def test_parity_rows_cover_every_tile_row(M, n):
+    rows = bench.parity_rows(M, n)
+    assert rows == sorted(set(rows)) and rows[0] == 0 and rows[-1] == M - 1
+    assert len(rows) == min(M, n)
+    # every 128-row tile (the smallest tile height of the kernels) is sampled
+    # when there are at least as many samples as tiles
+    if n >= -(-M // 128):
+        assert {r // 128 for r in rows} == set(range(-(-M // 128)))
+
+
+def _fake_res(name, variant, ms):
+    return {"w": workloads.WORKLOADS[name], "variant": variant, "launch_ms": ms}
+
+
+def test_per_workload_records_fit_the_drivers_tail():
+    """The short per-workload table ends the bench line and must fit, whole,
+    in the last 1500 characters that the driver keeps of it."""
+    peaks = {"hbm_gbs": 6532.5, "bf16_tflops": 1672.3, "bf16_tflops_sustained": 1370.4}
+    res = [_fake_res("cube8192", "relu", 0.73226), _fake_res("mlp_up", "relu", 0.65612),
+           _fake_res("decode", "relu", 0.07163), _fake_res("cube1024", "relu", 0.00915),
+           _fake_res("ragged1000", "relu", 0.00913), _fake_res("cube256", "relu", 0.00716),
+           _fake_res("mlp_up", "bias_gelu", 0.71361), _fake_res("decode", "wT", 0.07597)]
+    recs = [bench.compact_record(r, peaks, "measured") for r in res]
+    for rec, r in zip(recs, res):
+        rec["traffic"] = 1004495616
+        rec["frac_probe"] = 0.9347
+        rec["parity"] = bench.parity_text({"pass": True, "out_of_tolerance": 0,
+                                           "sign_mismatches": 0, "rows": 512}, r["w"].M)
+    text = json.dumps({"configs": recs}, separators=(",", ":"))
+    assert len(text) < 1450, len(text)
+    assert recs[2]["unit"] == "GB/s" and recs[0]["unit"] == "TFLOP/s"
+    assert recs[0]["value"] == pytest.approx(1501.5, abs=0.1)
+    assert recs[1]["parity"] == "pass 512/8192 rows"
+    bad = bench.parity_text({"pass": False, "out_of_tolerance": 3, "sign_mismatches": 1,
+                             "rows": 32}, 32)
+    assert bad.startswith("FAIL 3 out, 1 sign")
+
+
+def test_oracle_check_catches_a_planted_error():
+    """The cpu_baseline leg's comparison against the oracle, on the host: the
+    oracle's own rows pass, a row with one flipped element fails."""
+    import numpy as np
+    import torch
+
+    import oracle
+    w = workloads.WORKLOADS["cube256"]
+    a, b = workloads.workload_inputs("cube256")
+    rows = bench.parity_rows(w.M, 64)
+    good = torch.from_numpy(np.ascontiguousarray(oracle.gemm_relu(a[rows], b)))
+    res = {"w": w, "variant": "relu", "check": {"rows": rows, "c_rows": good, "bias": None}}
+    s = bench.oracle_check(res)
+    assert s["pass"] and s["rows"] == 64 and s["elements"] == 64 * 256
+    bad = good.clone()
+    i = int(torch.argmax(bad[3].float()))
+    bad[3, i] = 0.0  # a positive value zeroed
+    res["check"]["c_rows"] = bad
+    s = bench.oracle_check(res)
+    assert not s["pass"] and s["out_of_tolerance"] >= 1

@@ -106,11 +106,19 @@ def test_mlp_up_gelu_sampled(oracle_mod):
     bias_h = (rng.standard_normal(w.N) * 0.5).astype(np.float16)
     c = ops.gemm_bias_act_f16(a_cpu.cuda(), b_cpu.cuda(), torch.from_numpy(bias_h).cuda(), "gelu")
     torch.cuda.synchronize()
+    c_np = dev_to_np(c)
+    # 512 whole rows spread over M, from the oracle's fused bias + GELU
+    rows_full = np.unique(np.round(np.linspace(0, w.M - 1, 512)).astype(np.int64))
+    ref_rows = oracle_mod.gemm_bias_act(a_cpu[torch.from_numpy(rows_full)], b_cpu, bias_h,
+                                        "gelu")
+    check_parity(c_np[rows_full], ref_rows, False, "mlp_up gelu 512 whole rows")
+    # random elements, built from the oracle's fp64 sums, its own GELU and
+    # its own fp16 encoder
     rows = rng.integers(0, w.M, 2048)
     cols = rng.integers(0, w.N, 2048)
     s = oracle_mod.gemm_f64_at(a_cpu, b_cpu, rows, cols) + bias_h.astype(np.float64)[cols]
-    ref = pe.to_f16_bits(pe.gelu64(s)).view(np.float16)
-    check_parity(dev_to_np(c)[rows, cols], ref, False, "mlp_up gelu sampled")
+    ref = oracle_mod.encode_f16(oracle_mod.activation_f64(s, "gelu")).view(np.float16)
+    check_parity(c_np[rows, cols], ref, False, "mlp_up gelu sampled")
 
 
 def test_bias_must_be_aligned():

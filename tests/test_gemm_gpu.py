@@ -184,13 +184,23 @@ def test_workload_fullsize_sampled(oracle_mod, name):
     assert not torch.isnan(c).any()
     assert (c >= 0).all()
     assert not (c.view(torch.int16) == -32768).any()
-    # sampled parity: two whole rows, two whole columns (first and last: ragged
-    # tile edges of the grid), 4096 random elements
+    c_np = dev_to_np(c)
+    # whole rows against the oracle: all of them for the small-M workload (C
+    # is 32 x 28672), 512 spread over M (first and last included, every
+    # 128-row tile sampled) for the large ones
+    if w.M <= 64:
+        rows_full = np.arange(w.M)
+    else:
+        rows_full = np.unique(np.round(np.linspace(0, w.M - 1, 512)).astype(np.int64))
+        assert len(rows_full) == 512
+    ref_rows = oracle_mod.gemm_relu(a_cpu[torch.from_numpy(rows_full)], b_cpu)
+    check_parity(c_np[rows_full], ref_rows, True, f"{name} {len(rows_full)} whole rows")
+    # and whole columns (first and last: ragged tile edges of the grid) plus
+    # 4096 random elements
     rng = np.random.default_rng(w.seed)
-    rows, cols = sample_points(w.M, w.N, rng, rows=(0, w.M - 1), cols=(0, w.N - 1))
+    rows, cols = sample_points(w.M, w.N, rng, rows=(), cols=(0, w.N - 1))
     ref = oracle_mod.gemm_relu_at(a_cpu, b_cpu, rows, cols)
-    got = dev_to_np(c)[rows, cols]
-    check_parity(got, ref, True, f"{name} sampled")
+    check_parity(c_np[rows, cols], ref, True, f"{name} sampled")
     frac = float((c > 0).float().mean())
     assert 0.45 < frac < 0.55, frac
 

@@ -9,10 +9,12 @@ counters) in a fixed array inside the library, limited to M <= 32.
 
 These tests call it through the C ABI, twice in a row on the same inputs
 (the second call finds the first call's leftovers in the shared array), and
-compare each result with the allocating entry point gemm_relu_f16 within the
-tolerance the other GPU tests use.  They set up everything they need, so they
-pass on their own in a fresh process as well as after the rest of the suite;
-the file name makes pytest collect them last.
+compare each result with the allocating entry point gemm_relu_f16 and with
+the CPU oracle (the plain fp64 definition, which shares no code with either
+entry point), within the tolerance the other GPU tests use and with the same
+sign and zero pattern.  They set up everything they need, so they pass on
+their own in a fresh process as well as after the rest of the suite; the file
+name makes pytest collect them last.
 """
 import numpy as np
 import pytest
@@ -44,10 +46,20 @@ def _call(fn, a, b, c):
               torch.cuda.current_stream().cuda_stream)
 
 
-def _close(c: torch.Tensor, ref: torch.Tensor) -> bool:
+def _close(c: torch.Tensor, ref) -> bool:
+    """Within the tolerance of a device result (tensor) or an oracle result."""
     c64 = c.double().cpu().numpy()
-    r64 = ref.double().cpu().numpy()
+    r64 = ref.double().cpu().numpy() if isinstance(ref, torch.Tensor) else np.float64(ref)
     return bool(np.all(np.abs(c64 - r64) <= ATOL + RTOL * np.abs(r64)))
+
+
+def _same_relu_pattern(c: torch.Tensor, ref: np.ndarray) -> bool:
+    """c > 0 wherever ref > 1e-2, no negative value, no -0, no NaN."""
+    bits = c.cpu().contiguous().view(torch.int16).numpy()
+    c64 = c.double().cpu().numpy()
+    r64 = np.asarray(ref, dtype=np.float64)
+    return bool((c64[r64 > ATOL] > 0).all() and (c64 >= 0).all() and not (bits == -32768).any()
+                and not np.isnan(c64).any())
 
 
 @pytest.fixture(scope="module")
@@ -73,9 +85,12 @@ def test_noalloc_matches_allocating_entry_point_on_two_calls(lib, m, n, k, seed)
         assert _call(lib.gemm_relu_f16_noalloc, a, b, c) == 0
     torch.cuda.synchronize()
     free_after = torch.cuda.mem_get_info()[0]
+    import oracle
+    want = oracle.gemm_relu(a_cpu, b_cpu).astype(np.float64)
     for i, c in enumerate(outs):
         assert _close(c, ref), f"call {i + 1} differs from gemm_relu_f16"
-        assert (c >= 0).all() and not torch.isnan(c).any()
+        assert _close(c, want), f"call {i + 1} differs from the oracle"
+        assert _same_relu_pattern(c, want), f"call {i + 1}: sign or zero pattern differs"
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
     # nothing was allocated on the device by the two calls
     assert free_before - free_after < (1 << 20), (free_before, free_after)
