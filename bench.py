@@ -578,11 +578,18 @@ def sharded_decode(dist, world, rank, steps, warmup, gather=True):
                            gather=gather)
 
     total_ms, _ = time_launches(step, steps, warmup, stream, dist)
-    ms = total_ms / steps
-    rec = {"workload": "decode", "n_gpus": world, "scaling": "strong", "gather": gather,
-           "ms": round(ms, 5), "value": round(w.bytes_min / (ms * 1e-3) / 1e9, 1),
-           "unit": "GB/s", "columns_per_rank": n1 - n0}
-    return rec, (out if gather else None)
+    return shard_record(w, world, rank, total_ms / steps, gather), (out if gather else None)
+
+
+def shard_record(w, world: int, rank: int, ms: float, gather: bool) -> dict:
+    """The sharded leg's record: the whole problem's algorithmic bytes (A, B
+    and C once) over the max-over-ranks time per step `ms` (strong scaling:
+    the problem does not grow with the rank count)."""
+    from tiled_tensor_core_05_b200 import shard
+    n0, n1 = shard.column_range(w.N, world, rank)
+    return {"workload": w.name, "n_gpus": world, "scaling": "strong", "gather": gather,
+            "ms": round(ms, 5), "value": round(w.bytes_min / (ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s", "columns_per_rank": n1 - n0}
 
 
 def run_ours(args):
@@ -645,7 +652,7 @@ def run_ours(args):
     # streams its 1/N of B; every rank takes the same steps and collectives
     if not args.no_shard:
         srec, s_out = sharded_decode(dist, world, rank, max(args.steps, 20),
-                                     max(args.warmup, 3))
+                                     max(args.warmup, 3), gather=world > 1)
         if s_out is not None and check:
             srec["check"] = {"rows": list(range(s_out.shape[0])), "c_rows": s_out.cpu(),
                              "bias": None}

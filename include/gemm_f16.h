@@ -156,8 +156,11 @@ typedef struct gemm_config {
                          or 256 for GEMM_PATH_SKINNY; 256 (the only width) for the pair
                          kernels */
   int32_t stages;     /* depth of the shared-memory operand ring (k-blocks of 64 in flight) */
-  int32_t group_rows; /* tile kernels: rows of op(A) per raster panel, the L2 grouping of
-                         the tile order; 0 = 2048.  Must be 0 for GEMM_PATH_SKINNY */
+  int32_t group_rows; /* tile kernels: the L2 grouping of the tile order.  > 0: rows of
+                         op(A) per row panel (tiles walked column by column inside
+                         it); < 0: minus the columns of op(B) per column panel (tiles
+                         walked row by row inside it); 0 = the default.  Must be 0 for
+                         GEMM_PATH_SKINNY */
   int32_t splits;     /* GEMM_PATH_SKINNY: k-slices per column tile, 1 <= splits <=
                          ceil(K / 64) and splits * ceil(N / block_n) <= the SM count when
                          > 1; 0 = chosen from the shape.  Must be 0 for the tile kernels */

@@ -78,3 +78,15 @@ def test_reference_arm_rank0_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_shard_record_is_strong_scaling():
+    from tiled_tensor_core_05_b200 import workloads
+    w = workloads.WORKLOADS["decode"]
+    one = bench.shard_record(w, 1, 0, 0.0716, False)
+    two = bench.shard_record(w, 2, 1, 0.0358, True)
+    assert one["columns_per_rank"] == 28672 and two["columns_per_rank"] == 14336
+    assert one["scaling"] == two["scaling"] == "strong"
+    # the same whole problem in half the time: twice the job rate
+    assert two["value"] == pytest.approx(2 * one["value"], rel=1e-3)
+    assert one["value"] == pytest.approx(w.bytes_min / 0.0716e-3 / 1e9, rel=1e-3)

@@ -70,7 +70,8 @@ def test_tile_configs_transposed(oracle_mod, cfg):
     check_parity(c, ref, True, f"{cfg!r} transposed")
 
 
-@pytest.mark.parametrize("group_rows", [1, 128, 256, 512, 1024, 100000])
+@pytest.mark.parametrize("group_rows", [1, 128, 256, 512, 1024, 100000,
+                                        -1, -256, -512, -768, -100000])
 @pytest.mark.parametrize("kernel", [ops.PATH_TILE, ops.PATH_TILE_PAIR, ops.PATH_TILE_PAIR_TALL])
 def test_raster_panels(oracle_mod, kernel, group_rows):
     m, n, k = 1300, 1100, 200

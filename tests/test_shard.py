@@ -46,6 +46,14 @@ def _free_port():
 
 
 def _worker(rank, world, port, q):
+    try:
+        _work(rank, world, port, q)
+    except Exception as e:  # report instead of leaving the parent to time out
+        q.put((rank, f"error: {e!r}", False, False))
+        raise
+
+
+def _work(rank, world, port, q):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -86,6 +94,8 @@ def test_gather_across_gloo_ranks(world):
     for p in procs:
         p.start()
     results = [q.get(timeout=120) for _ in range(world)]
+    errors = [r for r in results if isinstance(r[1], str)]
+    assert not errors, errors
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0

@@ -401,7 +401,8 @@ int default_stages(int kernel, int block_n) {
 // M x N output and checks the rest (the stage count is checked against the
 // compiled kernels at launch).  Returns GEMM_OK or GEMM_ERR_CONFIG.
 int resolve_config(KernelConfig& c, int64_t M, int64_t N, int sm_count) {
-  if (c.stages < 0 || c.group_rows < 0 || c.splits < 0) return GEMM_ERR_CONFIG;
+  if (c.stages < 0 || c.splits < 0) return GEMM_ERR_CONFIG;
+  if (c.group_rows < 0 && c.kernel == GEMM_PATH_SKINNY) return GEMM_ERR_CONFIG;
   switch (c.kernel) {
     case GEMM_PATH_TILE:
       if (c.block_n == 0) {

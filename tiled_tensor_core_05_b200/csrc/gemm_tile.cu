@@ -22,6 +22,7 @@
 // Out-of-range A/B elements (M, N or K not a multiple of the tile) are
 // zero-filled by TMA and so contribute nothing to the sum.
 #include <atomic>
+#include <cstdlib>
 
 #include "../../include/gemm_f16.h"
 #include "internal.h"
@@ -155,16 +156,40 @@ static_assert(variants_complete(), "built tile configurations != those within th
 
 // Grouped-panel rasterisation: consecutive tile indices sweep group_m
 // tile-rows of one panel column by column, so the CTAs that run at the same
-// time share A rows and B columns in L2.
+// time share A rows and B columns in L2.  A negative group_m gives panels of
+// -group_m tile-columns swept row by row instead (the same with the roles of
+// A and B exchanged).
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m,
                                             int& mb, int& nb) {
-  const int per_group = group_m * num_n;
-  const int g = tile / per_group;
-  const int first_m = g * group_m;
-  const int rows = min(num_m - first_m, group_m);
-  const int r = tile - g * per_group;
-  mb = first_m + r % rows;
-  nb = r / rows;
+  if (group_m > 0) {
+    const int per_group = group_m * num_n;
+    const int g = tile / per_group;
+    const int first_m = g * group_m;
+    const int rows = min(num_m - first_m, group_m);
+    const int r = tile - g * per_group;
+    mb = first_m + r % rows;
+    nb = r / rows;
+  } else {
+    const int group_n = -group_m;
+    const int per_group = group_n * num_m;
+    const int g = tile / per_group;
+    const int first_n = g * group_n;
+    const int cols = min(num_n - first_n, group_n);
+    const int r = tile - g * per_group;
+    nb = first_n + r % cols;
+    mb = r / cols;
+  }
+}
+
+// L2 eviction priority of the operand loads, one 2-bit field per operand
+// (bits 0-1 A, bits 2-3 B): 0 = no hint, 1 = evict-first, 2 = evict-normal,
+// 3 = evict-last.  The operand a raster panel re-reads across waves (A with
+// row panels, B with column panels) is the one worth keeping.
+enum : int { kHintNone = 0, kHintFirst = 1, kHintNormal = 2, kHintLast = 3 };
+__device__ __forceinline__ uint64_t l2_policy_for(int code) {
+  return code == kHintFirst ? l2_policy_evict_first()
+         : code == kHintLast ? l2_policy_evict_last()
+                             : l2_policy_evict_normal();
 }
 
 // Epilogue of one accumulator tile, run by one warp for its 32 TMEM lanes and
@@ -501,7 +526,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
                           int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
-                          int layout, int group_m, int split_from, int* status,
+                          int layout, int group_m, int split_from, int l2_hint, int* status,
                           uint64_t timeout_ns) {
   using Cfg = PairCfg<STAGES, SLABS>;
   const bool ta = (layout & kLayoutTransA) != 0;
@@ -584,6 +609,20 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
+      const int hint_a = l2_hint & 3, hint_b = (l2_hint >> 2) & 3;
+      const uint64_t pol_a = l2_policy_for(hint_a), pol_b = l2_policy_for(hint_b);
+      auto load_a = [&](uint32_t bar, void* dst, int c0, int c1) {
+        if (hint_a != kHintNone)
+          tma_load_2d_pair_hint(&tmA, bar, dst, c0, c1, pol_a);
+        else
+          tma_load_2d_pair(&tmA, bar, dst, c0, c1);
+      };
+      auto load_b = [&](uint32_t bar, void* dst, int c0, int c1) {
+        if (hint_b != kHintNone)
+          tma_load_2d_pair_hint(&tmB, bar, dst, c0, c1, pol_b);
+        else
+          tma_load_2d_pair(&tmB, bar, dst, c0, c1);
+      };
       for (int unit = pair; unit < num_units && ok; unit += npairs) {
         int mb, nb, row_base, slabs;
         unit_coords(unit, mb, nb, row_base, slabs);
@@ -603,18 +642,18 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
             uint8_t* adst = smA + stage * Cfg::kABytes + s * Cfg::kSlabBytes;
             const int row = a_row + s * 2 * kBM;
             if (!ta) {
-              tma_load_2d_pair(&tmA, bar, adst, kb * kBK, row);
+              load_a(bar, adst, kb * kBK, row);
             } else {
-              tma_load_2d_pair(&tmA, bar, adst, row, kb * kBK);
-              tma_load_2d_pair(&tmA, bar, adst + Cfg::kBChunk, row + 64, kb * kBK);
+              load_a(bar, adst, row, kb * kBK);
+              load_a(bar, adst + Cfg::kBChunk, row + 64, kb * kBK);
             }
           }
           uint8_t* bdst = smB + stage * Cfg::kBBytes;
           if (!tb) {
-            tma_load_2d_pair(&tmB, bar, bdst, b_col, kb * kBK);
-            tma_load_2d_pair(&tmB, bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
+            load_b(bar, bdst, b_col, kb * kBK);
+            load_b(bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
           } else {
-            tma_load_2d_pair(&tmB, bar, bdst, kb * kBK, b_col);
+            load_b(bar, bdst, kb * kBK, b_col);
           }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -846,10 +885,28 @@ int encode_operand_maps(const GemmProblem& p, int a_rows, int b_cols, CUtensorMa
   return encode_tmap_f16_2d(tB, p.B, p.N, p.K, p.ldb, 64, kBK);  // 64 n by 64 k
 }
 
-// Tile-rows per raster panel for `group_rows` rows of A.
-int group_tiles(int group_rows, int tile_rows) {
-  const int g = group_rows / tile_rows;
+// Raster panel of the tile kernels in tiles: `group` > 0 rows of A per row
+// panel -> that many tile-rows (at least 1); `group` < 0 columns of B per
+// column panel -> minus that many tile-columns.
+int group_tiles(int group, int tile_rows, int tile_cols) {
+  if (group < 0) {
+    const int g = -group / tile_cols;
+    return g > 0 ? -g : -1;
+  }
+  const int g = group / tile_rows;
   return g > 0 ? g : 1;
+}
+
+// The L2 hint code of the pair kernels' operand loads (see l2_policy_for):
+// TTC_L2HINT in the environment (a number 0-15), read once, else none.
+int l2_hint_code() {
+  static const int code = [] {
+    const char* s = std::getenv("TTC_L2HINT");
+    if (s == nullptr) return 0;
+    const int v = std::atoi(s);
+    return (v >= 0 && v <= 15) ? v : 0;
+  }();
+  return code;
 }
 
 template <int BN, int STAGES, int ACT>
@@ -880,7 +937,8 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
-      static_cast<int>(p.K), p.layout, group_tiles(group_rows, kBM), d.status, d.timeout_ns);
+      static_cast<int>(p.K), p.layout, group_tiles(group_rows, kBM, BN), d.status,
+      d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
@@ -938,8 +996,8 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
-      static_cast<int>(p.K), p.layout, group_tiles(group_rows, Cfg::kTileM),
-      static_cast<int>(split_from), d.status, d.timeout_ns);
+      static_cast<int>(p.K), p.layout, group_tiles(group_rows, Cfg::kTileM, Cfg::kBN),
+      static_cast<int>(split_from), l2_hint_code(), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 

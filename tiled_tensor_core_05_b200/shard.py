@@ -74,17 +74,31 @@ def gemm_sharded(a: torch.Tensor, b: torch.Tensor, *, n_total: int | None = None
         local(a, b_block, bias_block, act, out_block)
     if not gather:
         return out_block
+    if world == 1:  # the block is the whole result
+        return out if out is not None else out_block
     import torch.distributed as dist
-    # the collective wants equal-size blocks: rank 0's is the widest
+    # One collective into one contiguous buffer of `world` equal-size blocks:
+    # rank 0's block is the widest, narrower ones are padded to it.  The
+    # blocks cannot land in C directly: a column block of row-major C is a
+    # strided region, and the collective moves contiguous buffers; the copy
+    # out of the buffer is M x N x 2 bytes on the device (1.8 MB for a 32-row
+    # decode product).
     r00, r01 = column_range(N, world, 0)
-    send = torch.zeros((M, r01 - r00), dtype=out_block.dtype, device=out_block.device)
-    send[:, :n1 - n0] = out_block
-    chunks = [torch.empty_like(send) for _ in range(world)]
-    dist.all_gather(chunks, send, group=group)
+    width = r01 - r00
+    if n1 - n0 == width:
+        send = out_block.contiguous()
+    else:
+        send = torch.zeros((M, width), dtype=out_block.dtype, device=out_block.device)
+        send[:, :n1 - n0] = out_block
+    gathered = torch.empty((world, M, width), dtype=send.dtype, device=send.device)
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(gathered, send, group=group)
+    else:  # gloo has no single-buffer form: the same buffer as a list of views
+        dist.all_gather(list(gathered.unbind(0)), send, group=group)
     full = out if out is not None else torch.empty((M, N), dtype=a.dtype, device=a.device)
     for r in range(world):
         r0, r1 = column_range(N, world, r)
         if r1 <= r0 or (out is not None and r == rank):  # empty, or written in place
             continue
-        full[:, r0:r1] = chunks[r][:, :r1 - r0]
+        full[:, r0:r1] = gathered[r, :, :r1 - r0]
     return full
