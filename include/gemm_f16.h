@@ -34,9 +34,12 @@
  *     run, whatever the scheduling.
  *   - Small-M problems (M <= 64) use a split-K path whose fp32 partial tiles
  *     and arrival counters live in a workspace the library allocates once per
- *     (device, stream) on first use (cudaMalloc; about 10 MB on a 148-SM GPU)
- *     and keeps until process exit.  Make that first call outside CUDA-graph
- *     capture.  Two calls on different streams never share a workspace.
+ *     (device, stream) on first use (cudaMalloc of SMs x 256 x 64 x 4 bytes
+ *     plus the counters: 9.7 MB on a 148-SM GPU) and keeps until
+ *     gemm_release() or process exit, so a caller that cycles through many
+ *     streams holds 9.7 MB per stream it used.  Make that first call outside
+ *     CUDA-graph capture.  Two calls on different streams never share a
+ *     workspace.
  *   - The device-pointer entry points can be captured in CUDA graphs once a
  *     first call on the same device and stream has run outside the capture
  *     (it creates the workspace and caches kernel attributes); replays read
@@ -352,6 +355,17 @@ GEMM_API int gemm_f16_host_planned(const void* A, const void* B, const void* bia
  * exist any more).  Not to be called while another thread is inside
  * gemm_f16_host.  Returns GEMM_OK or GEMM_ERR_LAUNCH. */
 GEMM_API int gemm_host_release(void);
+
+/* Frees every device buffer the library holds: the small-M workspaces of all
+ * (device, stream) pairs and the host-buffer staging (gemm_host_release).  It
+ * first waits for all work on each device that holds a workspace
+ * (cudaDeviceSynchronize), since a workspace may still be in use by a kernel
+ * in flight on a stream the caller no longer has.  The next small-M call
+ * allocates a fresh workspace.  Not to be called while another thread is
+ * inside an entry point of the library, nor during CUDA-graph capture, nor
+ * while a captured graph that uses a workspace may still be launched.
+ * Returns GEMM_OK or GEMM_ERR_LAUNCH. */
+GEMM_API int gemm_release(void);
 
 /* y[i] = act(x[i]) for n fp32 values in device memory, with the exact code
  * the GEMM epilogues use (GELU: x * Phi(x), Phi from Abramowitz & Stegun

@@ -21,7 +21,8 @@ int main(void) {
       (any_fn)gemm_f16_host,         (any_fn)gemm_relu_f16_host,
       (any_fn)gemm_host_plan_for,    (any_fn)gemm_f16_host_planned,
       (any_fn)gemm_host_release,     (any_fn)gemm_activation_f32,
-      (any_fn)gemm_read_probe,       (any_fn)gemm_abi_version};
+      (any_fn)gemm_read_probe,       (any_fn)gemm_abi_version,
+      (any_fn)gemm_release};
   const int n_entry = (int)(sizeof(entry_points) / sizeof(entry_points[0]));
   int i, missing = 0;
   for (i = 0; i < n_entry; ++i) missing += entry_points[i] == NULL;

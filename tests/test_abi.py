@@ -73,7 +73,7 @@ def test_path_selection(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gemm_abi_version() >= 10200
+    assert lib.gemm_abi_version() >= 10300
 
 
 def test_argument_errors_are_reported_before_any_device_work(lib):

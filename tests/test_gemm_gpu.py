@@ -338,3 +338,26 @@ def test_bounded_wait_times_out_and_context_survives(oracle_mod):
     a, b = workloads.workload_inputs("cube256")
     check_parity(run(a, b), oracle_mod.gemm_relu(a, b), True, "after timeout")
     assert ops.device_status() == 0
+
+
+def test_release_frees_the_workspaces_and_later_calls_work(oracle_mod):
+    """gemm_release frees the small-M workspace of every (device, stream) that
+    has one; the next small-M call allocates a fresh one and is still right."""
+    a_cpu, b_cpu = workloads.make_inputs(32, 1000, 1000, seed=3)
+    a, b = a_cpu.cuda(), b_cpu.cuda()
+    ref = oracle_mod.gemm_relu(a_cpu, b_cpu)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):  # a workspace for this stream
+        c = ops.gemm_relu_f16(a, b)
+    torch.cuda.synchronize()
+    check_parity(dev_to_np(c), ref, True, "before release")
+    free0 = torch.cuda.mem_get_info()[0]
+    ops.release()
+    free1 = torch.cuda.mem_get_info()[0]
+    assert free1 - free0 >= 9 << 20, (free0, free1)  # at least that stream's 9.7 MB
+    for s in (side, torch.cuda.current_stream()):
+        with torch.cuda.stream(s):
+            c = ops.gemm_relu_f16(a, b)
+        torch.cuda.synchronize()
+        check_parity(dev_to_np(c), ref, True, "after release")
+    assert ops.device_status() == 0

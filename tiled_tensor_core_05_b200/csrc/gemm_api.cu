@@ -349,7 +349,7 @@ using namespace ttc;
 
 extern "C" {
 
-int gemm_abi_version(void) { return 10200; }
+int gemm_abi_version(void) { return 10300; }
 
 namespace ttc {
 namespace {
@@ -649,6 +649,33 @@ int gemm_activation_f32(const void* x, void* y, int64_t n, int activation,
   else
     activation_f32_kernel<kActNone><<<g, 256, 0, stream>>>(xf, yf, n);
   return cudaGetLastError() == cudaSuccess ? GEMM_OK : GEMM_ERR_LAUNCH;
+}
+
+int gemm_release(void) {
+  int rc = GEMM_OK;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int prev = 0;
+    if (cudaGetDevice(&prev) != cudaSuccess) return GEMM_ERR_LAUNCH;
+    uint64_t synced = 0;
+    for (const Workspace& w : g_workspaces) {
+      if (cudaSetDevice(w.device) != cudaSuccess) {
+        rc = GEMM_ERR_LAUNCH;
+        continue;
+      }
+      // the stream the workspace served may be gone: wait for the whole device
+      const uint64_t bit = 1ull << (w.device & 63);
+      if (!(synced & bit)) {
+        if (cudaDeviceSynchronize() != cudaSuccess) rc = GEMM_ERR_LAUNCH;
+        synced |= bit;
+      }
+      if (cudaFree(w.ptr) != cudaSuccess) rc = GEMM_ERR_LAUNCH;
+    }
+    g_workspaces.clear();
+    cudaSetDevice(prev);
+  }
+  const int h = gemm_host_release();
+  return rc != GEMM_OK ? rc : h;
 }
 
 int gemm_get_device_status(gemm_stream_t stream, int* device_status) {

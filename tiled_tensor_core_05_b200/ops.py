@@ -93,6 +93,7 @@ _SIGNATURES = {
                               [ctypes.c_int, ctypes.POINTER(HostPlan), ctypes.c_void_p],
                               ctypes.c_int),
     "gemm_host_release": ([], ctypes.c_int),
+    "gemm_release": ([], ctypes.c_int),
 }
 
 
@@ -413,3 +414,9 @@ def host_plan(M: int, N: int, K: int) -> dict:
 def host_release() -> None:
     """Free the device copies and copy streams ``gemm_host`` keeps."""
     _check(lib().gemm_host_release(), "gemm_host_release")
+
+
+def release() -> None:
+    """Free every device buffer the library keeps (small-M workspaces and the
+    host-buffer staging), after waiting for the devices that hold them."""
+    _check(lib().gemm_release(), "gemm_release")
