@@ -192,51 +192,136 @@ __device__ __forceinline__ uint64_t l2_policy_for(int code) {
                              : l2_policy_evict_normal();
 }
 
+// The 64 bias values of the chunk at column col0 as 32 packed pairs (0 past
+// N): eight 16-byte loads (the same address in every lane) when the chunk
+// lies inside N, else pair by pair.
+__device__ __forceinline__ void load_bias_chunk(const __half* __restrict__ bias, int col0, int N,
+                                                uint32_t (&bb)[32]) {
+  if (col0 + kEpiCols <= N) {
+    const uint4* src = reinterpret_cast<const uint4*>(bias + col0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 q = __ldg(src + i);
+      bb[4 * i] = q.x;
+      bb[4 * i + 1] = q.y;
+      bb[4 * i + 2] = q.z;
+      bb[4 * i + 3] = q.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int col = col0 + 2 * i;
+      if (col + 1 < N) {
+        bb[i] = __ldg(reinterpret_cast<const unsigned int*>(bias + col));
+      } else {
+        const unsigned short lo =
+            col < N ? __ldg(reinterpret_cast<const unsigned short*>(bias + col)) : 0;
+        bb[i] = lo;
+      }
+    }
+  }
+}
+
+// Bias and activation in fp32, then RNE to fp16, of one 64-column chunk of a
+// warp's 32 accumulator rows already in registers (`v`: 64 fp32 bit
+// patterns of this thread's row) into 32 packed pairs `h`.
+template <int ACT>
+__device__ __forceinline__ void convert_chunk(const uint32_t* v, const __half* __restrict__ bias,
+                                              int col0, int N, uint32_t* h) {
+  uint32_t bb[32];
+  if (bias != nullptr) load_bias_chunk(bias, col0, N, bb);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    // columns 2i, 2i + 1 and 32 + 2i, 32 + 2i + 1 of the chunk, in pairs
+    float2 xv = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+    float2 yv = make_float2(__uint_as_float(v[32 + 2 * i]), __uint_as_float(v[32 + 2 * i + 1]));
+    if (bias != nullptr) {
+      xv = __fadd2_rn(xv, __half22float2(*reinterpret_cast<const __half2*>(&bb[i])));
+      yv = __fadd2_rn(yv, __half22float2(*reinterpret_cast<const __half2*>(&bb[16 + i])));
+    }
+    xv = activate2<ACT>(xv);
+    yv = activate2<ACT>(yv);
+    h[i] = pack_half2(xv.x, xv.y);
+    h[16 + i] = pack_half2(yv.x, yv.y);
+  }
+}
+
+// The converted chunk `h` (row `lane` of a 32 x 64 fp16 box) -> 128-byte
+// swizzled staging row per thread -> TMA store of the box (BOXES boxes per
+// warp in turn).  Columns at and beyond N rounded down to 8 (the TMA store
+// writes whole 16-byte groups) are written with plain stores.
+template <int BOXES>
+__device__ __forceinline__ void stage_chunk(const uint32_t* h, uint8_t* bufs, uint32_t& chunk_no,
+                                            const CUtensorMap* tmC, __half* C, int64_t ldc,
+                                            int M, int N, int n8, int row0, int col0, int lane) {
+  uint8_t* buf = bufs + (chunk_no % BOXES) * kEpiBuf;
+  // the store that last used `buf` has read it
+  if (lane == 0) bulk_wait_group_read<BOXES - 1>();
+  __syncwarp();
+  // row `lane`, 128 bytes = 8 chunks of 16 bytes, chunk j stored at j ^ (row & 7)
+  const uint32_t row_addr = smem_u32(buf) + lane * 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), h[4 * j], h[4 * j + 1], h[4 * j + 2],
+                 h[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    if (row0 < M && col0 < n8) tma_store_2d(tmC, buf, col0, row0);
+    bulk_commit_group();
+  }
+  if (n8 < N && col0 + kEpiCols > n8 && col0 < N && row0 + lane < M) {
+    // ragged tail columns [max(n8, col0), min(N, col0 + 64)) of this row,
+    // read back from this thread's own (swizzled) staging row
+    const int j_end = min(N, col0 + kEpiCols);
+    __half* crow = C + static_cast<int64_t>(row0 + lane) * ldc;
+    for (int j = max(n8, col0); j < j_end; ++j) {
+      const int cc = j - col0;
+      const uint32_t addr = row_addr + ((((cc >> 3) ^ (lane & 7)) << 4) | ((cc & 7) << 1));
+      unsigned short bits;
+      asm volatile("ld.shared.u16 %0, [%1];" : "=h"(bits) : "r"(addr) : "memory");
+      crow[j] = __ushort_as_half(bits);
+    }
+  }
+  ++chunk_no;
+}
+
 // Epilogue of one accumulator tile, run by one warp for its 32 TMEM lanes and
-// COLS of the tile's columns: tcgen05.ld 64 columns at a time -> bias and
-// activation in fp32 -> RNE to fp16 -> 128-byte swizzled staging row per
-// thread -> TMA store of a 32 x 64 box (BOXES boxes per warp in turn).  Columns at and beyond N rounded down to 8 (the TMA
-// store writes whole 16-byte groups) are written with plain stores.
+// COLS of the tile's columns, 64 at a time: tcgen05.ld -> convert_chunk ->
+// stage_chunk.
 // `release()` runs once the last TMEM load of the tile has completed.
 // `bias` (N fp16 values or null) is added per column before the activation.
+// With COLS = 128, `early` set and no GELU, both chunks are read with one
+// 128-column load first, so the accumulator is handed back before any chunk
+// is converted or stored.
 template <int COLS, int BOXES, int ACT, class Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uint32_t& chunk_no,
                                               const CUtensorMap* tmC, __half* C, int64_t ldc,
                                               const __half* __restrict__ bias, int M, int N,
                                               int n8, int row0, int col_base, int lane,
-                                              Release release) {
+                                              Release release, bool early = false) {
+  // (not with GELU, whose arithmetic next to 128 live values exceeds the 168
+  // registers a thread of a 10-warp CTA may hold)
+  if constexpr (COLS == 128 && ACT != kActGelu) {
+    if (early) {
+      uint32_t v[128];
+      tmem_load_32x32b_x128(t_row, v);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) release();
+      uint32_t h[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) convert_chunk<ACT>(v + 64 * c, bias, col_base + c * kEpiCols, N,
+                                                    h + 32 * c);
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        stage_chunk<BOXES>(h + 32 * c, bufs, chunk_no, tmC, C, ldc, M, N, n8, row0,
+                           col_base + c * kEpiCols, lane);
+      return;
+    }
+  }
 #pragma unroll 1
   for (int c = 0; c < COLS / kEpiCols; ++c) {
-    // the 64 bias values of this chunk as 32 packed pairs (0 past N): eight
-    // 16-byte loads (the same address in every lane) when the chunk lies
-    // inside N, else pair by pair
-    uint32_t bb[32];
-    if (bias != nullptr) {
-      const int col0 = col_base + c * kEpiCols;
-      if (col0 + kEpiCols <= N) {
-        const uint4* src = reinterpret_cast<const uint4*>(bias + col0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 q = __ldg(src + i);
-          bb[4 * i] = q.x;
-          bb[4 * i + 1] = q.y;
-          bb[4 * i + 2] = q.z;
-          bb[4 * i + 3] = q.w;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = col0 + 2 * i;
-          if (col + 1 < N) {
-            bb[i] = __ldg(reinterpret_cast<const unsigned int*>(bias + col));
-          } else {
-            const unsigned short lo =
-                col < N ? __ldg(reinterpret_cast<const unsigned short*>(bias + col)) : 0;
-            bb[i] = lo;
-          }
-        }
-      }
-    }
     uint32_t v[64];
     tmem_load_32x32b_x64(t_row + c * kEpiCols, v);
     if (c == COLS / kEpiCols - 1) {
@@ -246,51 +331,9 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
       if (lane == 0) release();
     }
     uint32_t h[32];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      // columns 2i, 2i + 1 and 32 + 2i, 32 + 2i + 1 of the chunk, in pairs
-      float2 xv = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-      float2 yv = make_float2(__uint_as_float(v[32 + 2 * i]), __uint_as_float(v[32 + 2 * i + 1]));
-      if (bias != nullptr) {
-        xv = __fadd2_rn(xv, __half22float2(*reinterpret_cast<const __half2*>(&bb[i])));
-        yv = __fadd2_rn(yv, __half22float2(*reinterpret_cast<const __half2*>(&bb[16 + i])));
-      }
-      xv = activate2<ACT>(xv);
-      yv = activate2<ACT>(yv);
-      h[i] = pack_half2(xv.x, xv.y);
-      h[16 + i] = pack_half2(yv.x, yv.y);
-    }
-    uint8_t* buf = bufs + (chunk_no % BOXES) * kEpiBuf;
-    // the store that last used `buf` has read it
-    if (lane == 0) bulk_wait_group_read<BOXES - 1>();
-    __syncwarp();
-    // row `lane`, 128 bytes = 8 chunks of 16 bytes, chunk j stored at j ^ (row & 7)
-    const uint32_t row_addr = smem_u32(buf) + lane * 128;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      st_shared_v4(row_addr + ((j ^ (lane & 7)) << 4), h[4 * j], h[4 * j + 1], h[4 * j + 2],
-                   h[4 * j + 3]);
-    fence_proxy_async_smem();
-    __syncwarp();
-    const int col0 = col_base + c * kEpiCols;
-    if (lane == 0) {
-      if (row0 < M && col0 < n8) tma_store_2d(tmC, buf, col0, row0);
-      bulk_commit_group();
-    }
-    if (n8 < N && col0 + kEpiCols > n8 && col0 < N && row0 + lane < M) {
-      // ragged tail columns [max(n8, col0), min(N, col0 + 64)) of this row,
-      // read back from this thread's own (swizzled) staging row
-      const int j_end = min(N, col0 + kEpiCols);
-      __half* crow = C + static_cast<int64_t>(row0 + lane) * ldc;
-      for (int j = max(n8, col0); j < j_end; ++j) {
-        const int cc = j - col0;
-        const uint32_t addr = row_addr + ((((cc >> 3) ^ (lane & 7)) << 4) | ((cc & 7) << 1));
-        unsigned short bits;
-        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(bits) : "r"(addr) : "memory");
-        crow[j] = __ushort_as_half(bits);
-      }
-    }
-    ++chunk_no;
+    convert_chunk<ACT>(v, bias, col_base + c * kEpiCols, N, h);
+    stage_chunk<BOXES>(h, bufs, chunk_no, tmC, C, ldc, M, N, n8, row0, col_base + c * kEpiCols,
+                       lane);
   }
 }
 
@@ -526,8 +569,8 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
                           int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
-                          int layout, int group_m, int split_from, int l2_hint, int* status,
-                          uint64_t timeout_ns) {
+                          int layout, int group_m, int split_from, int l2_hint, int epi_early,
+                          int* status, uint64_t timeout_ns) {
   using Cfg = PairCfg<STAGES, SLABS>;
   const bool ta = (layout & kLayoutTransA) != 0;
   const bool tb = (layout & kLayoutTransB) != 0;
@@ -837,7 +880,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
                                static_cast<uint32_t>((acc * SLABS + s) * BN + g * kCols);
         epilogue_tile<kCols, Cfg::kEpiBoxes, ACT>(
             t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0, nb * BN + g * kCols, lane,
-            [release_bar] { mbar_arrive_cluster(release_bar); });
+            [release_bar] { mbar_arrive_cluster(release_bar); }, epi_early != 0);
       }
       if (++acc == NBUF) {
         acc = 0;
@@ -895,6 +938,17 @@ int group_tiles(int group, int tile_rows, int tile_cols) {
   }
   const int g = group / tile_rows;
   return g > 0 ? g : 1;
+}
+
+// Whether the 512-row pair tile's epilogue reads a warp's 128 columns with
+// one load and hands the accumulator back before converting them: TTC_EPI in
+// the environment (0 or 1), read once, else 0.
+int epi_early_code() {
+  static const int code = [] {
+    const char* s = std::getenv("TTC_EPI");
+    return (s != nullptr && s[0] == '1') ? 1 : 0;
+  }();
+  return code;
 }
 
 // The L2 hint code of the pair kernels' operand loads (see l2_policy_for):
@@ -997,7 +1051,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
       static_cast<int>(p.K), p.layout, group_tiles(group_rows, Cfg::kTileM, Cfg::kBN),
-      static_cast<int>(split_from), l2_hint_code(), d.status, d.timeout_ns);
+      static_cast<int>(split_from), l2_hint_code(), epi_early_code(), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 
