@@ -50,6 +50,10 @@ KERNEL_SOURCES = {
     "tile_gemm_kernel": ["tiled_tensor_core_05_b200/csrc/gemm_tile.cu",
                          "tiled_tensor_core_05_b200/csrc/sm100.cuh"],
     "skinny_gemm_kernel": ["tiled_tensor_core_05_b200/csrc/gemm_skinny.cu",
+                           "tiled_tensor_core_05_b200/csrc/skinny_common.cuh",
+                           "tiled_tensor_core_05_b200/csrc/sm100.cuh"],
+    "skinny_even_kernel": ["tiled_tensor_core_05_b200/csrc/gemm_skinny_even.cu",
+                           "tiled_tensor_core_05_b200/csrc/skinny_common.cuh",
                            "tiled_tensor_core_05_b200/csrc/sm100.cuh"],
 }
 
@@ -298,7 +302,8 @@ def kernel_for(w) -> str:
     from tiled_tensor_core_05_b200 import ops
     return {ops.PATH_SKINNY: "skinny_gemm_kernel", ops.PATH_TILE: "tile_gemm_kernel",
             ops.PATH_TILE_PAIR: "tile_pair_gemm_kernel",
-            ops.PATH_TILE_PAIR_TALL: "tile_pair_gemm_kernel"}[ops.select_path(w.M, w.N, w.K)]
+            ops.PATH_TILE_PAIR_TALL: "tile_pair_gemm_kernel",
+            ops.PATH_SKINNY_EVEN: "skinny_even_kernel"}[ops.select_path(w.M, w.N, w.K)]
 
 
 def roofline_entry(name, launch_ms, peaks, peak_src, long_run: bool, variant: str = "relu"):

@@ -78,10 +78,12 @@ enum gemm_status {
 };
 
 enum gemm_path {
-  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY; fewer than 64 tiles of
-                              256 x 256 -> TILE; K < 3072 (6144 with GELU) -> TILE_PAIR;
-                              otherwise TILE_PAIR_TALL, or TILE_PAIR when the 512-row
-                              tiles leave a much emptier last wave */
+  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY_EVEN when its busiest SM
+                              streams >= 10 % less of B than SKINNY's tiling, else
+                              SKINNY; fewer than 64 tiles of 256 x 256 -> TILE; K < 3072
+                              (6144 with GELU) -> TILE_PAIR; otherwise TILE_PAIR_TALL, or
+                              TILE_PAIR when the 512-row tiles leave a much emptier
+                              last wave */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile, BN = 64, 128 or
                               256 by the tile count (any shape) */
   GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 128 columns of B per CTA when
@@ -89,9 +91,14 @@ enum gemm_path {
                               split-K only when tiles < SMs (M <= 64 only) */
   GEMM_PATH_TILE_PAIR = 3, /* persistent kernel, two SMs (a CTA pair) per 256 x 256 tile
                               (any shape) */
-  GEMM_PATH_TILE_PAIR_TALL = 4 /* persistent kernel, a CTA pair per 512 x 256 tile: fewer
-                                  bytes staged per MAC; a single accumulator, so a tile's
-                                  epilogue overlaps only the start of the next tile */
+  GEMM_PATH_TILE_PAIR_TALL = 4, /* persistent kernel, a CTA pair per 512 x 256 tile: fewer
+                                   bytes staged per MAC; a single accumulator, so a tile's
+                                   epilogue overlaps only the start of the next tile */
+  GEMM_PATH_SKINNY_EVEN = 5 /* small-M kernel with the same bytes of B on every SM: one
+                               CTA per SM with q = floor(ceil(N / 64) / SMs) whole
+                               64-column units for the full K, the leftover units split
+                               along K over the CTAs with a deterministic fix-up (M <= 64
+                               and 1 <= q <= 4 only; GEMM_ERR_INVALID_ARG otherwise) */
 };
 
 enum gemm_activation {
@@ -154,19 +161,23 @@ GEMM_API int gemm_f16_general(const void* A, const void* B, const void* bias, vo
  * (the library itself never times or chooses among these at run time).
  * A field left at 0 takes the value GEMM_PATH_AUTO would use. */
 typedef struct gemm_config {
-  int32_t kernel;     /* GEMM_PATH_TILE, _TILE_PAIR, _TILE_PAIR_TALL or _SKINNY (not AUTO) */
+  int32_t kernel;     /* GEMM_PATH_TILE, _TILE_PAIR, _TILE_PAIR_TALL, _SKINNY or
+                         _SKINNY_EVEN (not AUTO) */
   int32_t block_n;    /* output columns per tile: 64, 128 or 256 for GEMM_PATH_TILE; 128
                          or 256 for GEMM_PATH_SKINNY; 256 (the only width) for the pair
-                         kernels */
+                         kernels; for GEMM_PATH_SKINNY_EVEN the main columns per CTA,
+                         64 q (fixed by the shape: 0 takes it, another value is
+                         GEMM_ERR_CONFIG) */
   int32_t stages;     /* depth of the shared-memory operand ring (k-blocks of 64 in flight) */
   int32_t group_rows; /* tile kernels: the L2 grouping of the tile order.  > 0: rows of
                          op(A) per row panel (tiles walked column by column inside
                          it); < 0: minus the columns of op(B) per column panel (tiles
                          walked row by row inside it); 0 = the default.  Must be 0 for
-                         GEMM_PATH_SKINNY */
+                         the small-M kernels */
   int32_t splits;     /* GEMM_PATH_SKINNY: k-slices per column tile, 1 <= splits <=
                          ceil(K / 64) and splits * ceil(N / block_n) <= the SM count when
-                         > 1; 0 = chosen from the shape.  Must be 0 for the tile kernels */
+                         > 1; 0 = chosen from the shape.  Must be 0 for the tile kernels
+                         and GEMM_PATH_SKINNY_EVEN */
 } gemm_config;
 
 /* gemm_f16_general with the kernel configuration `cfg` instead of a path.

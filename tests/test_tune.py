@@ -17,13 +17,16 @@ def lib():
 
 def test_built_configs_are_exactly_those_within_the_budget(lib):
     built = {(c.kernel, c.block_n, c.stages) for c in ops.config_list()}
-    kinds = tune.TILE_KINDS + [(ops.PATH_SKINNY, w) for w in tune.SKINNY_WIDTHS]
+    kinds = tune.TILE_KINDS + [(ops.PATH_SKINNY, w) for w in tune.SKINNY_WIDTHS] + \
+        [(ops.PATH_SKINNY_EVEN, w) for w in tune.EVEN_WIDTHS]
     expect = set()
     for kernel, bn in kinds:
         for st in range(3, 17):
             if ops.config_smem_bytes({"kernel": kernel, "block_n": bn, "stages": st}) > BUDGET:
                 continue
             if kernel == ops.PATH_SKINNY and st > 6:  # the small-M ring's depth cap
+                continue
+            if kernel == ops.PATH_SKINNY_EVEN and st not in tune.EVEN_STAGES:
                 continue
             expect.add((kernel, bn, st))
     assert built == expect
@@ -45,6 +48,12 @@ def test_smem_formula(lib):
         1024 + 5 * 40960 + 13 * 8 + 16
     assert ops.config_smem_bytes({"kernel": 2, "block_n": 128, "stages": 6}) == \
         1024 + 6 * 24576 + 15 * 8 + 16
+    # the even small-M schedule: max(q, 2) slabs of 8 KiB of B + 8 KiB of A per stage
+    assert ops.config_smem_bytes({"kernel": 5, "block_n": 192, "stages": 6}) == \
+        1024 + 6 * (3 * 8192 + 8192) + 16 * 8 + 16
+    assert ops.config_smem_bytes({"kernel": 5, "block_n": 64, "stages": 4}) == \
+        1024 + 4 * (2 * 8192 + 8192) + 12 * 8 + 16
+    assert ops.config_smem_bytes({"kernel": 5, "block_n": 96, "stages": 4}) == -8
     assert ops.config_smem_bytes({"kernel": 2, "block_n": 64, "stages": 4}) == -8
     assert ops.config_smem_bytes({"kernel": 2, "stages": 4}) == -8  # width must be given
     # defaults when stages = 0; AUTO and bad widths name no kernel
@@ -121,3 +130,15 @@ def test_host_plan_candidates():
     assert {"split": ops.HOST_SPLIT_COLS, "panel_extent": 1024} not in d
     assert [p for p in d if p["split"] == ops.HOST_SPLIT_ROWS] == [
         {"split": ops.HOST_SPLIT_ROWS, "panel_extent": 32}]
+
+
+def test_candidates_decode_include_the_even_schedule(lib):
+    kept, _ = tune.candidates(32, 28672, 8192, 148, ops.config_smem_bytes)
+    even = [c for c in kept if c["kernel"] == ops.PATH_SKINNY_EVEN]
+    # 448 units of 64 columns on 148 SMs: 3 whole units per CTA
+    assert {c["block_n"] for c in even} == {192}
+    within = {st for st in tune.STAGE_RANGE
+              if ops.config_smem_bytes({"kernel": 5, "block_n": 192, "stages": st}) <= BUDGET}
+    assert {c["stages"] for c in even} == within
+    kept, _ = tune.candidates(32, 4096, 8192, 148, ops.config_smem_bytes)
+    assert not [c for c in kept if c["kernel"] == ops.PATH_SKINNY_EVEN]  # 64 units < 148

@@ -23,8 +23,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libttc05.so")
-SOURCES = ["gemm_api.cu", "gemm_tile.cu", "gemm_skinny.cu", "gemm_host.cu"]
-HEADERS = ["sm100.cuh", "internal.h"]
+SOURCES = ["gemm_api.cu", "gemm_tile.cu", "gemm_skinny.cu", "gemm_skinny_even.cu", "gemm_host.cu"]
+HEADERS = ["sm100.cuh", "internal.h", "skinny_common.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC",

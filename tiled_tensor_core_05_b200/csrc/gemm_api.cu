@@ -372,8 +372,17 @@ double wave_efficiency(int64_t tiles, int64_t pairs) {
 // So the 512-row tile is taken from K = 3072 (6144 with GELU) unless its last
 // wave wastes more than 6 points more of the SM pairs than the 256-row
 // tiling's (the MLP up-projection with ReLU: 93 % against 97 %, still faster).
+//
+// Small M (<= 64): the even schedule when its busiest SM streams at least 10 %
+// fewer k-blocks of B than the small-M kernel's default tiling would (e.g. the
+// decode shape: 388 against 512), else the small-M kernel.
 int select_path_for(int64_t M, int64_t N, int64_t K, int sm_count, int activation) {
-  if (M >= 1 && M <= 64) return GEMM_PATH_SKINNY;
+  if (M >= 1 && M <= 64) {
+    const EvenPlan plan = even_plan(N, K, sm_count);
+    if (plan.q > 0 && 10 * plan.work <= 9 * skinny_default_work(N, K, sm_count))
+      return GEMM_PATH_SKINNY_EVEN;
+    return GEMM_PATH_SKINNY;
+  }
   const int64_t pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
   const int64_t col_tiles = (N + 255) / 256;
   const int64_t tiles256 = ((M + 255) / 256) * col_tiles;
@@ -393,6 +402,7 @@ int default_stages(int kernel, int block_n) {
     case GEMM_PATH_TILE_PAIR: return kDefaultStagesPair;
     case GEMM_PATH_TILE_PAIR_TALL: return kDefaultStagesTall;
     case GEMM_PATH_SKINNY: return block_n == 128 ? kDefaultStagesSkinnyNarrow : kDefaultStagesSkinny;
+    case GEMM_PATH_SKINNY_EVEN: return block_n == 256 ? kDefaultStagesEven4 : kDefaultStagesEven;
     default: return 0;
   }
 }
@@ -400,9 +410,8 @@ int default_stages(int kernel, int block_n) {
 // Fills the fields of `c` left at 0 with what GEMM_PATH_AUTO would use for an
 // M x N output and checks the rest (the stage count is checked against the
 // compiled kernels at launch).  Returns GEMM_OK or GEMM_ERR_CONFIG.
-int resolve_config(KernelConfig& c, int64_t M, int64_t N, int sm_count) {
+int resolve_config(KernelConfig& c, int64_t M, int64_t N, int64_t K, int sm_count) {
   if (c.stages < 0 || c.splits < 0) return GEMM_ERR_CONFIG;
-  if (c.group_rows < 0 && c.kernel == GEMM_PATH_SKINNY) return GEMM_ERR_CONFIG;
   switch (c.kernel) {
     case GEMM_PATH_TILE:
       if (c.block_n == 0) {
@@ -424,11 +433,20 @@ int resolve_config(KernelConfig& c, int64_t M, int64_t N, int sm_count) {
       if (c.block_n == 0) c.block_n = (N + 127) / 128 <= sm_count ? 128 : 256;
       if (c.block_n != 128 && c.block_n != 256) return GEMM_ERR_CONFIG;
       break;
+    case GEMM_PATH_SKINNY_EVEN: {
+      const EvenPlan plan = even_plan(N, K, sm_count);
+      if (plan.q == 0) return GEMM_ERR_CONFIG;
+      if (c.block_n == 0) c.block_n = 64 * plan.q;
+      if (c.block_n != 64 * plan.q) return GEMM_ERR_CONFIG;
+      break;
+    }
     default:
       return GEMM_ERR_CONFIG;
   }
   if (c.stages == 0) c.stages = default_stages(c.kernel, c.block_n);
-  if (c.kernel == GEMM_PATH_SKINNY) {
+  if (c.kernel == GEMM_PATH_SKINNY_EVEN) {
+    if (c.group_rows != 0 || c.splits != 0 || skinny_m_pad(M) == 0) return GEMM_ERR_CONFIG;
+  } else if (c.kernel == GEMM_PATH_SKINNY) {
     if (c.group_rows != 0 || skinny_m_pad(M) == 0) return GEMM_ERR_CONFIG;
   } else {
     if (c.splits != 0) return GEMM_ERR_CONFIG;
@@ -451,7 +469,7 @@ int run_gemm(const void* A, const void* B, const void* bias, void* C, int64_t M,
     return GEMM_ERR_INVALID_ARG;
   if (cfg == nullptr && path != GEMM_PATH_AUTO && path != GEMM_PATH_TILE &&
       path != GEMM_PATH_SKINNY && path != GEMM_PATH_TILE_PAIR &&
-      path != GEMM_PATH_TILE_PAIR_TALL)
+      path != GEMM_PATH_TILE_PAIR_TALL && path != GEMM_PATH_SKINNY_EVEN)
     return GEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return GEMM_OK;
   DeviceCtx d;
@@ -460,12 +478,12 @@ int run_gemm(const void* A, const void* B, const void* bias, void* C, int64_t M,
   KernelConfig kc{};
   if (cfg != nullptr) {
     kc = KernelConfig{cfg->kernel, cfg->block_n, cfg->stages, cfg->group_rows, cfg->splits};
-    rc = resolve_config(kc, M, N, d.sm_count);
+    rc = resolve_config(kc, M, N, K, d.sm_count);
     if (rc != GEMM_OK) return rc;
   } else {
     if (path == GEMM_PATH_AUTO) path = select_path_for(M, N, K, d.sm_count, activation);
     kc = KernelConfig{path, 0, 0, 0, 0};
-    if (resolve_config(kc, M, N, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
+    if (resolve_config(kc, M, N, K, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
   }
   load_entry_points();
   rc = check_matrix(C, M, N, ldc, d.device);
@@ -486,11 +504,12 @@ int run_gemm(const void* A, const void* B, const void* bias, void* C, int64_t M,
   if (rc == GEMM_OK)
     rc = trans_b ? check_matrix(B, N, K, ldb, d.device) : check_matrix(B, K, N, ldb, d.device);
   if (rc != GEMM_OK) return rc;
-  if (kc.kernel == GEMM_PATH_SKINNY) {
+  if (kc.kernel == GEMM_PATH_SKINNY || kc.kernel == GEMM_PATH_SKINNY_EVEN) {
     void* ws = nullptr;
     size_t ws_bytes = 0;
     rc = get_workspace(d, stream, &ws, &ws_bytes);
     if (rc != GEMM_OK) return rc;
+    if (kc.kernel == GEMM_PATH_SKINNY_EVEN) return launch_skinny_even(p, d, ws, ws_bytes, kc);
     return launch_skinny_gemm(p, d, ws, ws_bytes, kc);
   }
   return launch_tile_gemm(p, d, kc);
@@ -538,12 +557,15 @@ int gemm_f16_config(const void* A, const void* B, const void* bias, void* C, int
 int gemm_config_smem_bytes(const gemm_config* cfg) {
   if (cfg == nullptr) return GEMM_ERR_INVALID_ARG;
   int block_n = cfg->block_n;
-  if (block_n == 0 && cfg->kernel != GEMM_PATH_TILE && cfg->kernel != GEMM_PATH_SKINNY)
+  if (block_n == 0 && cfg->kernel != GEMM_PATH_TILE && cfg->kernel != GEMM_PATH_SKINNY &&
+      cfg->kernel != GEMM_PATH_SKINNY_EVEN)
     block_n = 256;
   const int stages = cfg->stages != 0 ? cfg->stages : default_stages(cfg->kernel, block_n);
   int bytes = -1;
   if (cfg->kernel == GEMM_PATH_SKINNY)
     bytes = skinny_config_smem_bytes(block_n, stages);
+  else if (cfg->kernel == GEMM_PATH_SKINNY_EVEN)
+    bytes = even_config_smem_bytes(block_n, stages);
   else
     bytes = tile_config_smem_bytes(cfg->kernel, block_n, stages);
   return bytes > 0 ? bytes : GEMM_ERR_CONFIG;
@@ -553,6 +575,7 @@ int gemm_config_list(gemm_config* out, int capacity) {
   KernelConfig all[64];
   int n = tile_configs_built(all, 64);
   n += skinny_configs_built(all + n, 64 - n);
+  n += even_configs_built(all + n, 64 - n);
   for (int i = 0; i < n && i < capacity && out != nullptr; ++i)
     out[i] = gemm_config{all[i].kernel, all[i].block_n, all[i].stages, 0, 0};
   return n;
@@ -569,7 +592,7 @@ int gemm_auto_config(int64_t M, int64_t N, int64_t K, int activation, gemm_confi
   const int rc = get_device(&d);
   if (rc != GEMM_OK) return rc;
   KernelConfig c{select_path_for(M, N, K, d.sm_count, activation), 0, 0, 0, 0};
-  if (resolve_config(c, M, N, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
+  if (resolve_config(c, M, N, K, d.sm_count) != GEMM_OK) return GEMM_ERR_INVALID_ARG;
   *out = gemm_config{c.kernel, c.block_n, c.stages, c.group_rows, c.splits};
   return GEMM_OK;
 }

@@ -32,17 +32,14 @@
 
 #include "../../include/gemm_f16.h"
 #include "internal.h"
+#include "skinny_common.cuh"
 #include "sm100.cuh"
 
 namespace ttc {
 namespace {
 
+using namespace skinny;
 constexpr int kMaxTW = 256;    // widest tile: columns of B (rows of C^T) per CTA
-constexpr int kSub = 128;      // columns per MMA (MMA M)
-constexpr int kBK = 64;        // k-depth of a stage: one 128-byte swizzle row of A
-constexpr int kUmmaK = 16;
-constexpr int kThreads = 192;  // producer, MMA, 4 epilogue warps
-constexpr int kEpiWarps = 4;
 
 // Dynamic shared memory of the small-M kernel with `tw` columns of B per CTA:
 // 1 KiB of alignment slack, the ring (tw columns of B and room for A^T per
@@ -100,53 +97,6 @@ constexpr bool skinny_variants_complete() {
 }
 static_assert(skinny_variants_complete(),
               "built skinny configurations != those within the budget and depth cap");
-
-__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
-  return __ldcg(reinterpret_cast<const float4*>(p));
-}
-
-// Column n of C (rows m < M): activation of the fp32 sums plus the column's
-// bias, rounded to fp16.
-template <int MP, int ACT>
-__device__ __forceinline__ void store_column(const float (&v)[MP], __half* C, int M, int N,
-                                             int64_t ldc, int n, const __half* bias) {
-  if (n >= N) return;
-  const float b = bias != nullptr ? __half2float(bias[n]) : 0.0f;
-#pragma unroll
-  for (int m = 0; m < MP; m += 2) {
-    const float2 x = activate2<ACT>(__fadd2_rn(make_float2(v[m], v[m + 1]), splat2(b)));
-    if (m < M) C[static_cast<int64_t>(m) * ldc + n] = __float2half_rn(x.x);
-    if (m + 1 < M) C[static_cast<int64_t>(m + 1) * ldc + n] = __float2half_rn(x.y);
-  }
-}
-
-// Rows m0 .. m0 + 31 (those < M) of column n of C from 32 fp32 sums, as
-// store_column does for all MP rows.
-template <int ACT>
-__device__ __forceinline__ void store_rows(const float (&v)[32], __half* C, int M, int N,
-                                           int64_t ldc, int n, int m0, const __half* bias) {
-  if (n >= N) return;
-  const float b = bias != nullptr ? __half2float(bias[n]) : 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const float2 x = activate2<ACT>(__fadd2_rn(make_float2(v[i], v[i + 1]), splat2(b)));
-    const int m = m0 + i;
-    if (m < M) C[static_cast<int64_t>(m) * ldc + n] = __float2half_rn(x.x);
-    if (m + 1 < M) C[static_cast<int64_t>(m + 1) * ldc + n] = __float2half_rn(x.y);
-  }
-}
-
-// MP fp32 accumulator columns of this thread's TMEM lane.
-template <int MP>
-__device__ __forceinline__ void load_accumulator(uint32_t taddr, float (&v)[MP]) {
-#pragma unroll
-  for (int j = 0; j < MP / 32; ++j) {
-    uint32_t r[32];
-    tmem_load_32x32b_x32(taddr + j * 32, r);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[j * 32 + i] = __uint_as_float(r[i]);
-  }
-}
 
 // One CTA per (tile, k-slice); blockIdx.x = tile * S + slice.  B (streamed
 // once) is loaded with an L2 evict-first policy and A (re-read by every CTA)
@@ -395,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   }
                 }
               }
-              store_rows<ACT>(acc, C, M, N, ldc, n0 + h * kSub, mc * 32, bias);
+              store_rows<32, ACT>(acc, C, M, N, ldc, n0 + h * kSub, mc * 32, bias);
             }
           }
         }
@@ -410,21 +360,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, Cfg::kTmemCols);
   }
-}
-
-bool ensure_smem_attr_skinny(const void* func, int bytes, int device,
-                             std::atomic<uint64_t>& done) {
-  const uint64_t bit = 1ull << (device & 63);
-  if (done.load(std::memory_order_acquire) & bit) return true;
-  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-      cudaSuccess)
-    return false;
-  done.fetch_or(bit, std::memory_order_acq_rel);
-  return true;
-}
-
-constexpr size_t counter_bytes(int n) {
-  return (static_cast<size_t>(n) * sizeof(int) + 255) & ~static_cast<size_t>(255);
 }
 
 // Number of k-slices per tile: 1 when the tiles already cover the SMs,
@@ -482,8 +417,8 @@ int launch_impl(const GemmProblem& p, const DeviceCtx& d, void* ws, size_t ws_by
     rc = encode_tmap_f16_2d(&tB, p.B, p.N, p.K, p.ldb, 64, kBK);
   if (rc != 0) return rc;
   auto kern = skinny_gemm_kernel<MP, STAGES, TW, ACT>;
-  if (!ensure_smem_attr_skinny(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
-                               attr_done))
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, d.device,
+                        attr_done))
     return GEMM_ERR_LAUNCH;
   const int64_t grid = tiles * S;
   if (grid > INT32_MAX) return GEMM_ERR_INVALID_ARG;
@@ -508,6 +443,16 @@ int skinny_m_pad(int64_t M) {
   if (M <= 32) return 32;
   if (M <= 64) return 64;
   return 0;
+}
+
+int64_t skinny_default_work(int64_t N, int64_t K, int sm_count) {
+  const int64_t KB = (K + kBK - 1) / kBK;
+  const int tw = (N + 127) / 128 <= sm_count ? 128 : 256;
+  const int64_t tiles = (N + tw - 1) / tw;
+  const int S = choose_slices(tiles, KB, 32, tw, sm_count, sm_count);
+  const int64_t items = tiles * S;
+  const int64_t waves = (items + sm_count - 1) / sm_count;
+  return waves * (tw / 64) * ((KB + S - 1) / S);
 }
 
 size_t skinny_workspace_bytes(int sm_count, int m_pad) {

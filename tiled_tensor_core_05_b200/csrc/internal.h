@@ -22,7 +22,7 @@ struct GemmProblem {
 // One kernel configuration, resolved (no zero "default" fields left): the
 // validated form of the public gemm_config.
 struct KernelConfig {
-  int kernel;      // GEMM_PATH_TILE / _TILE_PAIR / _TILE_PAIR_TALL / _SKINNY
+  int kernel;      // GEMM_PATH_TILE / _TILE_PAIR / _TILE_PAIR_TALL / _SKINNY / _SKINNY_EVEN
   int block_n;     // output columns per CTA (TILE: 128 or 256) or per pair / tile (256)
   int stages;      // depth of the shared-memory operand ring
   int group_rows;  // tile kernels: rows of A per raster panel
@@ -48,6 +48,10 @@ constexpr int kDefaultStagesSkinny = 4;
 // faster than 256-column tiles there; on N = 28672 (224 narrow tiles) the
 // wide ones are 1.3x faster.
 constexpr int kDefaultStagesSkinnyNarrow = 6;
+// The even small-M schedule: 6 stages (5 with four units per CTA, the
+// deepest ring that fits), about 144-200 KiB in flight per SM.
+constexpr int kDefaultStagesEven = 6;
+constexpr int kDefaultStagesEven4 = 5;
 
 struct DeviceCtx {
   int device;
@@ -94,6 +98,28 @@ int launch_skinny_gemm(const GemmProblem& p, const DeviceCtx& d, void* workspace
 int skinny_m_pad(int64_t M);  // MMA N used for M rows (0 if M is too large)
 int skinny_config_smem_bytes(int block_n, int stages);  // -1 when block_n is not 128 / 256
 int skinny_configs_built(KernelConfig* out, int cap);
+
+// Even small-M schedule (gemm_skinny_even.cu): one CTA per SM, each with q
+// whole 64-column units of B for the full K, the left_units leftover units
+// split along K into left_slices slices each.  q == 0 when the shape does not
+// suit it (fewer units than SMs, or more than four per SM).  `work` is the
+// busiest CTA's k-blocks of 64 columns.
+struct EvenPlan {
+  int q;
+  int ctas;
+  int left_units;
+  int left_slices;
+  int64_t work;
+};
+EvenPlan even_plan(int64_t N, int64_t K, int sm_count);
+size_t even_workspace_bytes(const EvenPlan& plan, int m_pad);
+int launch_skinny_even(const GemmProblem& p, const DeviceCtx& d, void* workspace,
+                       size_t workspace_bytes, const KernelConfig& c);
+int even_config_smem_bytes(int block_n, int stages);  // -1 when block_n is not 64 q, q in 1..4
+int even_configs_built(KernelConfig* out, int cap);
+// The busiest CTA's k-blocks of 64 columns in the default configuration of
+// the small-M kernel (gemm_skinny.cu) for this shape, waves included.
+int64_t skinny_default_work(int64_t N, int64_t K, int sm_count);
 
 // The small-M kernel with its scratch in a fixed device array of the library
 // (no allocation); M <= 32.  Returns GEMM_ERR_SCRATCH_LIMIT beyond.

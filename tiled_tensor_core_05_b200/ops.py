@@ -25,6 +25,7 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libttc05.so")
 
 PATH_AUTO, PATH_TILE, PATH_SKINNY, PATH_TILE_PAIR, PATH_TILE_PAIR_TALL = 0, 1, 2, 3, 4
+PATH_SKINNY_EVEN = 5
 ACT_NONE, ACT_RELU, ACT_GELU = 0, 1, 2
 _ACTS = {"none": ACT_NONE, "relu": ACT_RELU, "gelu": ACT_GELU}
 

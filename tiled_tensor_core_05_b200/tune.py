@@ -60,14 +60,19 @@ TILE_KINDS = [(ops.PATH_TILE, 64), (ops.PATH_TILE, 128), (ops.PATH_TILE, 256),
               (ops.PATH_TILE_PAIR, 256), (ops.PATH_TILE_PAIR_TALL, 256)]
 TILE_ROWS = {ops.PATH_TILE: 128, ops.PATH_TILE_PAIR: 256, ops.PATH_TILE_PAIR_TALL: 512}
 KERNEL_NAMES = {ops.PATH_TILE: "tile", ops.PATH_SKINNY: "skinny",
-                ops.PATH_TILE_PAIR: "pair", ops.PATH_TILE_PAIR_TALL: "pair-tall"}
+                ops.PATH_TILE_PAIR: "pair", ops.PATH_TILE_PAIR_TALL: "pair-tall",
+                ops.PATH_SKINNY_EVEN: "skinny-even"}
 SKINNY_WIDTHS = (128, 256)
+EVEN_WIDTHS = (64, 128, 192, 256)  # 64 q columns per CTA, q whole 64-column units
+EVEN_STAGES = range(4, 7)          # the compiled depths of the even small-M schedule
 
 def describe(cfg: dict) -> str:
     k = cfg["kernel"]
     if k == ops.PATH_SKINNY:
         s = cfg["splits"]
         return f"skinny {cfg['block_n']} st{cfg['stages']} splits={'auto' if s == 0 else s}"
+    if k == ops.PATH_SKINNY_EVEN:
+        return f"skinny-even {cfg['block_n']} st{cfg['stages']}"
     rows = TILE_ROWS[k]
     return (f"{KERNEL_NAMES[k]} {rows}x{cfg['block_n']} st{cfg['stages']} "
             f"panel={cfg['group_rows']}")
@@ -82,6 +87,11 @@ def candidates(M: int, N: int, K: int, sm_count: int, smem_fn, budget: int = SME
     kinds = list(TILE_KINDS)
     if M <= 64:
         kinds += [(ops.PATH_SKINNY, w) for w in SKINNY_WIDTHS]
+        # the even schedule's width is fixed by the shape: 64 q, q whole
+        # 64-column units per SM (none when there are fewer units than SMs)
+        q = -(-N // 64) // sm_count
+        if 1 <= q <= 4:
+            kinds.append((ops.PATH_SKINNY_EVEN, 64 * q))
     for kernel, bn in kinds:
         for st in STAGE_RANGE:
             base = {"kernel": kernel, "block_n": bn, "stages": st, "group_rows": 0,
@@ -105,6 +115,8 @@ def candidates(M: int, N: int, K: int, sm_count: int, smem_fn, budget: int = SME
                         continue
                     seen.add(s)
                     kept.append({**base, "splits": s})
+            elif kernel == ops.PATH_SKINNY_EVEN:
+                kept.append(base)
             else:
                 rows = TILE_ROWS[kernel]
                 tile_rows = -(-M // rows)
