@@ -181,6 +181,33 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
   }
 }
 
+// Whether the (whole-tile) work unit `tile` is the first of the units running
+// together (the wave of `npairs` units that contains it) to read its A block
+// (bit 0) and its B block (bit 1) under the raster of tile_coords.  Only that
+// unit prefetches the block into L2, so the others find it there.
+__device__ __forceinline__ int first_reader(int tile, int num_m, int num_n, int group_m,
+                                            int npairs) {
+  const int wave_start = (tile / npairs) * npairs;
+  int own = 0;
+  if (group_m > 0) {
+    const int per_group = group_m * num_n;
+    const int g = tile / per_group;
+    const int rows = min(num_m - g * group_m, group_m);
+    const int r = tile - g * per_group;
+    if (r < rows || tile - rows < wave_start) own |= 1;  // first of its tile-row here
+    if (r % rows == 0 || tile - 1 < wave_start) own |= 2;  // first of its tile-column
+  } else {
+    const int group_n = -group_m;
+    const int per_group = group_n * num_m;
+    const int g = tile / per_group;
+    const int cols = min(num_n - g * group_n, group_n);
+    const int r = tile - g * per_group;
+    if (r < cols || tile - cols < wave_start) own |= 2;
+    if (r % cols == 0 || tile - 1 < wave_start) own |= 1;
+  }
+  return own;
+}
+
 // L2 eviction priority of the operand loads, one 2-bit field per operand
 // (bits 0-1 A, bits 2-3 B): 0 = no hint, 1 = evict-first, 2 = evict-normal,
 // 3 = evict-last.  The operand a raster panel re-reads across waves (A with
@@ -570,7 +597,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
                           int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
                           int layout, int group_m, int split_from, int l2_hint, int epi_early,
-                          int* status, uint64_t timeout_ns) {
+                          int pf_dist, int* status, uint64_t timeout_ns) {
   using Cfg = PairCfg<STAGES, SLABS>;
   const bool ta = (layout & kLayoutTransA) != 0;
   const bool tb = (layout & kLayoutTransB) != 0;
@@ -697,6 +724,42 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
             load_b(bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
           } else {
             load_b(bar, bdst, kb * kBK, b_col);
+          }
+          if (pf_dist > 0) {
+            // L2 prefetch of this CTA's part of k-block kb + pf_dist (of this
+            // unit, or of its next unit near the end), by the unit that reads
+            // the block first among those running together
+            int pu = unit, pk = kb + pf_dist;
+            if (pk >= num_kb) {
+              pu = unit + npairs;
+              pk -= num_kb;
+            }
+            if (pu < split_from && pk < num_kb) {
+              int pmb, pnb;
+              tile_coords(pu, num_m, num_n, group_m, pmb, pnb);
+              const int own = first_reader(pu, num_m, num_n, group_m, npairs);
+              if (own & 1) {
+                const int prow = pmb * Cfg::kTileM + static_cast<int>(rank) * kBM;
+#pragma unroll
+                for (int s = 0; s < SLABS; ++s) {
+                  if (!ta) {
+                    tma_prefetch_l2_2d(&tmA, pk * kBK, prow + s * 2 * kBM);
+                  } else {
+                    tma_prefetch_l2_2d(&tmA, prow + s * 2 * kBM, pk * kBK);
+                    tma_prefetch_l2_2d(&tmA, prow + s * 2 * kBM + 64, pk * kBK);
+                  }
+                }
+              }
+              if (own & 2) {
+                const int pcol = pnb * BN + static_cast<int>(rank) * 128;
+                if (!tb) {
+                  tma_prefetch_l2_2d(&tmB, pcol, pk * kBK);
+                  tma_prefetch_l2_2d(&tmB, pcol + 64, pk * kBK);
+                } else {
+                  tma_prefetch_l2_2d(&tmB, pk * kBK, pcol);
+                }
+              }
+            }
           }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -951,6 +1014,18 @@ int epi_early_code() {
   return code;
 }
 
+// L2 prefetch distance of the pair kernels in k-blocks (0 = none): TTC_PF in
+// the environment, read once.
+int prefetch_distance() {
+  static const int dist = [] {
+    const char* s = std::getenv("TTC_PF");
+    if (s == nullptr) return 0;
+    const int v = std::atoi(s);
+    return (v >= 0 && v <= 64) ? v : 0;
+  }();
+  return dist;
+}
+
 // The L2 hint code of the pair kernels' operand loads (see l2_policy_for):
 // TTC_L2HINT in the environment (a number 0-15), read once, else none.
 int l2_hint_code() {
@@ -1051,7 +1126,8 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
       static_cast<int>(p.K), p.layout, group_tiles(group_rows, Cfg::kTileM, Cfg::kBN),
-      static_cast<int>(split_from), l2_hint_code(), epi_early_code(), d.status, d.timeout_ns);
+      static_cast<int>(split_from), l2_hint_code(), epi_early_code(), prefetch_distance(),
+      d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 

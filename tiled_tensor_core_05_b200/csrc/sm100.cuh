@@ -150,6 +150,16 @@ __device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap* map, uint64_
       : "memory");
 }
 
+// Prefetch a 2-D tile of a tensor map into L2 (no shared memory, no
+// completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t c0,
+                                                   int32_t c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // 2-D tiled store shared -> global (out-of-range rows/columns are clipped).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src,
                                              int32_t c0, int32_t c1) {
