@@ -78,12 +78,11 @@ enum gemm_status {
 };
 
 enum gemm_path {
-  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY_EVEN when its busiest SM
-                              streams >= 10 % less of B than SKINNY's tiling, else
-                              SKINNY; fewer than 64 tiles of 256 x 256 -> TILE; K < 3072
-                              (6144 with GELU) -> TILE_PAIR; otherwise TILE_PAIR_TALL, or
-                              TILE_PAIR when the 512-row tiles leave a much emptier
-                              last wave */
+  GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY; fewer than 64 tiles of
+                              256 x 256 -> TILE; K < 3072 (6144 with GELU) -> TILE_PAIR;
+                              otherwise TILE_PAIR_TALL, or TILE_PAIR when the 512-row
+                              tiles leave a much emptier last wave (SKINNY_EVEN only
+                              when asked for) */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile, BN = 64, 128 or
                               256 by the tile count (any shape) */
   GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 128 columns of B per CTA when

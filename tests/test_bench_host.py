@@ -45,7 +45,7 @@ def test_roofline_arithmetic(lib):
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(d.bytes_min / 1e-4 / 1e9, rel=1e-4)
     assert d.bytes_min == 472121344
-    assert r["kernel"] == "skinny_even_kernel"
+    assert r["kernel"] == "skinny_gemm_kernel"
 
 
 def test_traffic_is_reported_only_for_the_captured_source(lib, tmp_path, monkeypatch):

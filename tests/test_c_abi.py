@@ -41,7 +41,7 @@ def test_c_program_links_and_runs(program):
     declared = set(re.findall(r"GEMM_API\s+[\w\s\*]+?\b(gemm_\w+)\s*\(", open(HEADER).read()))
     assert lines["entry_points"] == f"{len(declared)} missing 0"
     assert int(lines["abi"]) >= 10300
-    assert lines["path_cube"] == f"{ops.PATH_TILE_PAIR_TALL} path_decode {ops.PATH_SKINNY_EVEN}"
+    assert lines["path_cube"] == f"{ops.PATH_TILE_PAIR_TALL} path_decode {ops.PATH_SKINNY}"
     assert lines["plan"] == "rc 0 split 0 panels 8 extent 1024"
     smem, configs = lines["smem"].split(" configs ")
     assert 0 < int(smem) <= 232448 and int(configs) == len(ops.config_list())

@@ -42,8 +42,12 @@ def _ids(c):
 
 
 BUILT = ops.config_list()
-TILE_BUILT = [c for c in BUILT if c.kernel != ops.PATH_SKINNY]
+TILE_KERNELS = (ops.PATH_TILE, ops.PATH_TILE_PAIR, ops.PATH_TILE_PAIR_TALL)
+TILE_BUILT = [c for c in BUILT if c.kernel in TILE_KERNELS]
 SKINNY_BUILT = [c for c in BUILT if c.kernel == ops.PATH_SKINNY]
+# the even small-M schedule's configurations (their width is fixed by the
+# shape) are covered, depth by depth, in test_skinny_even_gpu.py
+assert all(c.kernel in TILE_KERNELS + (ops.PATH_SKINNY, ops.PATH_SKINNY_EVEN) for c in BUILT)
 
 
 @pytest.mark.parametrize("cfg", TILE_BUILT, ids=_ids)

@@ -373,16 +373,14 @@ double wave_efficiency(int64_t tiles, int64_t pairs) {
 // wave wastes more than 6 points more of the SM pairs than the 256-row
 // tiling's (the MLP up-projection with ReLU: 93 % against 97 %, still faster).
 //
-// Small M (<= 64): the even schedule when its busiest SM streams at least 10 %
-// fewer k-blocks of B than the small-M kernel's default tiling would (e.g. the
-// decode shape: 388 against 512), else the small-M kernel.
+// Small M (<= 64) takes the small-M kernel.  The even schedule
+// (GEMM_PATH_SKINNY_EVEN), which keeps every SM busy, streams B more slowly
+// than the 256-column tiling on the decode shape although it spreads the bytes
+// over 148 SMs instead of 112 (M = 32, N = 28672: 75.5 against 69.9 us at
+// K = 8192; 6.9 against 7.4 TB/s at the margin over K = 8192-16384), so AUTO
+// does not take it.
 int select_path_for(int64_t M, int64_t N, int64_t K, int sm_count, int activation) {
-  if (M >= 1 && M <= 64) {
-    const EvenPlan plan = even_plan(N, K, sm_count);
-    if (plan.q > 0 && 10 * plan.work <= 9 * skinny_default_work(N, K, sm_count))
-      return GEMM_PATH_SKINNY_EVEN;
-    return GEMM_PATH_SKINNY;
-  }
+  if (M >= 1 && M <= 64) return GEMM_PATH_SKINNY;
   const int64_t pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
   const int64_t col_tiles = (N + 255) / 256;
   const int64_t tiles256 = ((M + 255) / 256) * col_tiles;

@@ -445,16 +445,6 @@ int skinny_m_pad(int64_t M) {
   return 0;
 }
 
-int64_t skinny_default_work(int64_t N, int64_t K, int sm_count) {
-  const int64_t KB = (K + kBK - 1) / kBK;
-  const int tw = (N + 127) / 128 <= sm_count ? 128 : 256;
-  const int64_t tiles = (N + tw - 1) / tw;
-  const int S = choose_slices(tiles, KB, 32, tw, sm_count, sm_count);
-  const int64_t items = tiles * S;
-  const int64_t waves = (items + sm_count - 1) / sm_count;
-  return waves * (tw / 64) * ((KB + S - 1) / S);
-}
-
 size_t skinny_workspace_bytes(int sm_count, int m_pad) {
   // split-K happens only with fewer tiles than SMs, so at most sm_count
   // (tile, slice) items carry a partial tile

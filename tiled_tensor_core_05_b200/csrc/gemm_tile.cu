@@ -22,7 +22,6 @@
 // Out-of-range A/B elements (M, N or K not a multiple of the tile) are
 // zero-filled by TMA and so contribute nothing to the sum.
 #include <atomic>
-#include <cstdlib>
 
 #include "../../include/gemm_f16.h"
 #include "internal.h"
@@ -181,44 +180,6 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
   }
 }
 
-// Whether the (whole-tile) work unit `tile` is the first of the units running
-// together (the wave of `npairs` units that contains it) to read its A block
-// (bit 0) and its B block (bit 1) under the raster of tile_coords.  Only that
-// unit prefetches the block into L2, so the others find it there.
-__device__ __forceinline__ int first_reader(int tile, int num_m, int num_n, int group_m,
-                                            int npairs) {
-  const int wave_start = (tile / npairs) * npairs;
-  int own = 0;
-  if (group_m > 0) {
-    const int per_group = group_m * num_n;
-    const int g = tile / per_group;
-    const int rows = min(num_m - g * group_m, group_m);
-    const int r = tile - g * per_group;
-    if (r < rows || tile - rows < wave_start) own |= 1;  // first of its tile-row here
-    if (r % rows == 0 || tile - 1 < wave_start) own |= 2;  // first of its tile-column
-  } else {
-    const int group_n = -group_m;
-    const int per_group = group_n * num_m;
-    const int g = tile / per_group;
-    const int cols = min(num_n - g * group_n, group_n);
-    const int r = tile - g * per_group;
-    if (r < cols || tile - cols < wave_start) own |= 2;
-    if (r % cols == 0 || tile - 1 < wave_start) own |= 1;
-  }
-  return own;
-}
-
-// L2 eviction priority of the operand loads, one 2-bit field per operand
-// (bits 0-1 A, bits 2-3 B): 0 = no hint, 1 = evict-first, 2 = evict-normal,
-// 3 = evict-last.  The operand a raster panel re-reads across waves (A with
-// row panels, B with column panels) is the one worth keeping.
-enum : int { kHintNone = 0, kHintFirst = 1, kHintNormal = 2, kHintLast = 3 };
-__device__ __forceinline__ uint64_t l2_policy_for(int code) {
-  return code == kHintFirst ? l2_policy_evict_first()
-         : code == kHintLast ? l2_policy_evict_last()
-                             : l2_policy_evict_normal();
-}
-
 // The 64 bias values of the chunk at column col0 as 32 packed pairs (0 past
 // N): eight 16-byte loads (the same address in every lane) when the chunk
 // lies inside N, else pair by pair.
@@ -318,35 +279,12 @@ __device__ __forceinline__ void stage_chunk(const uint32_t* h, uint8_t* bufs, ui
 // stage_chunk.
 // `release()` runs once the last TMEM load of the tile has completed.
 // `bias` (N fp16 values or null) is added per column before the activation.
-// With COLS = 128, `early` set and no GELU, both chunks are read with one
-// 128-column load first, so the accumulator is handed back before any chunk
-// is converted or stored.
 template <int COLS, int BOXES, int ACT, class Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uint32_t& chunk_no,
                                               const CUtensorMap* tmC, __half* C, int64_t ldc,
                                               const __half* __restrict__ bias, int M, int N,
                                               int n8, int row0, int col_base, int lane,
-                                              Release release, bool early = false) {
-  // (not with GELU, whose arithmetic next to 128 live values exceeds the 168
-  // registers a thread of a 10-warp CTA may hold)
-  if constexpr (COLS == 128 && ACT != kActGelu) {
-    if (early) {
-      uint32_t v[128];
-      tmem_load_32x32b_x128(t_row, v);
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) release();
-      uint32_t h[64];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) convert_chunk<ACT>(v + 64 * c, bias, col_base + c * kEpiCols, N,
-                                                    h + 32 * c);
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-        stage_chunk<BOXES>(h + 32 * c, bufs, chunk_no, tmC, C, ldc, M, N, n8, row0,
-                           col_base + c * kEpiCols, lane);
-      return;
-    }
-  }
+                                              Release release) {
 #pragma unroll 1
   for (int c = 0; c < COLS / kEpiCols; ++c) {
     uint32_t v[64];
@@ -596,8 +534,8 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, __half* __restrict__ C,
                           int64_t ldc, const __half* __restrict__ bias, int M, int N, int K,
-                          int layout, int group_m, int split_from, int l2_hint, int epi_early,
-                          int pf_dist, int* status, uint64_t timeout_ns) {
+                          int layout, int group_m, int split_from, int* status,
+                          uint64_t timeout_ns) {
   using Cfg = PairCfg<STAGES, SLABS>;
   const bool ta = (layout & kLayoutTransA) != 0;
   const bool tb = (layout & kLayoutTransB) != 0;
@@ -679,20 +617,6 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
-      const int hint_a = l2_hint & 3, hint_b = (l2_hint >> 2) & 3;
-      const uint64_t pol_a = l2_policy_for(hint_a), pol_b = l2_policy_for(hint_b);
-      auto load_a = [&](uint32_t bar, void* dst, int c0, int c1) {
-        if (hint_a != kHintNone)
-          tma_load_2d_pair_hint(&tmA, bar, dst, c0, c1, pol_a);
-        else
-          tma_load_2d_pair(&tmA, bar, dst, c0, c1);
-      };
-      auto load_b = [&](uint32_t bar, void* dst, int c0, int c1) {
-        if (hint_b != kHintNone)
-          tma_load_2d_pair_hint(&tmB, bar, dst, c0, c1, pol_b);
-        else
-          tma_load_2d_pair(&tmB, bar, dst, c0, c1);
-      };
       for (int unit = pair; unit < num_units && ok; unit += npairs) {
         int mb, nb, row_base, slabs;
         unit_coords(unit, mb, nb, row_base, slabs);
@@ -712,54 +636,18 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
             uint8_t* adst = smA + stage * Cfg::kABytes + s * Cfg::kSlabBytes;
             const int row = a_row + s * 2 * kBM;
             if (!ta) {
-              load_a(bar, adst, kb * kBK, row);
+              tma_load_2d_pair(&tmA, bar, adst, kb * kBK, row);
             } else {
-              load_a(bar, adst, row, kb * kBK);
-              load_a(bar, adst + Cfg::kBChunk, row + 64, kb * kBK);
+              tma_load_2d_pair(&tmA, bar, adst, row, kb * kBK);
+              tma_load_2d_pair(&tmA, bar, adst + Cfg::kBChunk, row + 64, kb * kBK);
             }
           }
           uint8_t* bdst = smB + stage * Cfg::kBBytes;
           if (!tb) {
-            load_b(bar, bdst, b_col, kb * kBK);
-            load_b(bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
+            tma_load_2d_pair(&tmB, bar, bdst, b_col, kb * kBK);
+            tma_load_2d_pair(&tmB, bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
           } else {
-            load_b(bar, bdst, kb * kBK, b_col);
-          }
-          if (pf_dist > 0) {
-            // L2 prefetch of this CTA's part of k-block kb + pf_dist (of this
-            // unit, or of its next unit near the end), by the unit that reads
-            // the block first among those running together
-            int pu = unit, pk = kb + pf_dist;
-            if (pk >= num_kb) {
-              pu = unit + npairs;
-              pk -= num_kb;
-            }
-            if (pu < split_from && pk < num_kb) {
-              int pmb, pnb;
-              tile_coords(pu, num_m, num_n, group_m, pmb, pnb);
-              const int own = first_reader(pu, num_m, num_n, group_m, npairs);
-              if (own & 1) {
-                const int prow = pmb * Cfg::kTileM + static_cast<int>(rank) * kBM;
-#pragma unroll
-                for (int s = 0; s < SLABS; ++s) {
-                  if (!ta) {
-                    tma_prefetch_l2_2d(&tmA, pk * kBK, prow + s * 2 * kBM);
-                  } else {
-                    tma_prefetch_l2_2d(&tmA, prow + s * 2 * kBM, pk * kBK);
-                    tma_prefetch_l2_2d(&tmA, prow + s * 2 * kBM + 64, pk * kBK);
-                  }
-                }
-              }
-              if (own & 2) {
-                const int pcol = pnb * BN + static_cast<int>(rank) * 128;
-                if (!tb) {
-                  tma_prefetch_l2_2d(&tmB, pcol, pk * kBK);
-                  tma_prefetch_l2_2d(&tmB, pcol + 64, pk * kBK);
-                } else {
-                  tma_prefetch_l2_2d(&tmB, pk * kBK, pcol);
-                }
-              }
-            }
+            tma_load_2d_pair(&tmB, bar, bdst, kb * kBK, b_col);
           }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -943,7 +831,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
                                static_cast<uint32_t>((acc * SLABS + s) * BN + g * kCols);
         epilogue_tile<kCols, Cfg::kEpiBoxes, ACT>(
             t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0, nb * BN + g * kCols, lane,
-            [release_bar] { mbar_arrive_cluster(release_bar); }, epi_early != 0);
+            [release_bar] { mbar_arrive_cluster(release_bar); });
       }
       if (++acc == NBUF) {
         acc = 0;
@@ -1001,41 +889,6 @@ int group_tiles(int group, int tile_rows, int tile_cols) {
   }
   const int g = group / tile_rows;
   return g > 0 ? g : 1;
-}
-
-// Whether the 512-row pair tile's epilogue reads a warp's 128 columns with
-// one load and hands the accumulator back before converting them: TTC_EPI in
-// the environment (0 or 1), read once, else 0.
-int epi_early_code() {
-  static const int code = [] {
-    const char* s = std::getenv("TTC_EPI");
-    return (s != nullptr && s[0] == '1') ? 1 : 0;
-  }();
-  return code;
-}
-
-// L2 prefetch distance of the pair kernels in k-blocks (0 = none): TTC_PF in
-// the environment, read once.
-int prefetch_distance() {
-  static const int dist = [] {
-    const char* s = std::getenv("TTC_PF");
-    if (s == nullptr) return 0;
-    const int v = std::atoi(s);
-    return (v >= 0 && v <= 64) ? v : 0;
-  }();
-  return dist;
-}
-
-// The L2 hint code of the pair kernels' operand loads (see l2_policy_for):
-// TTC_L2HINT in the environment (a number 0-15), read once, else none.
-int l2_hint_code() {
-  static const int code = [] {
-    const char* s = std::getenv("TTC_L2HINT");
-    if (s == nullptr) return 0;
-    const int v = std::atoi(s);
-    return (v >= 0 && v <= 15) ? v : 0;
-  }();
-  return code;
 }
 
 template <int BN, int STAGES, int ACT>
@@ -1126,8 +979,7 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
       &cfg, kern, tA, tB, tC, static_cast<__half*>(p.C), p.ldc,
       static_cast<const __half*>(p.bias), static_cast<int>(p.M), static_cast<int>(p.N),
       static_cast<int>(p.K), p.layout, group_tiles(group_rows, Cfg::kTileM, Cfg::kBN),
-      static_cast<int>(split_from), l2_hint_code(), epi_early_code(), prefetch_distance(),
-      d.status, d.timeout_ns);
+      static_cast<int>(split_from), d.status, d.timeout_ns);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : GEMM_ERR_LAUNCH;
 }
 

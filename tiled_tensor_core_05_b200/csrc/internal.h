@@ -117,9 +117,6 @@ int launch_skinny_even(const GemmProblem& p, const DeviceCtx& d, void* workspace
                        size_t workspace_bytes, const KernelConfig& c);
 int even_config_smem_bytes(int block_n, int stages);  // -1 when block_n is not 64 q, q in 1..4
 int even_configs_built(KernelConfig* out, int cap);
-// The busiest CTA's k-blocks of 64 columns in the default configuration of
-// the small-M kernel (gemm_skinny.cu) for this shape, waves included.
-int64_t skinny_default_work(int64_t N, int64_t K, int sm_count);
 
 // The small-M kernel with its scratch in a fixed device array of the library
 // (no allocation); M <= 32.  Returns GEMM_ERR_SCRATCH_LIMIT beyond.
