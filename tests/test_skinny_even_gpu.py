@@ -96,7 +96,7 @@ def test_even_transposed_storage(oracle_mod, trans_a, trans_b):
 
 @pytest.mark.parametrize("stages", [4, 5, 6])
 def test_even_every_compiled_depth(oracle_mod, stages):
-    m, n, k = 32, cols(3, 4), 700
+    m, n, k = 32, cols(3, 4), 704  # 11 k-blocks; row strides multiples of 8
     a, b = workloads.make_inputs(m, n, k, seed=79, a_scale=1.0 / k ** 0.5)
     ref = oracle_mod.gemm_relu(a, b)
     c = ops.gemm_config_run(a.cuda(), b.cuda(), {"kernel": EVEN, "stages": stages}, None, "relu")

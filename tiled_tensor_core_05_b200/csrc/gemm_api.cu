@@ -296,9 +296,17 @@ int encode_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
   const cuuint64_t strides[1] = {ld * 2u};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estrides[2] = {1, 1};
+  static const CUtensorMapL2promotion promo = [] {
+    const char* s = std::getenv("TTC_PROMO");
+    const int v = s != nullptr ? std::atoi(s) : 3;
+    return v == 0 ? CU_TENSOR_MAP_L2_PROMOTION_NONE
+           : v == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_64B
+           : v == 2 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                    : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+  }();
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base),
                               dims, strides, box, estrides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_SWIZZLE_128B, promo,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_INVALID_ARG;
 }
