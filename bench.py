@@ -177,12 +177,14 @@ def parity_rows(M: int, max_rows: int) -> list:
 
 
 def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
-                     comparator=False, variant="relu", path=0, check_rows=0):
+                     comparator=False, variant="relu", path=0, check_rows=0, min_ms=0.0):
     """Time one workload.  variant: "relu" (gemm_relu_f16, the measured path),
     "bias_gelu" (gemm_bias_act_f16 with a per-column bias and GELU) or "wT"
     (gemm_f16_general with B stored N x K, ReLU).  With `check_rows` > 0 the
     result's rows (all, or that many spread over M) are kept for the oracle
-    check."""
+    check.  With `min_ms` > 0 (single-process context runs only) a timed
+    region shorter than that is timed again with enough launches to fill it,
+    so that short kernels are measured over many launches."""
     import torch
 
     from tiled_tensor_core_05_b200 import ops, workloads
@@ -222,6 +224,9 @@ def measure_workload(name, steps, warmup, dist=None, sampler=None, e2e=True,
             raise RuntimeError(f"{variant} call failed: {ops.status_string(rc)}")
 
     total_ms, launch_ms = time_launches(step, steps, warmup, stream, dist, sampler)
+    if dist is None and min_ms > 0 and total_ms < min_ms:
+        n = min(2000, int(min_ms / max(launch_ms, 1e-4)) + 1)
+        total_ms, launch_ms = time_launches(step, n, warmup, stream, None, None)
     st = ops.device_status()
     if st != 0:
         raise RuntimeError(f"device reported status {st:#x}")
@@ -677,7 +682,7 @@ def run_ours(args):
                 continue
             r = measure_workload(name, max(args.steps, 20), max(args.warmup, 3), None, None,
                                  e2e=False, comparator=not args.no_comparator, variant=variant,
-                                 check_rows=512 if check else 0)
+                                 check_rows=512 if check else 0, min_ms=20.0)
             r.pop("step")
             r.pop("tensors")
             others.append(r)

@@ -79,10 +79,10 @@ enum gemm_status {
 
 enum gemm_path {
   GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY; fewer than 64 tiles of
-                              256 x 256 -> TILE; K < 3072 (6144 with GELU) -> TILE_PAIR;
-                              otherwise TILE_PAIR_TALL, or TILE_PAIR when the 512-row
-                              tiles leave a much emptier last wave (SKINNY_EVEN only
-                              when asked for) */
+                              256 x 256 -> TILE; K < 6144 -> TILE_PAIR; otherwise
+                              TILE_PAIR_TALL, or TILE_PAIR when the 512-row tiles leave
+                              a much emptier last wave (SKINNY_EVEN only when asked
+                              for) */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile, BN = 64, 128 or
                               256 by the tile count (any shape) */
   GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 128 columns of B per CTA when
@@ -171,8 +171,9 @@ typedef struct gemm_config {
   int32_t group_rows; /* tile kernels: the L2 grouping of the tile order.  > 0: rows of
                          op(A) per row panel (tiles walked column by column inside
                          it); < 0: minus the columns of op(B) per column panel (tiles
-                         walked row by row inside it); 0 = the default.  Must be 0 for
-                         the small-M kernels */
+                         walked row by row inside it); 0 = the default (4096 for
+                         GEMM_PATH_TILE_PAIR, 2048 otherwise).  Must be 0 for the
+                         small-M kernels */
   int32_t splits;     /* GEMM_PATH_SKINNY: k-slices per column tile, 1 <= splits <=
                          ceil(K / 64) and splits * ceil(N / block_n) <= the SM count when
                          > 1; 0 = chosen from the shape.  Must be 0 for the tile kernels

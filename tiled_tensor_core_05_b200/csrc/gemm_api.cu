@@ -296,17 +296,11 @@ int encode_tmap_f16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
   const cuuint64_t strides[1] = {ld * 2u};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estrides[2] = {1, 1};
-  static const CUtensorMapL2promotion promo = [] {
-    const char* s = std::getenv("TTC_PROMO");
-    const int v = s != nullptr ? std::atoi(s) : 3;
-    return v == 0 ? CU_TENSOR_MAP_L2_PROMOTION_NONE
-           : v == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_64B
-           : v == 2 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
-                    : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
-  }();
+  // (L2 promotion none / 128 B / 256 B measured alike on the pair kernels:
+  // the same DRAM bytes and time)
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base),
                               dims, strides, box, estrides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, promo,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_INVALID_ARG;
 }
@@ -371,29 +365,24 @@ double wave_efficiency(int64_t tiles, int64_t pairs) {
 
 // The kernel chosen for a shape on a GPU with `sm_count` SMs.  The 512 x 256
 // pair tile stages 25 % fewer bytes per MAC than the 256 x 256 one, but its
-// single accumulator leaves each tile's epilogue exposed, which costs more
-// the shorter the main loop and the heavier the epilogue.  Measured on an
-// 8192 x 8192 output (time of the 512-row tile / time of the 256-row tile):
-//   K            3072   4096   5120   6144   8192
-//   ReLU + bias  1.002  0.995  0.981  0.964  0.943
-//   GELU + bias  1.054  1.024  1.015  0.993  0.966
-// So the 512-row tile is taken from K = 3072 (6144 with GELU) unless its last
+// single accumulator leaves part of each tile's epilogue exposed, which costs
+// more the shorter the main loop.  Measured (ReLU, 30-launch bursts and
+// 2-second runs under the power cap, the 256-row tile with 6 stages and
+// 4096-row panels, the 512-row tile with 2048-row panels):
+//   8192 x 8192 x 8192:   512-row tile 0.723 / 0.839 ms, 256-row 0.742 / 0.855
+//   8192 x 14336 x 4096:  512-row tile 0.647 / 0.746 ms, 256-row 0.633 / 0.732
+//   8192 x 8192 x K:      even at K = 6144, the 256-row tile ahead below
+// So the 512-row tile is taken from K = 6144 (any activation) unless its last
 // wave wastes more than 6 points more of the SM pairs than the 256-row
-// tiling's (the MLP up-projection with ReLU: 93 % against 97 %, still faster).
-//
-// Small M (<= 64) takes the small-M kernel.  The even schedule
-// (GEMM_PATH_SKINNY_EVEN), which keeps every SM busy, streams B more slowly
-// than the 256-column tiling on the decode shape although it spreads the bytes
-// over 148 SMs instead of 112 (M = 32, N = 28672: 75.5 against 69.9 us at
-// K = 8192; 6.9 against 7.4 TB/s at the margin over K = 8192-16384), so AUTO
-// does not take it.
+// tiling's.
 int select_path_for(int64_t M, int64_t N, int64_t K, int sm_count, int activation) {
   if (M >= 1 && M <= 64) return GEMM_PATH_SKINNY;
   const int64_t pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
   const int64_t col_tiles = (N + 255) / 256;
   const int64_t tiles256 = ((M + 255) / 256) * col_tiles;
   if (tiles256 < 64) return GEMM_PATH_TILE;
-  if (K < (activation == GEMM_ACT_GELU ? 6144 : 3072)) return GEMM_PATH_TILE_PAIR;
+  (void)activation;
+  if (K < 6144) return GEMM_PATH_TILE_PAIR;
   const int64_t tiles512 = ((M + 511) / 512) * col_tiles;
   return wave_efficiency(tiles512, pairs) >= wave_efficiency(tiles256, pairs) - 0.06
              ? GEMM_PATH_TILE_PAIR_TALL
@@ -456,7 +445,8 @@ int resolve_config(KernelConfig& c, int64_t M, int64_t N, int64_t K, int sm_coun
     if (c.group_rows != 0 || skinny_m_pad(M) == 0) return GEMM_ERR_CONFIG;
   } else {
     if (c.splits != 0) return GEMM_ERR_CONFIG;
-    if (c.group_rows == 0) c.group_rows = kDefaultGroupRows;
+    if (c.group_rows == 0)
+      c.group_rows = c.kernel == GEMM_PATH_TILE_PAIR ? kDefaultGroupRowsPair : kDefaultGroupRows;
   }
   return GEMM_OK;
 }

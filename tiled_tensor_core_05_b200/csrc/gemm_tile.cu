@@ -831,7 +831,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
                                static_cast<uint32_t>((acc * SLABS + s) * BN + g * kCols);
         epilogue_tile<kCols, Cfg::kEpiBoxes, ACT>(
             t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0, nb * BN + g * kCols, lane,
-            [release_bar] { mbar_arrive_cluster(release_bar); });
+            [release_bar] { mbar_arrive_cluster_relaxed(release_bar); });
       }
       if (++acc == NBUF) {
         acc = 0;
