@@ -276,8 +276,9 @@ __device__ __forceinline__ void stage_chunk(const uint32_t* h, uint8_t* bufs, ui
 
 // Epilogue of one accumulator tile, run by one warp for its 32 TMEM lanes and
 // COLS of the tile's columns, 64 at a time: tcgen05.ld -> convert_chunk ->
-// stage_chunk.
-// `release()` runs once the last TMEM load of the tile has completed.
+// stage_chunk, with each chunk staged only after the next chunk's TMEM load,
+// so that `release()` runs as soon as the last TMEM load of the tile has
+// completed (only the last chunk's conversion and two stagings follow it).
 // `bias` (N fp16 values or null) is added per column before the activation.
 template <int COLS, int BOXES, int ACT, class Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uint32_t& chunk_no,
@@ -285,21 +286,25 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
                                               const __half* __restrict__ bias, int M, int N,
                                               int n8, int row0, int col_base, int lane,
                                               Release release) {
+  constexpr int kChunks = COLS / kEpiCols;
+  uint32_t h[32];  // the previous chunk, converted, not yet staged
 #pragma unroll 1
-  for (int c = 0; c < COLS / kEpiCols; ++c) {
+  for (int c = 0; c < kChunks; ++c) {
     uint32_t v[64];
     tmem_load_32x32b_x64(t_row + c * kEpiCols, v);
-    if (c == COLS / kEpiCols - 1) {
+    if (c == kChunks - 1) {
       // the accumulator has been read: hand it back to the MMA issuer
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) release();
     }
-    uint32_t h[32];
+    if (c > 0)
+      stage_chunk<BOXES>(h, bufs, chunk_no, tmC, C, ldc, M, N, n8, row0,
+                         col_base + (c - 1) * kEpiCols, lane);
     convert_chunk<ACT>(v, bias, col_base + c * kEpiCols, N, h);
-    stage_chunk<BOXES>(h, bufs, chunk_no, tmC, C, ldc, M, N, n8, row0, col_base + c * kEpiCols,
-                       lane);
   }
+  stage_chunk<BOXES>(h, bufs, chunk_no, tmC, C, ldc, M, N, n8, row0,
+                     col_base + (kChunks - 1) * kEpiCols, lane);
 }
 
 template <int BN, int STAGES, int ACT>
