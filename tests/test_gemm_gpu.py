@@ -114,21 +114,19 @@ def test_tall_tile_last_wave_halves(oracle_mod, m, n, k):
 
 @pytest.mark.parametrize("m,n,k", [(8192, 14336, 256), (2000, 3000, 300), (4600, 2300, 520),
                                    (300, 1000, 130), (100, 200, 64)])
-def test_pair_tile_last_wave_column_halves(oracle_mod, m, n, k):
-    """The 256-row pair tile splits the tiles of a sparse last wave into two
-    128-column halves (pair MMAs of N = 128): whole tiles followed by halves
-    (1792 tiles on 74 pairs: 16 split; 96: 22 split, the last half 56 columns
-    wide), halves only (8 tiles, 1 tile), ragged rows and columns.  Compared
-    in full."""
+def test_pair_tile_sparse_last_wave(oracle_mod, m, n, k):
+    """The 256-row pair tile on shapes whose last wave holds few tiles (1792
+    tiles on 74 pairs, 96, 8, 1), with ragged rows and columns (the last
+    column tile of 3000 is 184 columns wide).  Compared in full."""
     a, b = workloads.make_inputs(m, n, k, seed=6000 + m + n + k)
     for relu in (True, False):
         ref = oracle_mod.gemm_relu(a, b) if relu else oracle_mod.gemm(a, b)
         check_parity(run(a, b, relu=relu, path=PAIR), ref, relu, f"pair {m}x{n}x{k}")
 
 
-def test_pair_tile_column_halves_transposed_b_and_gelu(oracle_mod):
-    """Column-half units with B stored N x K (one 128-row box per CTA, of
-    which the N = 128 MMAs read the first 64 rows) and with bias + GELU."""
+def test_pair_tile_transposed_b_and_gelu(oracle_mod):
+    """The 256-row pair tile with B stored N x K and bias + GELU on a ragged
+    shape (96 tiles, the last column tile 184 columns wide)."""
     m, n, k = 2000, 3000, 304  # row strides of A and of B stored N x K: multiples of 8
     a, b = workloads.make_inputs(m, n, k, seed=6100)
     bias = (np.random.default_rng(61).standard_normal(n) * 0.5).astype(np.float16)
@@ -136,7 +134,7 @@ def test_pair_tile_column_halves_transposed_b_and_gelu(oracle_mod):
     c = ops.gemm_general(a.cuda(), b.T.contiguous().cuda(), torch.from_numpy(bias).cuda(), "gelu",
                          trans_b=True, path=PAIR)
     torch.cuda.synchronize()
-    check_parity(dev_to_np(c), ref, False, "pair halves, B stored N x K, bias + GELU")
+    check_parity(dev_to_np(c), ref, False, "pair, B stored N x K, bias + GELU")
     assert ops.device_status() == 0
 
 

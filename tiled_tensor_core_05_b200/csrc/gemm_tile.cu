@@ -275,7 +275,7 @@ __device__ __forceinline__ void stage_chunk(const uint32_t* h, uint8_t* bufs, ui
 }
 
 // Epilogue of one accumulator tile, run by one warp for its 32 TMEM lanes and
-// `cols` (a multiple of 64, at most COLS) of the tile's columns, 64 at a time: tcgen05.ld -> convert_chunk ->
+// COLS of the tile's columns, 64 at a time: tcgen05.ld -> convert_chunk ->
 // stage_chunk, with each chunk staged only after the next chunk's TMEM load,
 // so that `release()` runs as soon as the last TMEM load of the tile has
 // completed (only the last chunk's conversion and two stagings follow it).
@@ -285,8 +285,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* bufs, uin
                                               const CUtensorMap* tmC, __half* C, int64_t ldc,
                                               const __half* __restrict__ bias, int M, int N,
                                               int n8, int row0, int col_base, int lane,
-                                              Release release, int cols = COLS) {
-  const int kChunks = cols / kEpiCols;  // 64-column chunks, at most COLS / 64
+                                              Release release) {
+  constexpr int kChunks = COLS / kEpiCols;
   uint32_t h[32];  // the previous chunk, converted, not yet staged
 #pragma unroll 1
   for (int c = 0; c < kChunks; ++c) {
@@ -572,30 +572,16 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
   const int num_kb = (K + kBK - 1) / kBK;
   const int n8 = N & ~7;
   // Work units: tiles [0, split_from) whole, then each tile from split_from
-  // on as two halves (the host splits the tiles of a last wave that holds at
-  // most half as many tiles as there are pairs, so that wave takes about half
-  // a tile's time; split_from == num_tiles otherwise): the 512-row tile in
-  // two 256-row slabs, the 256-row tile in two 128-column halves (pair MMAs
-  // of N = 128, 64 columns of B per CTA).
+  // on as two units of one 256-row slab (the host splits the tiles of a last
+  // wave that holds at most half as many tiles as there are pairs, so that
+  // wave takes about half a tile's time; split_from == num_tiles otherwise).
   const int num_units = 2 * num_tiles - split_from;
-  // unit -> tile coordinates, first row and column of the unit, its slab
-  // count and its column count
-  auto unit_coords = [&](int u, int& mb, int& nb, int& row_base, int& slabs, int& col_base,
-                         int& ncols) {
+  // unit -> tile coordinates, first row of the unit and its slab count
+  auto unit_coords = [&](int u, int& mb, int& nb, int& row_base, int& slabs) {
     const bool half = u >= split_from;
-    const int hi = half ? ((u - split_from) & 1) : 0;
     tile_coords(half ? split_from + (u - split_from) / 2 : u, num_m, num_n, group_m, mb, nb);
-    if constexpr (SLABS == 2) {
-      row_base = mb * Cfg::kTileM + hi * 2 * kBM;
-      slabs = half ? 1 : SLABS;
-      col_base = nb * BN;
-      ncols = BN;
-    } else {
-      row_base = mb * Cfg::kTileM;
-      slabs = 1;
-      col_base = nb * BN + hi * (BN / 2);
-      ncols = half ? BN / 2 : BN;
-    }
+    row_base = mb * Cfg::kTileM + (half ? ((u - split_from) & 1) * 2 * kBM : 0);
+    slabs = half ? 1 : SLABS;
   };
 
   if (threadIdx.x == 0) {
@@ -637,16 +623,11 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
       for (int unit = pair; unit < num_units && ok; unit += npairs) {
-        int mb, nb, row_base, slabs, col_base, ncols;
-        unit_coords(unit, mb, nb, row_base, slabs, col_base, ncols);
+        int mb, nb, row_base, slabs;
+        unit_coords(unit, mb, nb, row_base, slabs);
         const int a_row = row_base + static_cast<int>(rank) * kBM;  // slab 0
-        // this CTA's half of the unit's columns; row-major B moves 64-column
-        // boxes (one for a column-half unit), B stored N x K one box of 128
-        // rows (of which a column-half unit's MMAs read the first 64)
-        const int b_col = col_base + static_cast<int>(rank) * (ncols / 2);
-        const bool b_one_box = !tb && ncols < BN;
-        const uint32_t b_bytes = b_one_box ? Cfg::kBChunk : Cfg::kBBytes;
-        const uint32_t tx = 2u * static_cast<uint32_t>(slabs * Cfg::kSlabBytes + b_bytes);
+        const int b_col = nb * BN + static_cast<int>(rank) * 128;
+        const uint32_t tx = 2u * static_cast<uint32_t>(slabs * Cfg::kSlabBytes + Cfg::kBBytes);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             ok = false;
@@ -669,8 +650,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
           uint8_t* bdst = smB + stage * Cfg::kBBytes;
           if (!tb) {
             tma_load_2d_pair(&tmB, bar, bdst, b_col, kb * kBK);
-            if (!b_one_box)
-              tma_load_2d_pair(&tmB, bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
+            tma_load_2d_pair(&tmB, bar, bdst + Cfg::kBChunk, b_col + 64, kb * kBK);
           } else {
             tma_load_2d_pair(&tmB, bar, bdst, kb * kBK, b_col);
           }
@@ -705,9 +685,7 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       uint32_t slab1_phase = 0;
       bool ok = true;
       int site = 0;
-      const uint32_t idesc_full = idesc_f16_f32(2 * kBM, BN, ta, !tb);
-      const uint32_t idesc_half_n = idesc_f16_f32(2 * kBM, BN / 2, ta, !tb);
-      uint32_t idesc = idesc_full;
+      const uint32_t idesc = idesc_f16_f32(2 * kBM, BN, ta, !tb);
       // The MMAs of k-block `kb` (held in ring stage `st`) for slabs
       // [s_begin, s_end) into the accumulator at `d_tmem`.
       auto issue = [&](uint32_t d_tmem, int st, int kb, int s_begin, int s_end) {
@@ -796,8 +774,6 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
             break;
           }
           tc_fence_after_sync();
-          // a column-half unit: pair MMAs of N = 128 into the first 128 columns
-          idesc = unit < split_from ? idesc_full : idesc_half_n;
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * SLABS * BN);
           for (int kb = 0; kb < num_kb; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag, timeout_ns)) {
@@ -838,9 +814,8 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
     uint32_t acc_phase = 0;
     uint32_t chunk_no = 0;
     for (int unit = pair; unit < num_units; unit += npairs) {
-      int mb, nb, row_base, slabs, col_base, ncols;
-      unit_coords(unit, mb, nb, row_base, slabs, col_base, ncols);
-      const int cols_w = ncols * 4 / Cfg::kEpiWarps;  // this warp's columns of the unit
+      int mb, nb, row_base, slabs;
+      unit_coords(unit, mb, nb, row_base, slabs);
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, timeout_ns) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -860,8 +835,8 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                static_cast<uint32_t>((acc * SLABS + s) * BN + g * kCols);
         epilogue_tile<kCols, Cfg::kEpiBoxes, ACT>(
-            t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0, col_base + g * cols_w,
-            lane, [release_bar] { mbar_arrive_cluster_relaxed(release_bar); }, cols_w);
+            t_row, bufs, chunk_no, &tmC, C, ldc, bias, M, N, n8, row0, nb * BN + g * kCols, lane,
+            [release_bar] { mbar_arrive_cluster_relaxed(release_bar); });
       }
       if (++acc == NBUF) {
         acc = 0;
@@ -994,10 +969,10 @@ int launch_pair_impl(const GemmProblem& p, const DeviceCtx& d, int group_rows) {
     max_pairs[d.device & 63].store(n, std::memory_order_relaxed);
   }
   const int64_t num_tiles = ((p.M + Cfg::kTileM - 1) / Cfg::kTileM) * ((p.N + 255) / 256);
-  // a last wave of at most resident / 2 tiles runs as twice as many halves
-  // (256-row slabs of the 512-row tile, 128-column halves of the 256-row one)
+  // with the 512-row tile, a last wave of at most resident / 2 tiles runs as
+  // twice as many 256-row halves
   int64_t split_from = num_tiles;
-  {
+  if constexpr (SLABS == 2) {
     const int64_t rem = num_tiles % resident;
     if (rem != 0 && 2 * rem <= resident) split_from = num_tiles - rem;
   }
