@@ -255,7 +255,9 @@ __device__ __forceinline__ void stage_chunk(const uint32_t* h, uint8_t* bufs, ui
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    if (row0 < M && col0 < n8) tma_store_2d(tmC, buf, col0, row0);
+    // C is written once and not read again here: evict-first keeps the
+    // operand tiles that later tiles re-read in L2 (0.1-0.7 % faster)
+    if (row0 < M && col0 < n8) tma_store_2d_hint(tmC, buf, col0, row0, l2_policy_evict_first());
     bulk_commit_group();
   }
   if (n8 < N && col0 + kEpiCols > n8 && col0 < N && row0 + lane < M) {
