@@ -171,9 +171,9 @@ typedef struct gemm_config {
   int32_t group_rows; /* tile kernels: the L2 grouping of the tile order.  > 0: rows of
                          op(A) per row panel (tiles walked column by column inside
                          it); < 0: minus the columns of op(B) per column panel (tiles
-                         walked row by row inside it); 0 = the default (4096 for
-                         GEMM_PATH_TILE_PAIR, 2048 otherwise).  Must be 0 for the
-                         small-M kernels */
+                         walked row by row inside it); odd panels are walked in
+                         reverse; 0 = the default (4096 for the pair kernels, 2048
+                         for GEMM_PATH_TILE).  Must be 0 for the small-M kernels */
   int32_t splits;     /* GEMM_PATH_SKINNY: k-slices per column tile, 1 <= splits <=
                          ceil(K / 64) and splits * ceil(N / block_n) <= the SM count when
                          > 1; 0 = chosen from the shape.  Must be 0 for the tile kernels

@@ -61,12 +61,13 @@ def test_path_selection(lib):
     assert ops.select_path(65, 100, 100) == ops.PATH_TILE
     assert ops.select_path(1024, 1024, 1024) == ops.PATH_TILE
     assert ops.select_path(8192, 8192, 8192) == ops.PATH_TILE_PAIR_TALL
-    # below K = 6144 the double-buffered 256-row tile (its epilogue hidden) wins
-    assert ops.select_path(8192, 14336, 4096) == ops.PATH_TILE_PAIR
-    assert ops.select_path(5120, 5120, 4096) == ops.PATH_TILE_PAIR
+    # with ReLU the 512-row tile from K = 4096; below, the double-buffered
+    # 256-row tile (its epilogue hidden) wins
+    assert ops.select_path(8192, 14336, 4096) == ops.PATH_TILE_PAIR_TALL
+    assert ops.select_path(5120, 5120, 4096) == ops.PATH_TILE_PAIR_TALL
     assert ops.select_path(8192, 8192, 3072) == ops.PATH_TILE_PAIR
-    assert ops.select_path(8192, 8192, 6143) == ops.PATH_TILE_PAIR
-    assert ops.select_path(8192, 8192, 6144) == ops.PATH_TILE_PAIR_TALL
+    assert ops.select_path(8192, 8192, 4095) == ops.PATH_TILE_PAIR
+    assert ops.select_path(8192, 8192, 4096) == ops.PATH_TILE_PAIR_TALL
     # 20 x 20 tiles of 256: 400 / 74 = 5.4 waves (90 %); 10 x 20 of 512: 2.7 (90 %)
     assert ops.select_path(5120, 5120, 8192) == ops.PATH_TILE_PAIR_TALL
     # 9 x 9 = 81 tiles (55 % of two waves) against 5 x 9 = 45 (61 % of one)

@@ -86,6 +86,22 @@ def test_raster_panels(oracle_mod, kernel, group_rows):
     check_parity(c, ref, True, f"{cfg}")
 
 
+@pytest.mark.parametrize("kernel,m,n", [(ops.PATH_TILE_PAIR_TALL, 6556, 3278),
+                                         (ops.PATH_TILE_PAIR, 4000, 3000)])
+@pytest.mark.parametrize("group_rows", [0, 1024, -768])
+def test_waves_sweep_k_both_ways(oracle_mod, kernel, m, n, group_rows):
+    """Enough tiles for two to three waves of pairs, so that every pair also
+    runs units whose k-blocks are loaded from the top down (starting on the
+    partial last k-block of K = 200), in panels walked alternately forwards
+    and backwards (an odd panel count, the last one partial)."""
+    k = 200
+    a, b = workloads.make_inputs(m, n, k, seed=47)
+    ref = oracle_mod.gemm_relu(a.numpy(), b.numpy())
+    cfg = {"kernel": kernel, "group_rows": group_rows}
+    c = _run(a, b, cfg, m=m, n=n)
+    check_parity(c, ref, True, f"{cfg} {m}x{n}x{k}")
+
+
 @pytest.mark.parametrize("cfg", SKINNY_BUILT, ids=_ids)
 @pytest.mark.parametrize("m", [1, 20, 33, 64])
 def test_skinny_configs(oracle_mod, cfg, m):
@@ -119,6 +135,17 @@ def test_skinny_splits_are_deterministic_and_agree():
     for s, o in outs.items():
         assert np.allclose(o.astype(np.float32), outs[1].astype(np.float32), rtol=2e-3,
                            atol=2e-3), s
+
+
+def test_auto_tile_by_activation():
+    """With GELU (the longest epilogue) AUTO keeps the double-buffered 256-row
+    pair tile up to K = 6144; with ReLU or none it takes the 512-row tile from
+    K = 4096."""
+    assert ops.auto_config(8192, 14336, 4096, "gelu").kernel == ops.PATH_TILE_PAIR
+    assert ops.auto_config(8192, 14336, 6144, "gelu").kernel == ops.PATH_TILE_PAIR_TALL
+    for act in ("relu", "none"):
+        assert ops.auto_config(8192, 14336, 4096, act).kernel == ops.PATH_TILE_PAIR_TALL
+        assert ops.auto_config(8192, 14336, 4095, act).kernel == ops.PATH_TILE_PAIR
 
 
 @pytest.mark.parametrize("m,n,k,act", [(8192, 1024, 512, "relu"), (1000, 1000, 1000, "relu"),

@@ -366,23 +366,22 @@ double wave_efficiency(int64_t tiles, int64_t pairs) {
 // The kernel chosen for a shape on a GPU with `sm_count` SMs.  The 512 x 256
 // pair tile stages 25 % fewer bytes per MAC than the 256 x 256 one, but its
 // single accumulator leaves part of each tile's epilogue exposed, which costs
-// more the shorter the main loop.  Measured (ReLU, 30-launch bursts and
-// 2-second runs under the power cap, the 256-row tile with 6 stages and
-// 4096-row panels, the 512-row tile with 2048-row panels):
-//   8192 x 8192 x 8192:   512-row tile 0.723 / 0.839 ms, 256-row 0.742 / 0.855
-//   8192 x 14336 x 4096:  512-row tile 0.647 / 0.746 ms, 256-row 0.633 / 0.732
-//   8192 x 8192 x K:      even at K = 6144, the 256-row tile ahead below
-// So the 512-row tile is taken from K = 6144 (any activation) unless its last
-// wave wastes more than 6 points more of the SM pairs than the 256-row
-// tiling's.
+// more the shorter the main loop and the longer the epilogue.  Measured
+// (30-launch bursts and 2-second runs under the power cap, both tiles with
+// 4096-row panels, the 256-row tile with 6 stages, waves sweeping K both ways):
+//   8192 x 8192 x 8192, ReLU:    512-row tile 0.723 / 0.832 ms, 256-row 0.771 / 0.886
+//   8192 x 14336 x 4096, ReLU:   512-row tile 0.643 / 0.750 ms, 256-row 0.649 / 0.766
+//   8192 x 14336 x 4096, GELU:   512-row tile 0.695 / 0.806 ms, 256-row 0.682 / 0.798
+// So the 512-row tile is taken from K = 4096 with ReLU or no activation and
+// from K = 6144 with GELU (its epilogue is the longest), unless its last wave
+// wastes more than 6 points more of the SM pairs than the 256-row tiling's.
 int select_path_for(int64_t M, int64_t N, int64_t K, int sm_count, int activation) {
   if (M >= 1 && M <= 64) return GEMM_PATH_SKINNY;
   const int64_t pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
   const int64_t col_tiles = (N + 255) / 256;
   const int64_t tiles256 = ((M + 255) / 256) * col_tiles;
   if (tiles256 < 64) return GEMM_PATH_TILE;
-  (void)activation;
-  if (K < 6144) return GEMM_PATH_TILE_PAIR;
+  if (K < (activation == GEMM_ACT_GELU ? 6144 : 4096)) return GEMM_PATH_TILE_PAIR;
   const int64_t tiles512 = ((M + 511) / 512) * col_tiles;
   return wave_efficiency(tiles512, pairs) >= wave_efficiency(tiles256, pairs) - 0.06
              ? GEMM_PATH_TILE_PAIR_TALL
@@ -446,7 +445,7 @@ int resolve_config(KernelConfig& c, int64_t M, int64_t N, int64_t K, int sm_coun
   } else {
     if (c.splits != 0) return GEMM_ERR_CONFIG;
     if (c.group_rows == 0)
-      c.group_rows = c.kernel == GEMM_PATH_TILE_PAIR ? kDefaultGroupRowsPair : kDefaultGroupRows;
+      c.group_rows = c.kernel == GEMM_PATH_TILE ? kDefaultGroupRows : kDefaultGroupRowsPair;
   }
   return GEMM_OK;
 }

@@ -155,9 +155,11 @@ static_assert(variants_complete(), "built tile configurations != those within th
 
 // Grouped-panel rasterisation: consecutive tile indices sweep group_m
 // tile-rows of one panel column by column, so the CTAs that run at the same
-// time share A rows and B columns in L2.  A negative group_m gives panels of
-// -group_m tile-columns swept row by row instead (the same with the roles of
-// A and B exchanged).
+// time share A rows and B columns in L2.  Odd panels sweep their columns in
+// reverse (a snake), so the first tiles of a panel reuse the B columns the
+// previous panel read last.  A negative group_m gives panels of -group_m
+// tile-columns swept row by row instead (the same with the roles of A and B
+// exchanged).
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m,
                                             int& mb, int& nb) {
   if (group_m > 0) {
@@ -168,6 +170,7 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
     const int r = tile - g * per_group;
     mb = first_m + r % rows;
     nb = r / rows;
+    if (g & 1) nb = num_n - 1 - nb;
   } else {
     const int group_n = -group_m;
     const int per_group = group_n * num_m;
@@ -177,6 +180,7 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
     const int r = tile - g * per_group;
     nb = first_n + r % cols;
     mb = r / cols;
+    if (g & 1) mb = num_m - 1 - mb;
   }
 }
 
@@ -624,13 +628,21 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
-      for (int unit = pair; unit < num_units && ok; unit += npairs) {
+      // The pairs run their j-th units at about the same time (a wave); odd
+      // waves sweep K from the top down, so a wave starts on the k-blocks the
+      // previous wave read last -- still in L2 -- instead of the ones it read
+      // first, which it evicted long ago.  The MMA issuer consumes the stages
+      // in ring order either way; only its first k-block (not k-block 0)
+      // starts the accumulation.
+      uint32_t down = 0;
+      for (int unit = pair; unit < num_units && ok; unit += npairs, down ^= 1u) {
         int mb, nb, row_base, slabs;
         unit_coords(unit, mb, nb, row_base, slabs);
         const int a_row = row_base + static_cast<int>(rank) * kBM;  // slab 0
         const int b_col = nb * BN + static_cast<int>(rank) * 128;
         const uint32_t tx = 2u * static_cast<uint32_t>(slabs * Cfg::kSlabBytes + Cfg::kBBytes);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int i = 0; i < num_kb; ++i) {
+          const int kb = down ? num_kb - 1 - i : i;  // the k-block this stage holds
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             ok = false;
             break;
@@ -688,7 +700,8 @@ __global__ void __launch_bounds__(PairCfg<STAGES, SLABS>::kThreads, 1)
       bool ok = true;
       int site = 0;
       const uint32_t idesc = idesc_f16_f32(2 * kBM, BN, ta, !tb);
-      // The MMAs of k-block `kb` (held in ring stage `st`) for slabs
+      // The MMAs of the unit's kb-th k-block in load order (held in ring
+      // stage `st`; the first one starts the accumulation) for slabs
       // [s_begin, s_end) into the accumulator at `d_tmem`.
       auto issue = [&](uint32_t d_tmem, int st, int kb, int s_begin, int s_end) {
         const uint32_t a_addr = smem_u32(smA + st * Cfg::kABytes);
