@@ -79,10 +79,10 @@ enum gemm_status {
 
 enum gemm_path {
   GEMM_PATH_AUTO = 0,      /* choose by shape: M <= 64 -> SKINNY; fewer than 64 tiles of
-                              256 x 256 -> TILE; K < 6144 -> TILE_PAIR; otherwise
-                              TILE_PAIR_TALL, or TILE_PAIR when the 512-row tiles leave
-                              a much emptier last wave (SKINNY_EVEN only when asked
-                              for) */
+                              256 x 256 -> TILE; K < 4096 (K < 6144 with GELU) ->
+                              TILE_PAIR; otherwise TILE_PAIR_TALL, or TILE_PAIR when
+                              the 512-row tiles leave a much emptier last wave
+                              (SKINNY_EVEN only when asked for) */
   GEMM_PATH_TILE = 1,      /* persistent kernel, one SM per 128 x BN tile, BN = 64, 128 or
                               256 by the tile count (any shape) */
   GEMM_PATH_SKINNY = 2,    /* small-M kernel: swap-AB, 128 columns of B per CTA when
@@ -215,7 +215,7 @@ GEMM_API int gemm_auto_config(int64_t M, int64_t N, int64_t K, int activation, g
 /* The path GEMM_PATH_AUTO takes for this shape with ReLU (or no activation)
  * on a 148-SM B200 (pure host function; GEMM_PATH_AUTO itself uses the SM
  * count of the current device, and with GELU keeps the 256-row pair tile up
- * to K < 6144). */
+ * to K < 6144, where ReLU switches to the 512-row tile from K = 4096). */
 GEMM_API int gemm_select_path(int64_t M, int64_t N, int64_t K);
 
 /* Human-readable text for a gemm_status value (static storage). */
