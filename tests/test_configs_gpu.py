@@ -102,6 +102,20 @@ def test_waves_sweep_k_both_ways(oracle_mod, kernel, m, n, group_rows):
     check_parity(c, ref, True, f"{cfg} {m}x{n}x{k}")
 
 
+@pytest.mark.parametrize("kernel", [ops.PATH_TILE_PAIR_TALL, ops.PATH_TILE_PAIR])
+def test_waves_both_ways_transposed_bias_gelu(oracle_mod, kernel):
+    """The same two-way K sweeps with both operands stored transposed (K x M
+    and N x K) and the bias + GELU epilogue, over two to three waves."""
+    m, n, k = 4000, 3000, 328
+    a, b = workloads.make_inputs(m, n, k, seed=48)
+    rng = np.random.default_rng(48)
+    bias = rng.standard_normal(n).astype(np.float16)
+    ref = oracle_mod.gemm_general(a, b, bias, "gelu")
+    c = _run(a.T.contiguous(), b.T.contiguous(), {"kernel": kernel}, bias, "gelu", True, True,
+             m=m, n=n)
+    check_parity(c, ref, False, f"kernel {kernel} transposed bias + gelu {m}x{n}x{k}")
+
+
 @pytest.mark.parametrize("cfg", SKINNY_BUILT, ids=_ids)
 @pytest.mark.parametrize("m", [1, 20, 33, 64])
 def test_skinny_configs(oracle_mod, cfg, m):
