@@ -36,6 +36,45 @@ __device__ __forceinline__ void store_column(const float (&v)[MP], __half* C, in
   }
 }
 
+// Column `col` of a staged MP x TW fp16 tile of C (row-major, TW columns per
+// row) from this thread's MP fp32 sums: bias of column n, activation, RNE.
+// Columns at or past N are left unwritten (never copied out).
+template <int MP, int ACT>
+__device__ __forceinline__ void stage_column(const float (&v)[MP], __half* tile, int tw, int col,
+                                             int N, int n, const __half* bias) {
+  if (n >= N) return;
+  const float b = bias != nullptr ? __half2float(bias[n]) : 0.0f;
+#pragma unroll
+  for (int m = 0; m < MP; m += 2) {
+    const float2 x = activate2<ACT>(__fadd2_rn(make_float2(v[m], v[m + 1]), splat2(b)));
+    tile[m * tw + col] = __float2half_rn(x.x);
+    tile[(m + 1) * tw + col] = __float2half_rn(x.y);
+  }
+}
+
+// Copies the staged tile's rows m < M, columns n0 .. min(N, n0 + TW) - 1, to
+// C with 16-byte stores (`nthreads` threads, this one `tid`); a piece that
+// crosses N is stored element by element.
+template <int MP, int TW>
+__device__ __forceinline__ void store_staged_rows(const __half* tile, __half* C, int M, int N,
+                                                  int64_t ldc, int n0, int tid, int nthreads) {
+  constexpr int kPieces = TW / 8;  // 16-byte pieces per row
+  const int rows = M < MP ? M : MP;
+  for (int i = tid; i < rows * kPieces; i += nthreads) {
+    const int m = i / kPieces;
+    const int j = i - m * kPieces;
+    const int n = n0 + 8 * j;
+    if (n >= N) continue;
+    const __half* src = tile + m * TW + 8 * j;
+    __half* dst = C + static_cast<int64_t>(m) * ldc + n;
+    if (n + 8 <= N) {
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+    } else {
+      for (int e = 0; n + e < N; ++e) dst[e] = src[e];
+    }
+  }
+}
+
 // Rows m0 .. m0 + R - 1 (those < M) of column n of C from R fp32 sums, as
 // store_column does for all MP rows.
 template <int R, int ACT>
