@@ -374,6 +374,11 @@ __global__ void __launch_bounds__(TileCfg<BN, STAGES>::kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // The coordinates of this CTA's first tile (three integer divisions, about
+  // 0.3 us at the start of a small launch) are worked out before the wait, so
+  // they overlap the previous kernel of the stream.
+  int first_mb = 0, first_nb = 0;
+  tile_coords(blockIdx.x, num_m, num_n, group_m, first_mb, first_nb);
   // the set-up above overlaps the previous kernel of the stream; inputs and
   // outputs are touched only after it has finished
   grid_dependency_trigger();
@@ -386,8 +391,8 @@ __global__ void __launch_bounds__(TileCfg<BN, STAGES>::kThreads, 1)
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, num_m, num_n, group_m, mb, nb);
+        int mb = first_mb, nb = first_nb;
+        if (tile != static_cast<int>(blockIdx.x)) tile_coords(tile, num_m, num_n, group_m, mb, nb);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, timeout_ns)) {
             ok = false;
@@ -488,8 +493,8 @@ __global__ void __launch_bounds__(TileCfg<BN, STAGES>::kThreads, 1)
     uint32_t acc_phase = 0;
     uint32_t chunk_no = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      int mb, nb;
-      tile_coords(tile, num_m, num_n, group_m, mb, nb);
+      int mb = first_mb, nb = first_nb;
+      if (tile != static_cast<int>(blockIdx.x)) tile_coords(tile, num_m, num_n, group_m, mb, nb);
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, timeout_ns) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
